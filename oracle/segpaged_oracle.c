@@ -1,0 +1,152 @@
+/*
+ * CPU oracle for head-aware paged attention (SegPagedAttention).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark load this file's library.  It shares no code,
+ * header, table or constant with the CUDA path.
+ *
+ * What it computes is the plain definition the method must reproduce: dense
+ * attention over the full causal context with an explicit per-head visibility
+ * mask, accumulated in fp64.  The method's claim is that evaluating each head
+ * over only the tokens it stores gives this same result ("SegPagedAttention
+ * runtime design", §4: verify_against_dense compares against a dense + mask
+ * baseline and asks for cosine > 0.99998).
+ *
+ * Head kinds ("SegPagedAttention runtime design", §1 and §3; "RedKnot head
+ * classification", the four-kind table):
+ *   GLOBAL reads the whole causal prefix; DENSE reads the whole prefix as well
+ *   (its RoPE re-alignment belongs to KV reuse, not to attention);
+ *   LOCAL reads only the first `sink` tokens of the sequence and the `window`
+ *   most recent tokens.
+ * Readings where the pages are silent: the recent window counts the query's
+ * own position (positions p-window+1 .. p); sinks are absolute positions
+ * 0 .. sink-1 of the sequence; an overlap of sink and window is a plain union.
+ *
+ * Parity pins: O1 is checked in the tests against a brute-force enumeration of
+ * the visible set, against ordinary causal attention for GLOBAL heads, and
+ * against closed forms (window 1, equal keys).  See tests/test_oracle_pins.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Kind codes of this file only: 0 global, 1 local, 2 dense. */
+#define ORACLE_GLOBAL 0
+#define ORACLE_LOCAL 1
+#define ORACLE_DENSE 2
+
+/* Does query position p see key position j?  Causal for every kind; a local
+ * head additionally needs j among the first `sink` positions or among the
+ * `window` most recent positions ending at p. */
+static int oracle_sees(int kind, int64_t sink, int64_t window, int64_t p, int64_t j) {
+  if (j > p) return 0;
+  if (kind != ORACLE_LOCAL) return 1;
+  return (j < sink) || (j >= p - window + 1);
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/*
+ * Attention of n_rows query rows of one (sequence, query-head) against the
+ * dense K/V of its kv-head.
+ *   q    [n_rows][d]   fp64, post-RoPE queries
+ *   pos  [n_rows]      absolute position p of each query row
+ *   k, v [L][d]        dense keys / values of the kv-head, positions 0 .. L-1
+ *   out  [n_rows][d]   O = sum_j e_j v_j / sum_j e_j over visible j
+ *   lse  [n_rows]      m + ln sum_j e_j,  e_j = exp(s_j - m), m = max_j s_j
+ * Scores are s_j = scale * <q, k_j>.  Returns 0, or -1 if a row sees nothing
+ * or a position lies outside [0, L).
+ */
+int oracle_attention_rows(int64_t n_rows, int64_t d, const double* q, const int64_t* pos,
+                          int64_t L, const double* k, const double* v, int kind,
+                          int64_t sink, int64_t window, double scale, double* out,
+                          double* lse) {
+  int bad = 0;
+#pragma omp parallel
+  {
+    double* s = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    char* vis = (char*)malloc((size_t)(L > 0 ? L : 1));
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_rows; ++r) {
+      const int64_t p = pos[r];
+      const double* qr = q + r * d;
+      double* o = out + r * d;
+      if (p < 0 || p >= L) {
+#pragma omp atomic write
+        bad = 1;
+        continue;
+      }
+      double m = -INFINITY;
+      int64_t nvis = 0;
+      for (int64_t j = 0; j < L; ++j) {
+        vis[j] = (char)oracle_sees(kind, sink, window, p, j);
+        if (!vis[j]) continue;
+        double acc = 0.0;
+        for (int64_t t = 0; t < d; ++t) acc += qr[t] * k[j * d + t];
+        s[j] = scale * acc;
+        if (s[j] > m) m = s[j];
+        ++nvis;
+      }
+      if (nvis == 0) {
+#pragma omp atomic write
+        bad = 1;
+        continue;
+      }
+      double denom = 0.0;
+      for (int64_t t = 0; t < d; ++t) o[t] = 0.0;
+      for (int64_t j = 0; j < L; ++j) {
+        if (!vis[j]) continue;
+        const double e = exp(s[j] - m);
+        denom += e;
+        for (int64_t t = 0; t < d; ++t) o[t] += e * v[j * d + t];
+      }
+      for (int64_t t = 0; t < d; ++t) o[t] /= denom;
+      lse[r] = m + log(denom);
+    }
+    free(s);
+    free(vis);
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * Which positions of a (sequence, kv-head) the cache must keep so that every
+ * query of a call with queries at positions q0 .. L-1 finds its visible keys:
+ * the union of the queries' visible sets ("SegPagedAttention runtime design",
+ * §3: build_segpaged_cache keeps only the tokens a local head can see).
+ * mask[j] = 1 if position j is kept.  Returns the number kept.
+ */
+int64_t oracle_stored_mask(int kind, int64_t sink, int64_t window, int64_t L, int64_t q0,
+                           uint8_t* mask) {
+  int64_t n = 0;
+  for (int64_t j = 0; j < L; ++j) {
+    uint8_t keep = 0;
+    for (int64_t p = q0; p < L && !keep; ++p) keep = (uint8_t)oracle_sees(kind, sink, window, p, j);
+    mask[j] = keep;
+    n += keep;
+  }
+  return n;
+}
+
+/*
+ * Number of (query, key) pairs a call evaluates: sum over query positions
+ * q0 .. L-1 of the size of the visible set.  Used for the visible-FLOP ledger
+ * (4 * d FLOPs per pair: QK^T and PV, a multiply and an add each).
+ */
+int64_t oracle_visible_pairs(int kind, int64_t sink, int64_t window, int64_t L, int64_t q0) {
+  int64_t n = 0;
+  for (int64_t p = q0; p < L; ++p)
+    for (int64_t j = 0; j <= p; ++j) n += oracle_sees(kind, sink, window, p, j);
+  return n;
+}

@@ -1,0 +1,49 @@
+"""Plant plausible mistakes in the oracle and check that its pins catch each one.
+
+Each mutant is a copy of the oracle's C source with one textual change,
+compiled into a temporary directory; the pin suite is then run against it in a
+subprocess and must fail.  The committed oracle is never modified.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parent.parent
+SRC = ROOT / "oracle" / "segpaged_oracle.c"
+
+MUTANTS = {
+    "window_one_too_wide": ("(j >= p - window + 1)", "(j >= p - window)"),
+    "window_excludes_query": ("(j >= p - window + 1)", "(j >= p - window + 2)"),
+    "sink_one_too_wide": ("(j < sink)", "(j <= sink)"),
+    "sink_dropped": ("(j < sink) ||", "0 ||"),
+    "not_causal": ("if (j > p) return 0;", ""),
+    "scale_dropped": ("s[j] = scale * acc;", "s[j] = acc;"),
+    "values_from_keys": ("o[t] += e * v[j * d + t];", "o[t] += e * k[j * d + t];"),
+    "transposed_key_index": ("acc += qr[t] * k[j * d + t];", "acc += qr[t] * k[t * d + j % d];"),
+    "lse_without_max": ("lse[r] = m + log(denom);", "lse[r] = log(denom);"),
+    "dense_treated_as_local": ("if (kind != ORACLE_LOCAL) return 1;", "if (kind == ORACLE_GLOBAL) return 1;"),
+    "stored_only_last_query": ("for (int64_t p = q0; p < L && !keep; ++p)", "for (int64_t p = L - 1; p < L && !keep; ++p)"),
+}
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = SRC.read_text()
+    assert src.count(old) == 1, f"mutation site for {name} not unique"
+    mut = tmp_path / "mutant.c"
+    mut.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", str(mut), "-o", str(lib), "-lm"],
+                   check=True)
+    env = dict(os.environ, SEGPAGED_ORACLE_LIB=str(lib), OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        str(ROOT / "tests" / "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stdout[-2000:]}"

@@ -1,0 +1,238 @@
+"""Pins of the CPU oracle against facts fixed outside it (no GPU needed).
+
+Each pin is chosen so that a plausible mistake in the oracle (an off-by-one
+window, sinks counted from the chunk, a dropped scale, a transposed operand,
+a wrong GQA map) fails at least one of them; ``test_oracle_mutants.py`` plants
+such mistakes and checks that they are caught.
+"""
+from __future__ import annotations
+
+import math
+from pathlib import Path
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import brute
+from head_aware_paged_build_b200 import workloads as W
+
+GOLDEN = Path(__file__).parent / "golden"
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+def _read_golden(name):
+    kv = {}
+    for line in (GOLDEN / name).read_text().splitlines():
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        k, v = (x.strip() for x in line.split("=", 1))
+        kv[k] = v
+    return kv
+
+
+# (kind, sink, window) grid covering window 1, window < sink, overlap, s = 0, w >= L
+POLICIES = [("global", 0, 0), ("dense", 0, 0), ("local", 0, 1), ("local", 0, 2), ("local", 1, 1),
+            ("local", 4, 8), ("local", 3, 100), ("local", 8, 3), ("local", 2, 5)]
+
+
+@pytest.mark.parametrize("kind,sink,window", POLICIES)
+@pytest.mark.parametrize("L,q0,d", [(1, 0, 4), (9, 0, 8), (23, 11, 8), (40, 39, 16)])
+def test_oracle_matches_brute_force(kind, sink, window, L, q0, d):
+    rng = np.random.default_rng(1000 * L + 10 * d + sink + 7 * window)
+    q, k, v = _rand(rng, L - q0, d), _rand(rng, L, d), _rand(rng, L, d)
+    scale = 1.0 / math.sqrt(d)
+    pos = np.arange(q0, L)
+    out, lse = oracle.attention_rows(q, pos, k, v, kind, sink, window)
+    for i, p in enumerate(pos):
+        bo, bl = brute.attention_row(q[i].tolist(), k.tolist(), v.tolist(), kind, sink, window, int(p), scale)
+        np.testing.assert_allclose(out[i], bo, rtol=0, atol=1e-12)
+        assert abs(lse[i] - bl) <= 1e-12
+
+
+def test_global_head_is_causal_attention():
+    """GLOBAL = ordinary causal attention (library SDPA, fp64 CPU, bottom-right mask)."""
+    rng = np.random.default_rng(5)
+    L, C, d = 70, 30, 32
+    q, k, v = _rand(rng, C, d), _rand(rng, L, d), _rand(rng, L, d)
+    pos = np.arange(L - C, L)
+    out, _ = oracle.attention_rows(q, pos, k, v, "global", 0, 0)
+    mask = torch.from_numpy(np.arange(L)[None, :] <= pos[:, None])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(k)[None], torch.from_numpy(v)[None], attn_mask=mask[None])
+    np.testing.assert_allclose(out, ref[0].numpy(), rtol=0, atol=1e-12)
+
+
+def test_local_head_is_sdpa_with_sink_window_mask():
+    """LOCAL = SDPA with the sink-plus-window mask written from the text as sets."""
+    rng = np.random.default_rng(6)
+    L, C, d, s, w = 90, 50, 16, 3, 17
+    q, k, v = _rand(rng, C, d), _rand(rng, L, d), _rand(rng, L, d)
+    pos = np.arange(L - C, L)
+    mask = np.zeros((C, L), bool)
+    for i, p in enumerate(pos):
+        mask[i, brute.visible_positions("local", s, w, int(p))] = True
+    out, _ = oracle.attention_rows(q, pos, k, v, "local", s, w)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(k)[None], torch.from_numpy(v)[None],
+        attn_mask=torch.from_numpy(mask)[None])
+    np.testing.assert_allclose(out, ref[0].numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("sink", [0, 4])
+def test_local_with_window_covering_context_equals_global(sink):
+    rng = np.random.default_rng(7)
+    L, d = 50, 8
+    q, k, v = _rand(rng, L, d), _rand(rng, L, d), _rand(rng, L, d)
+    pos = np.arange(L)
+    og, lg = oracle.attention_rows(q, pos, k, v, "global", 0, 0)
+    ol, ll = oracle.attention_rows(q, pos, k, v, "local", sink, L)
+    assert np.array_equal(og, ol) and np.array_equal(lg, ll)
+
+
+def test_window_one_returns_own_value():
+    """sink 0, window 1: each query sees only itself, so O = V[p] and LSE = s_pp."""
+    rng = np.random.default_rng(8)
+    L, d = 33, 8
+    q, k, v = _rand(rng, L, d), _rand(rng, L, d), _rand(rng, L, d)
+    pos = np.arange(L)
+    out, lse = oracle.attention_rows(q, pos, k, v, "local", 0, 1)
+    assert np.array_equal(out, v)
+    np.testing.assert_allclose(lse, (q * k).sum(1) / math.sqrt(d), rtol=0, atol=1e-13)
+
+
+def test_window_two_with_equal_keys_averages_last_two_values():
+    rng = np.random.default_rng(9)
+    L, d = 20, 8
+    q, v = _rand(rng, L, d), _rand(rng, L, d)
+    k = np.tile(_rand(rng, 1, d), (L, 1))
+    pos = np.arange(1, L)
+    out, _ = oracle.attention_rows(q[1:], pos, k, v, "local", 0, 2)
+    np.testing.assert_allclose(out, (v[:-1] + v[1:]) / 2, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("sink,window", [(4, 8), (0, 5), (6, 1), (3, 3)])
+def test_equal_keys_average_visible_values_and_count(sink, window):
+    """All keys equal: O is the mean of the visible values, |V(p)| = min(p+1, s+w)."""
+    rng = np.random.default_rng(10 + sink)
+    L, d = 40, 4
+    q = _rand(rng, L, d)
+    k = np.tile(_rand(rng, 1, d), (L, 1))
+    v = np.zeros((L, d))
+    v[:, 0] = 1.0                       # column 0 counts the visible rows via LSE
+    v[:, 1] = np.arange(L, dtype=float)  # column 1 gives the mean visible position
+    v[:, 2:] = _rand(rng, L, d - 2)
+    pos = np.arange(L)
+    out, lse = oracle.attention_rows(q, pos, k, v, "local", sink, window)
+    for i, p in enumerate(pos):
+        n_vis = min(p + 1, sink + window)
+        s = float(q[i] @ k[0]) / 2.0
+        assert abs(lse[i] - (s + math.log(n_vis))) <= 1e-12
+        vis = [j for j in range(p + 1) if j < sink or j > p - window]
+        assert len(vis) == n_vis
+        np.testing.assert_allclose(out[i, 1], np.mean(vis), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(out[i, 2:], v[vis, 2:].mean(0), rtol=0, atol=1e-12)
+
+
+def test_gqa_equals_mha_with_repeated_kv_heads():
+    """Query head h uses kv-head h // g: repeating each kv-head g times gives the same result."""
+    rng = np.random.default_rng(11)
+    L, d, hkv, g = 24, 8, 2, 3
+    q = _rand(rng, hkv * g, L, d)
+    k, v = _rand(rng, hkv, L, d), _rand(rng, hkv, L, d)
+    pol = [("global", 0, 0), ("local", 2, 5)]
+    pos = np.arange(L)
+    for h in range(hkv * g):
+        kv = h // g
+        a, _ = oracle.attention_rows(q[h], pos, k[kv], v[kv], *pol[kv])
+        k_rep, v_rep = np.repeat(k, g, 0), np.repeat(v, g, 0)
+        b, _ = oracle.attention_rows(q[h], pos, k_rep[h], v_rep[h], *pol[h // g])
+        assert np.array_equal(a, b)
+
+
+def test_scale_override_and_positions_outside_context_rejected():
+    rng = np.random.default_rng(12)
+    L, d = 10, 4
+    q, k, v = _rand(rng, 1, d), _rand(rng, L, d), _rand(rng, L, d)
+    out, lse = oracle.attention_rows(q, [9], k, v, "global", 0, 0, scale=0.0)
+    np.testing.assert_allclose(out[0], v.mean(0), atol=1e-15)
+    assert abs(lse[0] - math.log(L)) < 1e-14
+    with pytest.raises(ValueError):
+        oracle.attention_rows(q, [10], k, v, "global", 0, 0)
+
+
+@pytest.mark.parametrize("kind,sink,window", POLICIES)
+@pytest.mark.parametrize("L,q0", [(1, 0), (17, 16), (30, 0), (64, 40), (5, 3)])
+def test_stored_mask_matches_brute_union(kind, sink, window, L, q0):
+    m = oracle.stored_mask(kind, sink, window, L, q0)
+    keep = brute.stored_positions(kind, sink, window, L, q0)
+    assert set(np.flatnonzero(m).tolist()) == keep
+    pairs = oracle.visible_pairs(kind, sink, window, L, q0)
+    assert pairs == sum(len(brute.visible_positions(kind, sink, window, p)) for p in range(q0, L))
+
+
+def test_stored_counts_closed_forms_at_decode():
+    """Decode keeps L tokens for a global head and min(L, s + w) for a local head."""
+    for L in (1, 3, 4, 5, 100, 517, 516, 515, 2000):
+        assert oracle.stored_mask("global", 0, 0, L, L - 1).sum() == L
+        assert oracle.stored_mask("local", 4, 512, L, L - 1).sum() == min(L, 516)
+        m = oracle.stored_mask("local", 4, 512, L, L - 1)
+        assert m[: min(4, L)].all() and m[max(0, L - 512):].all()
+
+
+def test_stored_counts_of_the_synthetic_layers():
+    """Closed-form stored token-heads: global L, local min(L, s + w + C - 1) (chunk of C queries)."""
+    def closed(wl, prob):
+        n = 0
+        for b in range(wl.batch):
+            L, q0 = prob.ctx_lens[b], prob.q_starts[b]
+            for kv in range(wl.num_kv_heads):
+                kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+                n += L if kind != "local" else min(L, s + w + (L - q0) - 1)
+        return n
+
+    expect = {"tiny": (293, 512), "mistral": (77920, 127048), "llama": (721120, 950440)}
+    for name, (dec, pre) in expect.items():
+        wl = W.ALL[name]()
+        assert closed(wl, wl.decode_problem()) == dec
+        assert closed(wl, wl.prefill_problem()) == pre
+    # brute-force union on the tiny layer agrees with the closed form
+    wl = W.tiny()
+    for prob, want in ((wl.decode_problem(), 293), (wl.prefill_problem(), 512)):
+        got = sum(oracle.stored_mask(*wl.policy[kv], prob.ctx_lens[0], prob.q_starts[0]).sum()
+                  for kv in range(2))
+        assert got == want
+    assert closed(W.mha(), W.mha().decode_problem()) == 4 * (8 * 131072 + 56 * 132)
+
+
+def test_visible_flops_of_tiny_prefill():
+    """Visible pairs of the tiny prefill: 2 q-heads x (global 256*257/2 + local sum_p min(p+1, 36))."""
+    wl = W.tiny()
+    glob = 256 * 257 // 2
+    loc = sum(min(p + 1, 36) for p in range(256))
+    got = 2 * (oracle.visible_pairs("global", 0, 0, 256, 0) + oracle.visible_pairs("local", 4, 32, 256, 0))
+    assert got == 2 * (glob + loc)
+    assert 4 * wl.head_dim * got == 21_238_784  # 2.12e7 visible FLOPs
+
+
+def test_golden_deepseek_policy_savings():
+    """The page's DeepSeek-V4-Flash policy: 56 of 64 heads local (87.5%), window 128, sink 4."""
+    g = _read_golden("deepseek_v4_flash_policy.txt")
+    n = int(g["heads_per_layer"])
+    glob = {int(x) for x in g["global_head_ids"].split(",")}
+    s, w = int(g["local_sink"]), int(g["local_window"])
+    assert glob == set(range(0, n, 8))
+    frac_local = (n - len(glob)) / n
+    assert frac_local == float(g["local_head_fraction_middle"])
+    for L in (65536, 131072, 262144):
+        stored = sum(int(oracle.stored_mask("global" if h in glob else "local", s, w, L, L - 1).sum())
+                     for h in range(n))
+        saving = 1 - stored / (n * L)
+        assert saving == pytest.approx(frac_local * (1 - (s + w) / L), abs=1e-12)
+        assert float(g["kv_saving_low"]) <= saving <= float(g["kv_saving_high"])
+    assert int(g["default_window"]) == 512 and int(g["default_sink"]) == 4
