@@ -1,0 +1,177 @@
+// Device entry points of libsegpaged.so (the C ABI of segpaged.h).
+//
+// Each call validates its arguments on the host, before any launch, then
+// enqueues kernels on the caller's stream.  There is no host or library
+// fallback: a dtype / shape without a kernel returns SP_ERR_UNSUPPORTED.
+#include <cmath>
+#include <cstdint>
+#include <string>
+
+#include "kernels.h"
+#include "sp_internal.h"
+
+namespace sp {
+cudaError_t launch_prefill_f32(const PrefillLaunch& a, cudaStream_t s);
+cudaError_t launch_prefill_bf16(const PrefillLaunch& a, cudaStream_t s);
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+template <typename T>
+const T* section(const void* d_table, int64_t off) {
+  return reinterpret_cast<const T*>(static_cast<const uint8_t*>(d_table) + off);
+}
+
+sp_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SP_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+sp_status check_table(const sp_plan* plan, const void* d_table) {
+  if (!plan) return fail(SP_ERR_INVALID_ARG, "plan is NULL");
+  if (!d_table || !aligned(d_table, 16)) return fail(SP_ERR_INVALID_ARG, "d_table must be a 16-byte aligned device pointer");
+  return SP_OK;
+}
+
+sp_status pack_common(const sp_plan* plan, const void* d_table, const void* k_in, const void* v_in, void* k_out,
+                      void* v_out, bool inverse, int64_t stride_seq, int64_t stride_head, int64_t stride_tok,
+                      void* stream) {
+  sp_status st = check_table(plan, d_table);
+  if (st != SP_OK) return st;
+  if (!k_in || !v_in || !k_out || !v_out) return fail(SP_ERR_INVALID_ARG, "K/V pointers must be non-NULL");
+  if (!aligned(k_in, 16) || !aligned(v_in, 16) || !aligned(k_out, 16) || !aligned(v_out, 16))
+    return fail(SP_ERR_INVALID_ARG, "K/V pointers must be 16-byte aligned");
+  const int64_t eb = plan->elem_bytes;
+  if (stride_head < 0 || stride_tok < 0 || (stride_seq < 0 && stride_seq != SP_VARLEN))
+    return fail(SP_ERR_INVALID_ARG, "strides must be >= 0 (stride_seq may be SP_VARLEN)");
+  if ((stride_head * eb) % 16 || (stride_tok * eb) % 16 || (stride_seq > 0 && (stride_seq * eb) % 16))
+    return fail(SP_ERR_INVALID_ARG, "strides must give 16-byte aligned rows");
+  PackLaunch L{};
+  L.heads = section<HeadDesc>(d_table, plan->hdr.off_heads);
+  L.pages = section<PageDesc>(d_table, plan->hdr.off_pages);
+  L.n_pages = plan->hdr.n_vpages;
+  L.D = plan->prob.head_dim;
+  L.P = plan->prob.page_size;
+  L.bf16 = plan->prob.dtype == SP_BF16;
+  L.inverse = inverse;
+  L.stride_seq = stride_seq;
+  L.stride_head = stride_head;
+  L.stride_tok = stride_tok;
+  L.page_bytes = plan->sizes.page_bytes;
+  if (inverse) {
+    L.kpool_in = k_in, L.vpool_in = v_in, L.kdense_out = k_out, L.vdense_out = v_out;
+  } else {
+    L.kdense_in = k_in, L.vdense_in = v_in, L.kpool_out = k_out, L.vpool_out = v_out;
+  }
+  launch_pack(L, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SP_OK : cuda_fail(e, inverse ? "segpaged_gather launch" : "build_segpaged_cache launch");
+}
+
+}  // namespace
+}  // namespace sp
+
+extern "C" {
+
+sp_status segpaged_table_write(const sp_plan* plan, void* d_table, size_t bytes, void* stream) {
+  if (!plan) return sp::fail(SP_ERR_INVALID_ARG, "plan is NULL");
+  if (!d_table || !sp::aligned(d_table, 16)) return sp::fail(SP_ERR_INVALID_ARG, "d_table must be 16-byte aligned");
+  if (bytes < plan->blob.size()) return sp::fail(SP_ERR_WORKSPACE, "table buffer smaller than table_bytes");
+  const cudaError_t e = cudaMemcpyAsync(d_table, plan->blob.data(), plan->blob.size(), cudaMemcpyHostToDevice,
+                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SP_OK : sp::cuda_fail(e, "segpaged_table_write");
+}
+
+sp_status build_segpaged_cache(const sp_plan* plan, const void* d_table, const void* k_dense, const void* v_dense,
+                               int64_t stride_seq, int64_t stride_head, int64_t stride_tok, void* k_pool,
+                               void* v_pool, void* stream) {
+  return sp::pack_common(plan, d_table, k_dense, v_dense, k_pool, v_pool, false, stride_seq, stride_head,
+                         stride_tok, stream);
+}
+
+sp_status segpaged_gather(const sp_plan* plan, const void* d_table, const void* k_pool, const void* v_pool,
+                          void* k_out, void* v_out, int64_t stride_seq, int64_t stride_head, int64_t stride_tok,
+                          void* stream) {
+  return sp::pack_common(plan, d_table, k_pool, v_pool, k_out, v_out, true, stride_seq, stride_head, stride_tok,
+                         stream);
+}
+
+sp_status segpaged_attention(const sp_plan* plan, const void* d_table, const void* k_pool, const void* v_pool,
+                             const void* q, void* out, float* lse, float softmax_scale, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  using namespace sp;
+  sp_status st = check_table(plan, d_table);
+  if (st != SP_OK) return st;
+  if (!k_pool || !v_pool || !q || !out) return fail(SP_ERR_INVALID_ARG, "pool, q and out must be non-NULL");
+  if (!aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(q, 16) || !aligned(out, 16))
+    return fail(SP_ERR_INVALID_ARG, "pools, q and out must be 16-byte aligned");
+  if (lse && !aligned(lse, 4)) return fail(SP_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  if (!workspace || !aligned(workspace, 256)) return fail(SP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (int64_t(workspace_bytes) < plan->sizes.workspace_bytes)
+    return fail(SP_ERR_WORKSPACE, "workspace smaller than workspace_bytes");
+  if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale))
+    return fail(SP_ERR_INVALID_ARG, "softmax_scale must be finite");
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(plan->prob.head_dim));
+  const float scale_log2 = scale * 1.4426950408889634f;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* status = static_cast<int32_t*>(workspace);
+  cudaError_t e;
+  if (plan->sizes.is_decode) {
+    DecodeLaunch L{};
+    L.heads = section<HeadDesc>(d_table, plan->hdr.off_heads);
+    L.pages = section<PageDesc>(d_table, plan->hdr.off_pages);
+    L.items = section<DecodeItem>(d_table, plan->hdr.off_decode_items);
+    L.cta_begin = section<int32_t>(d_table, plan->hdr.off_decode_cta);
+    L.combine = section<CombineItem>(d_table, plan->hdr.off_combine);
+    L.n_ctas = plan->hdr.n_decode_ctas;
+    L.n_combine = plan->hdr.n_combine;
+    L.D = plan->prob.head_dim;
+    L.P = plan->prob.page_size;
+    L.group = plan->group;
+    L.num_q_heads = plan->prob.num_q_heads;
+    L.bf16 = plan->prob.dtype == SP_BF16;
+    L.page_bytes = plan->sizes.page_bytes;
+    L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
+    L.scale_log2 = scale_log2;
+    L.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
+    L.status = status;
+    e = launch_decode(L, s);
+  } else {
+    PrefillLaunch L{};
+    L.heads = section<HeadDesc>(d_table, plan->hdr.off_heads);
+    L.pages = section<PageDesc>(d_table, plan->hdr.off_pages);
+    L.items = section<PrefillItem>(d_table, plan->hdr.off_prefill);
+    L.n_items = plan->hdr.n_prefill_items;
+    L.D = plan->prob.head_dim;
+    L.P = plan->prob.page_size;
+    L.group = plan->group;
+    L.num_q_heads = plan->prob.num_q_heads;
+    L.total_rows = int32_t(plan->sizes.num_queries);
+    L.bf16 = plan->prob.dtype == SP_BF16;
+    L.page_bytes = plan->sizes.page_bytes;
+    L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
+    L.scale_log2 = scale_log2;
+    L.status = status;
+    e = L.bf16 ? launch_prefill_bf16(L, s) : launch_prefill_f32(L, s);
+    if (e == cudaErrorNotSupported) return fail(SP_ERR_UNSUPPORTED, "no prefill kernel for this configuration");
+  }
+  return e == cudaSuccess ? SP_OK : cuda_fail(e, "segpaged_attention launch");
+}
+
+sp_status segpaged_read_device_status(const void* workspace, int32_t* code, void* stream) {
+  if (!workspace || !code) return sp::fail(SP_ERR_INVALID_ARG, "workspace and code must be non-NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return sp::cuda_fail(e, "segpaged_read_device_status sync");
+  e = cudaMemcpy(code, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return sp::cuda_fail(e, "segpaged_read_device_status copy");
+  if (*code != 0) return sp::fail(SP_ERR_DEVICE_CHECK, "device status code " + std::to_string(*code));
+  return SP_OK;
+}
+
+sp_status segpaged_clear_device_status(void* workspace, void* stream) {
+  if (!workspace) return sp::fail(SP_ERR_INVALID_ARG, "workspace must be non-NULL");
+  const cudaError_t e = cudaMemsetAsync(workspace, 0, sp::kStatusBytes, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SP_OK : sp::cuda_fail(e, "segpaged_clear_device_status");
+}
+
+}  // extern "C"

@@ -1,0 +1,148 @@
+// Device-side helpers of libsegpaged.so: pool page layouts, mbarriers, bulk
+// copies, warp-level MMA and the status word.  All inline PTX here is written
+// from the PTX ISA (sm_90 / sm_100a instructions).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sp_internal.h"
+
+namespace sp {
+
+// --------------------------------------------------------------------------
+// Pool page layouts.
+//
+// bf16 (page size 64): a K page is the tcgen05 "K-major, 128-byte swizzle"
+// operand layout of a [P tokens x D dims] tile: D/64 column blocks of
+// [P rows x 128 B]; within a row the 16-byte chunk c is stored at c ^ (row & 7).
+// A V page is stored transposed, [D rows x P tokens] with the same swizzle, so
+// that it is the K-major operand of O += P V.  Both are exactly what the
+// tensor cores and ldmatrix read, so a page moves with one plain bulk copy.
+// fp32: K page row-major [P][D], V page transposed [D][P], no swizzle.
+// --------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t kpage_chunk_offset_bf16(int t, int c16, int P) {
+  // c16: 16-byte chunk index inside the token's D*2-byte row
+  return int64_t(c16 >> 3) * (P * 128) + t * 128 + (((c16 & 7) ^ (t & 7)) << 4);
+}
+__host__ __device__ __forceinline__ int64_t vpage_chunk_offset_bf16(int i, int c16) {
+  // row i (dimension), chunk c16 holds tokens 8*c16 .. 8*c16+7 (P = 64)
+  return int64_t(i) * 128 + ((c16 ^ (i & 7)) << 4);
+}
+
+// --------------------------------------------------------------------------
+// Status word (workspace word 0).  The first error sticks.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void record_error(int32_t* status, int32_t code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// --------------------------------------------------------------------------
+// mbarrier
+// --------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                   smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait: ~2 s of wall time, then give up (returns false).  The fast
+// path is one try_wait; the slow path re-checks the clock every 256 tries.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 0) {
+      if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+      __nanosleep(64);
+    }
+  }
+}
+
+// --------------------------------------------------------------------------
+// Bulk (non-tensor) asynchronous copy global -> shared, completing on an mbarrier.
+// Both addresses 16-byte aligned, size a multiple of 16.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// --------------------------------------------------------------------------
+// Warp-level MMA (decode).  m16n8k16, bf16 inputs, fp32 accumulate.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 2^x on the SFU (ex2.approx, flush-to-zero); 2^-inf = 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Visibility of key position `a` for query position `p` of a head:
+// causal, and for a local head inside the sink or the recent window.
+__device__ __forceinline__ bool sees(int local, int sink, int window, int p, int a) {
+  return a <= p && (!local || a < sink || a > p - window);
+}
+
+}  // namespace sp

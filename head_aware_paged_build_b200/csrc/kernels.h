@@ -1,0 +1,68 @@
+// Launch descriptors of the CUDA kernels of libsegpaged.so (host <-> .cu glue).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "sp_internal.h"
+
+namespace sp {
+
+struct PackLaunch {
+  const HeadDesc* heads;
+  const PageDesc* pages;
+  int32_t n_pages;
+  int32_t D, P;
+  bool bf16;
+  bool inverse;  // gather (pool -> dense) instead of pack
+  int64_t stride_seq, stride_head, stride_tok, page_bytes;
+  const void* kdense_in;
+  const void* vdense_in;
+  void* kpool_out;
+  void* vpool_out;
+  const void* kpool_in;
+  const void* vpool_in;
+  void* kdense_out;
+  void* vdense_out;
+};
+void launch_pack(const PackLaunch& L, cudaStream_t s);
+
+struct DecodeLaunch {
+  const HeadDesc* heads;
+  const PageDesc* pages;
+  const DecodeItem* items;
+  const int32_t* cta_begin;
+  const CombineItem* combine;
+  int32_t n_ctas, n_combine;
+  int32_t D, P, group, num_q_heads;
+  bool bf16;
+  int64_t page_bytes;
+  const void* kpool;
+  const void* vpool;
+  const void* q;  // [B, Hq, D]
+  void* out;      // [B, Hq, D]
+  float* lse;     // [B, Hq] or null
+  float scale_log2;  // softmax scale * log2(e)
+  float* partial;    // workspace partial slots
+  int32_t* status;
+};
+cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t s);
+
+struct PrefillLaunch {
+  const HeadDesc* heads;
+  const PageDesc* pages;
+  const PrefillItem* items;
+  int32_t n_items;
+  int32_t D, P, group, num_q_heads, total_rows;
+  bool bf16;
+  int64_t page_bytes;
+  const void* kpool;
+  const void* vpool;
+  const void* q;  // [rows, Hq, D]
+  void* out;
+  float* lse;
+  float scale_log2;
+  int32_t* status;
+};
+cudaError_t launch_prefill(const PrefillLaunch& L, cudaStream_t s);
+
+}  // namespace sp

@@ -1,0 +1,416 @@
+// Decode: split-KV attention over each head's own page list, then a combine
+// pass for heads split across CTAs ("SegPagedAttention runtime design", §4:
+// each head is evaluated at its true KV length, straight from its pages).
+//
+// bf16: one CTA = 4 consumer warps + 1 producer warp.  The producer streams
+// the CTA's pages (a balanced range of the concatenated page lists) into a
+// ring of shared-memory stages with 1-D bulk copies (one per K page and one
+// per V page: pages are stored in the swizzled layout the consumers read).
+// Each consumer warp takes 16 of a page's 64 tokens: S = Q K^T and O += P V
+// run on mma.sync m16n8k16 with the GQA group's q-heads as the 16 rows, and
+// the online softmax runs on the accumulator fragments with quad shuffles.
+// At the end of a head's range the 4 warps' states merge through shared
+// memory in a fixed order, so results are bitwise reproducible.
+//
+// fp32: a plain SIMT kernel over the same work list (FP32 FMA only).
+#include <cmath>
+
+#include "device_common.cuh"
+#include "kernels.h"
+
+namespace sp {
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D, int NST>
+struct DecodeSmem {
+  static constexpr int kPageBytes = 64 * D * 2;
+  static constexpr int kMergePitch = D + 8;  // floats per merge row (breaks bank aliasing)
+  static constexpr int kStageOff = 0;
+  static constexpr int kMergeOff = NST * 2 * kPageBytes;
+  static constexpr int kMlOff = kMergeOff + kConsumerWarps * kMaxGroup * kMergePitch * 4;
+  static constexpr int kBarOff = kMlOff + kConsumerWarps * kMaxGroup * 2 * 4;
+  static constexpr int kBytes = kBarOff + 2 * NST * 8;
+};
+
+template <int D, int NST>
+__global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunch a) {
+  using S = DecodeSmem<D, NST>;
+  constexpr int P = 64;
+  constexpr int PB = S::kPageBytes;
+  constexpr int KSTEPS = D / 16;
+  constexpr int NT = D / 8;  // n-tiles of the output
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* stage = smem + S::kStageOff;
+  float* mbuf = reinterpret_cast<float*>(smem + S::kMergeOff);
+  float* mlbuf = reinterpret_cast<float*>(smem + S::kMlOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  uint64_t* empty = full + NST;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ib = a.cta_begin[blockIdx.x], ie = a.cta_begin[blockIdx.x + 1];
+  if (ib >= ie) return;
+  const int gb = a.items[ib].vp_begin, ge = a.items[ie - 1].vp_end;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const uint8_t* kpool = static_cast<const uint8_t*>(a.kpool);
+  const uint8_t* vpool = static_cast<const uint8_t*>(a.vpool);
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      for (int g = gb, k = 0; g < ge; ++g, ++k) {
+        const int s = k % NST;
+        if (k >= NST && !mbar_wait(&empty[s], ((k / NST) & 1) ^ 1)) {
+          record_error(a.status, kDevTimeoutEmpty);
+          break;
+        }
+        const int64_t phys = a.pages[g].phys;
+        uint8_t* kd = stage + s * 2 * PB;
+        mbar_arrive_expect_tx(&full[s], 2 * PB);
+        bulk_g2s(kd, kpool + phys * a.page_bytes, PB, &full[s]);
+        bulk_g2s(kd + PB, vpool + phys * a.page_bytes, PB, &full[s]);
+      }
+      // Do not leave while copies into this CTA's shared memory are in flight.
+      const int n = ge - gb;
+      for (int k = (n > NST ? n - NST : 0); k < n; ++k)
+        if (!mbar_wait(&full[k % NST], (k / NST) & 1)) break;
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int grp = lane >> 2, tq = lane & 3;  // fragment row group, thread in quad
+  const int r0 = grp, r1 = grp + 8;
+  const int G = a.group;
+  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
+  bool ok = true;
+  int k = 0;
+  for (int it = ib; it < ie; ++it) {
+    const DecodeItem item = a.items[it];
+    const HeadDesc hd = a.heads[item.head];
+    const int qh0 = hd.kv * G;
+    const __nv_bfloat16* qrow = qg + (int64_t(hd.q_row0) * a.num_q_heads + qh0) * D;
+    uint32_t qa[KSTEPS][4];
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      const int c0 = kk * 16 + tq * 2;
+      qa[kk][0] = r0 < G ? *reinterpret_cast<const uint32_t*>(qrow + r0 * D + c0) : 0u;
+      qa[kk][1] = r1 < G ? *reinterpret_cast<const uint32_t*>(qrow + r1 * D + c0) : 0u;
+      qa[kk][2] = r0 < G ? *reinterpret_cast<const uint32_t*>(qrow + r0 * D + c0 + 8) : 0u;
+      qa[kk][3] = r1 < G ? *reinterpret_cast<const uint32_t*>(qrow + r1 * D + c0 + 8) : 0u;
+    }
+    float o[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    const int qpos = hd.ctx_len - 1;
+
+    for (int g = item.vp_begin; g < item.vp_end; ++g, ++k) {
+      const int s = k % NST;
+      if (ok && !mbar_wait(&full[s], (k / NST) & 1)) {
+        record_error(a.status, kDevTimeoutFull);
+        ok = false;
+      }
+      const PageDesc pg = a.pages[g];
+      const int tok0 = warp * 16;
+      if (ok && tok0 < pg.nvalid) {
+        const uint32_t kst = smem_u32(stage + s * 2 * PB);
+        const uint32_t vst = kst + PB;
+        // S = Q K^T over this warp's 16 tokens (two n8 tiles)
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        const int mi = lane >> 3, rr = lane & 7;
+        const int ktok = tok0 + (mi >> 1) * 8 + rr;
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4(b0, b1, b2, b3, kst + uint32_t(kpage_chunk_offset_bf16(ktok, 2 * kk + (mi & 1), P)));
+          mma_bf16_16816(sc[0], qa[kk], b0, b1);
+          mma_bf16_16816(sc[1], qa[kk], b2, b3);
+        }
+        // mask and scale (log2 domain)
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int tok = tok0 + n * 8 + tq * 2 + (e & 1);
+            bool vis = tok < pg.nvalid;
+            if (hd.mask_local) vis = vis && sees(1, hd.sink, hd.window, qpos, pg.abs_start + tok);
+            sc[n][e] = vis ? sc[n][e] * a.scale_log2 : -INFINITY;
+          }
+        float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+        float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float al0 = fast_exp2(m0 - base0), al1 = fast_exp2(m1 - base1);
+        m0 = mn0, m1 = mn1;
+        float p[2][4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+          p[n][0] = fast_exp2(sc[n][0] - base0);
+          p[n][1] = fast_exp2(sc[n][1] - base0);
+          p[n][2] = fast_exp2(sc[n][2] - base1);
+          p[n][3] = fast_exp2(sc[n][3] - base1);
+        }
+        l0 = l0 * al0 + ((p[0][0] + p[0][1]) + (p[1][0] + p[1][1]));
+        l1 = l1 * al1 + ((p[0][2] + p[0][3]) + (p[1][2] + p[1][3]));
+        uint32_t pa[4];
+        pa[0] = pack_bf16x2(p[0][0], p[0][1]);
+        pa[1] = pack_bf16x2(p[0][2], p[0][3]);
+        pa[2] = pack_bf16x2(p[1][0], p[1][1]);
+        pa[3] = pack_bf16x2(p[1][2], p[1][3]);
+        // O = alpha O + P V
+        const int vc = 2 * warp + (mi & 1);
+#pragma unroll
+        for (int j = 0; j < NT / 2; ++j) {
+          const int dd = (2 * j + (mi >> 1)) * 8 + rr;
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4(b0, b1, b2, b3, vst + uint32_t(vpage_chunk_offset_bf16(dd, vc)));
+          o[2 * j][0] *= al0, o[2 * j][1] *= al0, o[2 * j][2] *= al1, o[2 * j][3] *= al1;
+          o[2 * j + 1][0] *= al0, o[2 * j + 1][1] *= al0, o[2 * j + 1][2] *= al1, o[2 * j + 1][3] *= al1;
+          mma_bf16_16816(o[2 * j], pa, b0, b1);
+          mma_bf16_16816(o[2 * j + 1], pa, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+
+    // ---- merge the 4 warps' partial states of this item ----
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    float* mw = mbuf + warp * kMaxGroup * S::kMergePitch;
+    if (tq == 0) {
+      mlbuf[(warp * kMaxGroup + r0) * 2 + 0] = m0;
+      mlbuf[(warp * kMaxGroup + r0) * 2 + 1] = l0;
+      mlbuf[(warp * kMaxGroup + r1) * 2 + 0] = m1;
+      mlbuf[(warp * kMaxGroup + r1) * 2 + 1] = l1;
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      *reinterpret_cast<float2*>(mw + r0 * S::kMergePitch + j * 8 + tq * 2) = make_float2(o[j][0], o[j][1]);
+      if (r1 < G)
+        *reinterpret_cast<float2*>(mw + r1 * S::kMergePitch + j * 8 + tq * 2) = make_float2(o[j][2], o[j][3]);
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    for (int e = threadIdx.x; e < G * D; e += kConsumerWarps * 32) {
+      const int row = e / D, col = e % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mlbuf[(w * kMaxGroup + row) * 2]);
+      const float base = M == -INFINITY ? 0.f : M;
+      float acc = 0.f, L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float f = fast_exp2(mlbuf[(w * kMaxGroup + row) * 2] - base);
+        acc += f * mbuf[(w * kMaxGroup + row) * S::kMergePitch + col];
+        L += f * mlbuf[(w * kMaxGroup + row) * 2 + 1];
+      }
+      if (item.slot < 0) {
+        const int64_t o_idx = (int64_t(hd.q_row0) * a.num_q_heads + qh0 + row) * D + col;
+        static_cast<__nv_bfloat16*>(a.out)[o_idx] = __float2bfloat16_rn(acc / L);
+        if (col == 0 && a.lse) a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + row] = (M + log2f(L)) * kLn2;
+      } else {
+        float* slot = a.partial + int64_t(item.slot) * G * (D + 2);
+        slot[row * D + col] = acc;
+        if (col == 0) slot[G * D + row * 2] = M, slot[G * D + row * 2 + 1] = L;
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// fp32 SIMT decode (FP32 FMA only, exp2f).
+// ---------------------------------------------------------------------------
+constexpr int kF32Threads = 128;
+
+template <int D, int P>
+__global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(DecodeLaunch a) {
+  constexpr int PB = P * D * 4;
+  constexpr int ACC = kMaxGroup * D / kF32Threads;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  float* kp = reinterpret_cast<float*>(smem);        // [P][D]
+  float* vp = kp + P * D;                            // [D][P]
+  float* qs = vp + P * D;                            // [G][D]
+  float* sc = qs + kMaxGroup * D;                    // [G][P]
+  float* st = sc + kMaxGroup * P;                    // alpha[G], m[G], l[G]
+  const int ib = a.cta_begin[blockIdx.x], ie = a.cta_begin[blockIdx.x + 1];
+  const int G = a.group;
+  const float* qg = static_cast<const float*>(a.q);
+  const uint8_t* kpool = static_cast<const uint8_t*>(a.kpool);
+  const uint8_t* vpool = static_cast<const uint8_t*>(a.vpool);
+  for (int it = ib; it < ie; ++it) {
+    const DecodeItem item = a.items[it];
+    const HeadDesc hd = a.heads[item.head];
+    const int qh0 = hd.kv * G;
+    const int qpos = hd.ctx_len - 1;
+    __syncthreads();  // the previous item's output phase still reads st
+    for (int e = threadIdx.x; e < G * D; e += kF32Threads)
+      qs[e] = qg[(int64_t(hd.q_row0) * a.num_q_heads + qh0) * D + e];
+    if (threadIdx.x < G) st[kMaxGroup + threadIdx.x] = -INFINITY, st[2 * kMaxGroup + threadIdx.x] = 0.f;
+    float acc[ACC];
+#pragma unroll
+    for (int j = 0; j < ACC; ++j) acc[j] = 0.f;
+    for (int g = item.vp_begin; g < item.vp_end; ++g) {
+      const PageDesc pg = a.pages[g];
+      __syncthreads();
+      const uint4* ks = reinterpret_cast<const uint4*>(kpool + int64_t(pg.phys) * a.page_bytes);
+      const uint4* vs = reinterpret_cast<const uint4*>(vpool + int64_t(pg.phys) * a.page_bytes);
+      for (int e = threadIdx.x; e < PB / 16; e += kF32Threads) {
+        reinterpret_cast<uint4*>(kp)[e] = ks[e];
+        reinterpret_cast<uint4*>(vp)[e] = vs[e];
+      }
+      __syncthreads();
+      for (int e = threadIdx.x; e < G * P; e += kF32Threads) {
+        const int h = e / P, t = e % P;
+        bool vis = t < pg.nvalid;
+        if (hd.mask_local) vis = vis && sees(1, hd.sink, hd.window, qpos, pg.abs_start + t);
+        float s = 0.f;
+        for (int i = 0; i < D; ++i) s = fmaf(qs[h * D + i], kp[t * D + i], s);
+        sc[e] = vis ? s * a.scale_log2 : -INFINITY;
+      }
+      __syncthreads();
+      if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float mx = -INFINITY;
+        for (int t = 0; t < P; ++t) mx = fmaxf(mx, sc[h * P + t]);
+        const float mo = st[kMaxGroup + h], mn = fmaxf(mo, mx);
+        const float base = mn == -INFINITY ? 0.f : mn;
+        const float al = exp2f(mo - base);
+        float sum = 0.f;
+        for (int t = 0; t < P; ++t) {
+          const float pv = exp2f(sc[h * P + t] - base);
+          sc[h * P + t] = pv;
+          sum += pv;
+        }
+        st[h] = al;
+        st[kMaxGroup + h] = mn;
+        st[2 * kMaxGroup + h] = st[2 * kMaxGroup + h] * al + sum;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < ACC; ++j) {
+        const int e = threadIdx.x + j * kF32Threads;
+        const int row = e / D, col = e % D;
+        if (row >= G) continue;
+        float x = acc[j] * st[row];
+        for (int t = 0; t < P; ++t) x = fmaf(sc[row * P + t], vp[col * P + t], x);
+        acc[j] = x;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < ACC; ++j) {
+      const int e = threadIdx.x + j * kF32Threads;
+      const int row = e / D, col = e % D;
+      if (row >= G) continue;
+      const float M = st[kMaxGroup + row], L = st[2 * kMaxGroup + row];
+      if (item.slot < 0) {
+        const int64_t o_idx = (int64_t(hd.q_row0) * a.num_q_heads + qh0 + row) * D + col;
+        static_cast<float*>(a.out)[o_idx] = acc[j] / L;
+        if (col == 0 && a.lse) a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + row] = (M + log2f(L)) * kLn2;
+      } else {
+        float* slot = a.partial + int64_t(item.slot) * G * (D + 2);
+        slot[row * D + col] = acc[j];
+        if (col == 0) slot[G * D + row * 2] = M, slot[G * D + row * 2 + 1] = L;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Combine: one warp per (split head, q-head of its group).
+// ---------------------------------------------------------------------------
+template <typename TOut, int D, bool FAST>
+__global__ void __launch_bounds__(128) combine_kernel(DecodeLaunch a) {
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  const int G = a.group;
+  if (gw >= a.n_combine * G) return;
+  const CombineItem ci = a.combine[gw / G];
+  const int row = gw % G;
+  const HeadDesc hd = a.heads[ci.head];
+  float M = -INFINITY;
+  for (int i = 0; i < ci.n_slots; ++i)
+    M = fmaxf(M, a.partial[int64_t(ci.slot_begin + i) * G * (D + 2) + G * D + row * 2]);
+  const float base = M == -INFINITY ? 0.f : M;
+  float acc[D / 32];
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j) acc[j] = 0.f;
+  float L = 0.f;
+  for (int i = 0; i < ci.n_slots; ++i) {
+    const float* slot = a.partial + int64_t(ci.slot_begin + i) * G * (D + 2);
+    const float mi = slot[G * D + row * 2];
+    const float f = FAST ? fast_exp2(mi - base) : exp2f(mi - base);
+    L += f * slot[G * D + row * 2 + 1];
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) acc[j] += f * slot[row * D + j * 32 + lane];
+  }
+  const int qh = hd.kv * G + row;
+  const int64_t o_idx = (int64_t(hd.q_row0) * a.num_q_heads + qh) * D;
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j) {
+    const float v = acc[j] / L;
+    if constexpr (sizeof(TOut) == 2)
+      static_cast<__nv_bfloat16*>(a.out)[o_idx + j * 32 + lane] = __float2bfloat16_rn(v);
+    else
+      static_cast<float*>(a.out)[o_idx + j * 32 + lane] = v;
+  }
+  if (lane == 0 && a.lse) a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh] = (M + log2f(L)) * kLn2;
+}
+
+constexpr int kStagesBf16 = 2;
+
+template <int D>
+cudaError_t launch_bf16(const DecodeLaunch& a, cudaStream_t s) {
+  using Sm = DecodeSmem<D, kStagesBf16>;
+  auto kern = decode_bf16_kernel<D, kStagesBf16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<a.n_ctas, kDecodeThreads, Sm::kBytes, s>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.n_combine == 0) return e;
+  combine_kernel<__nv_bfloat16, D, true><<<(a.n_combine * a.group + 3) / 4, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int P>
+cudaError_t launch_f32(const DecodeLaunch& a, cudaStream_t s) {
+  const int bytes = (2 * P * D + kMaxGroup * D + kMaxGroup * P + 3 * kMaxGroup) * 4;
+  auto kern = decode_f32_kernel<D, P>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  kern<<<a.n_ctas, kF32Threads, bytes, s>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.n_combine == 0) return e;
+  combine_kernel<float, D, false><<<(a.n_combine * a.group + 3) / 4, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s) {
+  if (a.n_ctas == 0) return cudaSuccess;
+  if (a.bf16) return a.D == 128 ? launch_bf16<128>(a, s) : launch_bf16<64>(a, s);
+  if (a.P == 16) return a.D == 128 ? launch_f32<128, 16>(a, s) : launch_f32<64, 16>(a, s);
+  return a.D == 128 ? launch_f32<128, 64>(a, s) : launch_f32<64, 64>(a, s);
+}
+
+}  // namespace sp

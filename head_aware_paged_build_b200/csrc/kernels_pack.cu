@@ -1,0 +1,158 @@
+// build_segpaged_cache (pack) and its inverse (gather).
+//
+// One CTA per page: it copies the page's stored rows of dense K/V (16-byte
+// vector loads, consecutive threads on consecutive chunks of a row) into the
+// pool's page layout.  K chunks move straight to their swizzled slot; V is
+// transposed through shared memory.  Slots past the last stored position of a
+// segment are written as zeros so that every pool byte the attention kernels
+// read is a finite number ("SegPagedAttention runtime design", §3:
+// build_segpaged_cache packs dense KV and keeps only what a head can see).
+#include "device_common.cuh"
+#include "kernels.h"
+
+namespace sp {
+namespace {
+
+constexpr int kPackThreads = 256;
+
+struct PackArgs {
+  const HeadDesc* heads;
+  const PageDesc* pages;
+  int64_t stride_seq, stride_head, stride_tok;  // stride_seq < 0: packed by context rows
+  int64_t page_bytes;
+};
+
+// Shared-memory row pitch of the V staging tile: one extra 32-bit word per row
+// makes column reads (the transpose) and row writes both bank-conflict free.
+template <typename T>
+__host__ __device__ constexpr int vstage_pitch_words(int D) {
+  return D * int(sizeof(T)) / 4 + 1;
+}
+
+template <typename T>
+__device__ __forceinline__ int64_t kpage_chunk(int t, int c16, int P, int D) {
+  if constexpr (sizeof(T) == 2) {
+    return kpage_chunk_offset_bf16(t, c16, P);
+  } else {
+    return (int64_t(t) * D) * 4 + c16 * 16;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ int64_t vpage_chunk(int i, int c16, int P) {
+  if constexpr (sizeof(T) == 2) {
+    return vpage_chunk_offset_bf16(i, c16);
+  } else {
+    return (int64_t(i) * P) * 4 + c16 * 16;
+  }
+}
+
+template <typename T, int D, int P>
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(PackArgs a, const T* __restrict__ kd,
+                                                            const T* __restrict__ vd, uint8_t* __restrict__ kpool,
+                                                            uint8_t* __restrict__ vpool) {
+  constexpr int CR = D * int(sizeof(T)) / 16;   // 16-byte chunks per dense row
+  constexpr int EPC = 16 / int(sizeof(T));      // elements per chunk
+  constexpr int PW = vstage_pitch_words<T>(D);  // staging pitch (32-bit words)
+  constexpr int VR = P / EPC;                   // chunks per transposed V row
+  __shared__ uint32_t stage[P * PW];
+
+  const PageDesc pg = a.pages[blockIdx.x];
+  const HeadDesc hd = a.heads[pg.head];
+  const int64_t base = (a.stride_seq >= 0 ? int64_t(hd.b) * a.stride_seq : int64_t(hd.ctx_row0) * a.stride_tok) +
+                       int64_t(hd.kv) * a.stride_head;
+  uint8_t* kdst = kpool + int64_t(pg.phys) * a.page_bytes;
+  uint8_t* vdst = vpool + int64_t(pg.phys) * a.page_bytes;
+
+  for (int idx = threadIdx.x; idx < P * CR; idx += kPackThreads) {
+    const int t = idx / CR, c = idx % CR;
+    uint4 kv4 = make_uint4(0, 0, 0, 0), vv4 = make_uint4(0, 0, 0, 0);
+    if (t < pg.nvalid) {
+      const int64_t row = base + int64_t(pg.abs_start + t) * a.stride_tok;
+      kv4 = __ldg(reinterpret_cast<const uint4*>(kd + row) + c);
+      vv4 = __ldg(reinterpret_cast<const uint4*>(vd + row) + c);
+    }
+    *reinterpret_cast<uint4*>(kdst + kpage_chunk<T>(t, c, P, D)) = kv4;
+    uint32_t* s = stage + t * PW + c * 4;
+    s[0] = vv4.x, s[1] = vv4.y, s[2] = vv4.z, s[3] = vv4.w;
+  }
+  __syncthreads();
+  // transposed V: row i (dimension) holds the page's P tokens
+  const T* st = reinterpret_cast<const T*>(stage);
+  for (int idx = threadIdx.x; idx < D * VR; idx += kPackThreads) {
+    const int i = idx / VR, c = idx % VR;
+    alignas(16) T vals[EPC];
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) vals[e] = st[(c * EPC + e) * (PW * 4 / int(sizeof(T))) + i];
+    *reinterpret_cast<uint4*>(vdst + vpage_chunk<T>(i, c, P)) = *reinterpret_cast<const uint4*>(vals);
+  }
+}
+
+template <typename T, int D, int P>
+__global__ void __launch_bounds__(kPackThreads) gather_kernel(PackArgs a, const uint8_t* __restrict__ kpool,
+                                                              const uint8_t* __restrict__ vpool, T* __restrict__ kd,
+                                                              T* __restrict__ vd) {
+  constexpr int CR = D * int(sizeof(T)) / 16;
+  constexpr int EPC = 16 / int(sizeof(T));
+  constexpr int PW = vstage_pitch_words<T>(D);
+  constexpr int VR = P / EPC;
+  __shared__ uint32_t stage[P * PW];
+
+  const PageDesc pg = a.pages[blockIdx.x];
+  const HeadDesc hd = a.heads[pg.head];
+  const int64_t base = (a.stride_seq >= 0 ? int64_t(hd.b) * a.stride_seq : int64_t(hd.ctx_row0) * a.stride_tok) +
+                       int64_t(hd.kv) * a.stride_head;
+  const uint8_t* ksrc = kpool + int64_t(pg.phys) * a.page_bytes;
+  const uint8_t* vsrc = vpool + int64_t(pg.phys) * a.page_bytes;
+
+  T* st = reinterpret_cast<T*>(stage);
+  for (int idx = threadIdx.x; idx < D * VR; idx += kPackThreads) {
+    const int i = idx / VR, c = idx % VR;
+    alignas(16) T vals[EPC];
+    *reinterpret_cast<uint4*>(vals) = *reinterpret_cast<const uint4*>(vsrc + vpage_chunk<T>(i, c, P));
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) st[(c * EPC + e) * (PW * 4 / int(sizeof(T))) + i] = vals[e];
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < P * CR; idx += kPackThreads) {
+    const int t = idx / CR, c = idx % CR;
+    if (t >= pg.nvalid) continue;
+    const int64_t row = base + int64_t(pg.abs_start + t) * a.stride_tok;
+    reinterpret_cast<uint4*>(kd + row)[c] = *reinterpret_cast<const uint4*>(ksrc + kpage_chunk<T>(t, c, P, D));
+    const uint32_t* s = stage + t * PW + c * 4;
+    reinterpret_cast<uint4*>(vd + row)[c] = make_uint4(s[0], s[1], s[2], s[3]);
+  }
+}
+
+template <typename T, int D, int P>
+void launch_pack_t(const PackLaunch& L, cudaStream_t s) {
+  PackArgs a{L.heads, L.pages, L.stride_seq, L.stride_head, L.stride_tok, L.page_bytes};
+  if (L.inverse)
+    gather_kernel<T, D, P><<<L.n_pages, kPackThreads, 0, s>>>(a, static_cast<const uint8_t*>(L.kpool_in),
+                                                              static_cast<const uint8_t*>(L.vpool_in),
+                                                              static_cast<T*>(L.kdense_out),
+                                                              static_cast<T*>(L.vdense_out));
+  else
+    pack_kernel<T, D, P><<<L.n_pages, kPackThreads, 0, s>>>(a, static_cast<const T*>(L.kdense_in),
+                                                            static_cast<const T*>(L.vdense_in),
+                                                            static_cast<uint8_t*>(L.kpool_out),
+                                                            static_cast<uint8_t*>(L.vpool_out));
+}
+
+}  // namespace
+
+void launch_pack(const PackLaunch& L, cudaStream_t s) {
+  if (L.n_pages == 0) return;
+  if (L.bf16) {
+    if (L.D == 128) launch_pack_t<__nv_bfloat16, 128, 64>(L, s);
+    else launch_pack_t<__nv_bfloat16, 64, 64>(L, s);
+  } else if (L.P == 16) {
+    if (L.D == 128) launch_pack_t<float, 128, 16>(L, s);
+    else launch_pack_t<float, 64, 16>(L, s);
+  } else {
+    if (L.D == 128) launch_pack_t<float, 128, 64>(L, s);
+    else launch_pack_t<float, 64, 64>(L, s);
+  }
+}
+
+}  // namespace sp

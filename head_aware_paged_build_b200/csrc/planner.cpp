@@ -1,0 +1,398 @@
+// Host planner of libsegpaged.so: policy -> segments -> pages -> work lists.
+//
+// Everything that depends only on the batch's layout is decided here, once,
+// when the plan is created ("SegPagedAttention runtime design", §5: page
+// tables and layout must be built when KV is written and reused, because
+// computing them on every attention call cost a 0.70x slowdown).
+#include <algorithm>
+#include <cstring>
+#include <limits>
+#include <new>
+#include <numeric>
+#include <string>
+#include <vector>
+
+#include "sp_internal.h"
+
+namespace sp {
+
+thread_local std::string g_last_error;
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+sp_status fail(sp_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+namespace {
+
+constexpr int kDefaultDecodeCtas = 2 * 148;
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+sp_status validate(const sp_problem& p) {
+  if (p.batch < 1 || p.num_q_heads < 1 || p.num_kv_heads < 1 || p.head_dim < 1 || p.page_size < 1)
+    return fail(SP_ERR_INVALID_ARG, "batch, head counts, head_dim and page_size must be >= 1");
+  if (!p.ctx_len || !p.q_start || !p.policy)
+    return fail(SP_ERR_INVALID_ARG, "ctx_len, q_start and policy must be non-NULL host arrays");
+  if (p.flags & ~uint32_t(SP_FLAG_DENSE_MASKED)) return fail(SP_ERR_INVALID_ARG, "unknown flag bits");
+  if (p.first_page < 0) return fail(SP_ERR_INVALID_ARG, "first_page must be >= 0");
+  if (p.target_ctas < 0) return fail(SP_ERR_INVALID_ARG, "target_ctas must be >= 0");
+  if (p.dtype != SP_F32 && p.dtype != SP_BF16) return fail(SP_ERR_UNSUPPORTED, "dtype must be SP_F32 or SP_BF16");
+  if (p.head_dim != 64 && p.head_dim != 128) return fail(SP_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (p.dtype == SP_BF16 && p.page_size != 64) return fail(SP_ERR_UNSUPPORTED, "bf16 pools need page_size 64");
+  if (p.dtype == SP_F32 && p.page_size != 16 && p.page_size != 64)
+    return fail(SP_ERR_UNSUPPORTED, "fp32 pools need page_size 16 or 64");
+  if (p.num_q_heads % p.num_kv_heads != 0)
+    return fail(SP_ERR_UNSUPPORTED, "num_q_heads must be a multiple of num_kv_heads");
+  if (p.num_q_heads / p.num_kv_heads > kMaxGroup)
+    return fail(SP_ERR_UNSUPPORTED, "at most 16 q-heads per kv-head");
+  int64_t rows = 0;
+  for (int b = 0; b < p.batch; ++b) {
+    const int64_t L = p.ctx_len[b], q0 = p.q_start[b];
+    if (L < 1) return fail(SP_ERR_INVALID_ARG, "ctx_len[" + std::to_string(b) + "] must be >= 1");
+    if (L > (int64_t(1) << 30)) return fail(SP_ERR_UNSUPPORTED, "ctx_len above 2^30");
+    if (q0 < 0 || q0 >= L)
+      return fail(SP_ERR_INVALID_ARG, "q_start[" + std::to_string(b) + "] must lie in [0, ctx_len)");
+    rows += L - q0;
+  }
+  if (rows > std::numeric_limits<int32_t>::max()) return fail(SP_ERR_UNSUPPORTED, "too many query rows");
+  for (int64_t i = 0; i < int64_t(p.batch) * p.num_kv_heads; ++i) {
+    const sp_head_policy& h = p.policy[i];
+    if (h.kind == SP_RETRIEVAL)
+      return fail(SP_ERR_UNSUPPORTED, "RETRIEVAL heads are not implemented (no scoring rule is defined)");
+    if (h.kind != SP_GLOBAL && h.kind != SP_LOCAL && h.kind != SP_DENSE)
+      return fail(SP_ERR_INVALID_ARG, "policy[" + std::to_string(i) + "].kind is not a head kind");
+    if (h.kind == SP_LOCAL && (h.sink < 0 || h.window < 1))
+      return fail(SP_ERR_INVALID_ARG, "policy[" + std::to_string(i) + "]: local heads need sink >= 0, window >= 1");
+  }
+  return SP_OK;
+}
+
+// Pages of a head (indices into its page list) holding any position of [x, y].
+void pages_touching(const sp_plan& pl, int h, int64_t x, int64_t y, int64_t* v0, int64_t* v1) {
+  *v0 = std::numeric_limits<int64_t>::max();
+  *v1 = std::numeric_limits<int64_t>::min();
+  const int P = pl.prob.page_size;
+  for (int s = pl.seg_begin[h]; s < pl.seg_begin[h + 1]; ++s) {
+    const sp_segment& g = pl.segments[s];
+    const int64_t lo = std::max<int64_t>(g.abs_start, x);
+    const int64_t hi = std::min<int64_t>(int64_t(g.abs_start) + g.length - 1, y);
+    if (lo > hi) continue;
+    *v0 = std::min<int64_t>(*v0, g.first_page_index + (lo - g.abs_start) / P);
+    *v1 = std::max<int64_t>(*v1, g.first_page_index + (hi - g.abs_start) / P + 1);
+  }
+  if (*v0 > *v1) *v0 = *v1 = 0;
+}
+
+void align_to(std::vector<uint8_t>& blob, size_t a) { blob.resize((blob.size() + a - 1) / a * a, 0); }
+
+template <typename T>
+int64_t append(std::vector<uint8_t>& blob, const std::vector<T>& v) {
+  align_to(blob, 256);
+  const int64_t off = int64_t(blob.size());
+  blob.resize(blob.size() + v.size() * sizeof(T));
+  if (!v.empty()) std::memcpy(blob.data() + off, v.data(), v.size() * sizeof(T));
+  return off;
+}
+
+sp_status plan_build(sp_plan& pl) {
+  const sp_problem& p = pl.prob;
+  const int B = p.batch, Hkv = p.num_kv_heads, P = p.page_size, D = p.head_dim;
+  const bool dense_masked = (p.flags & SP_FLAG_DENSE_MASKED) != 0;
+  pl.group = p.num_q_heads / Hkv;
+  pl.elem_bytes = p.dtype == SP_BF16 ? 2 : 4;
+  const int nh = B * Hkv;
+
+  // --- segments and pages ---------------------------------------------------
+  pl.seg_begin.assign(1, 0);
+  pl.heads.resize(nh);
+  int64_t n_pages = 0, stored = 0, dense_rows = 0, visible = 0;
+  std::vector<int32_t> qrow(B + 1, 0);
+  for (int b = 0; b < B; ++b) qrow[b + 1] = qrow[b] + (pl.ctx_len[b] - pl.q_start[b]);
+  bool decode = true;
+  for (int b = 0; b < B; ++b) decode = decode && (pl.ctx_len[b] - pl.q_start[b] == 1);
+
+  int64_t ctx_row = 0;
+  for (int b = 0; b < B; ++b, ctx_row += pl.ctx_len[b - 1]) {
+    const int64_t L = pl.ctx_len[b], q0 = pl.q_start[b];
+    if (ctx_row + L > std::numeric_limits<int32_t>::max())
+      return fail(SP_ERR_UNSUPPORTED, "sum of ctx_len above 2^31");
+    for (int kv = 0; kv < Hkv; ++kv) {
+      const int h = b * Hkv + kv;
+      const sp_head_policy& pol = pl.policy[h];
+      const bool local = pol.kind == SP_LOCAL;
+      const int64_t s = local ? pol.sink : 0, w = local ? pol.window : 0;
+      int64_t firsts[2], lens[2];
+      int ns = 0;
+      if (!local || dense_masked) {
+        firsts[ns] = 0, lens[ns++] = L;
+      } else {
+        const int64_t sink_len = std::min<int64_t>(s, L);
+        const int64_t rec = std::max<int64_t>(s, q0 - w + 1);
+        if (rec <= sink_len) {  // touching: one run [0, L)
+          firsts[ns] = 0, lens[ns++] = L;
+        } else {
+          if (sink_len > 0) firsts[ns] = 0, lens[ns++] = sink_len;
+          if (rec < L) firsts[ns] = rec, lens[ns++] = L - rec;
+        }
+      }
+      HeadDesc& hd = pl.heads[h];
+      hd = HeadDesc{};
+      hd.kind = local ? 1 : 0;
+      hd.sink = int32_t(s);
+      hd.window = int32_t(std::min<int64_t>(w, std::numeric_limits<int32_t>::max()));
+      hd.ctx_len = int32_t(L);
+      hd.q_start = int32_t(q0);
+      hd.vpage_begin = int32_t(n_pages);
+      hd.mask_local = (local && dense_masked) ? 1 : 0;
+      hd.b = b;
+      hd.kv = kv;
+      hd.q_row0 = qrow[b];
+      int32_t vp = 0;
+      for (int i = 0; i < ns; ++i) {
+        sp_segment g{int32_t(firsts[i]), int32_t(lens[i]), vp, int32_t(ceil_div(lens[i], P))};
+        pl.segments.push_back(g);
+        for (int k = 0; k < g.num_pages; ++k) {
+          PageDesc pd{};
+          pd.phys = 0;  // assigned below
+          pd.abs_start = g.abs_start + k * P;
+          pd.nvalid = int32_t(std::min<int64_t>(P, int64_t(g.abs_start) + g.length - pd.abs_start));
+          pd.head = h;
+          pl.pages.push_back(pd);
+        }
+        vp += g.num_pages;
+        stored += lens[i];
+      }
+      hd.n_vpages = vp;
+      hd.ctx_row0 = int32_t(ctx_row);
+      n_pages += vp;
+      if (n_pages > std::numeric_limits<int32_t>::max())
+        return fail(SP_ERR_UNSUPPORTED, "more than 2^31 pages");
+      pl.seg_begin.push_back(int32_t(pl.segments.size()));
+      dense_rows += L;
+      // visible (query, key) pairs: global p + 1, local min(p + 1, s + w)
+      for (int64_t q = q0; q < L; ++q) visible += local ? std::min<int64_t>(q + 1, s + w) : q + 1;
+    }
+  }
+  visible *= pl.group;
+
+  // --- physical page ids -----------------------------------------------------
+  int64_t max_id = n_pages - 1;
+  if (p.page_ids) {
+    std::vector<int32_t> ids(p.page_ids, p.page_ids + n_pages);
+    for (int32_t id : ids)
+      if (id < 0) return fail(SP_ERR_INVALID_ARG, "page_ids must be non-negative");
+    std::sort(ids.begin(), ids.end());
+    if (std::adjacent_find(ids.begin(), ids.end()) != ids.end())
+      return fail(SP_ERR_INVALID_ARG, "page_ids must be distinct");
+    max_id = n_pages ? ids.back() : -1;
+  }
+  if (p.first_page + max_id + 1 > std::numeric_limits<int32_t>::max())
+    return fail(SP_ERR_UNSUPPORTED, "pool above 2^31 pages");
+  for (int64_t i = 0; i < n_pages; ++i)
+    pl.pages[i].phys = int32_t(p.first_page + (p.page_ids ? p.page_ids[i] : i));
+
+  // --- decode: equal page ranges per CTA, cut at head boundaries ------------
+  int n_slots = 0;
+  if (decode) {
+    const int64_t G = std::min<int64_t>(p.target_ctas ? p.target_ctas : kDefaultDecodeCtas, n_pages);
+    pl.decode_cta_begin.assign(1, 0);
+    for (int64_t c = 0; c < G; ++c) {
+      int64_t lo = c * n_pages / G, hi = (c + 1) * n_pages / G;
+      while (lo < hi) {
+        const int h = pl.pages[lo].head;
+        const int64_t end = std::min<int64_t>(hi, pl.heads[h].vpage_begin + pl.heads[h].n_vpages);
+        pl.decode_items.push_back(DecodeItem{h, int32_t(lo), int32_t(end), -1});
+        lo = end;
+      }
+      pl.decode_cta_begin.push_back(int32_t(pl.decode_items.size()));
+    }
+    // items of a head are consecutive; split heads get consecutive slots
+    size_t i = 0;
+    while (i < pl.decode_items.size()) {
+      size_t j = i;
+      while (j < pl.decode_items.size() && pl.decode_items[j].head == pl.decode_items[i].head) ++j;
+      if (j - i > 1) {
+        pl.combine.push_back(CombineItem{pl.decode_items[i].head, n_slots, int32_t(j - i), 0});
+        for (size_t k = i; k < j; ++k) pl.decode_items[k].slot = n_slots++;
+      }
+      i = j;
+    }
+  } else {
+    // --- prefill: query tiles x visited KV tile ranges -----------------------
+    const int T = p.dtype == SP_BF16 ? kPrefillTileTokensBf16 : kPrefillTileTokensF32;
+    const int ppt = T / P;
+    pl.prefill_tile = T;
+    std::vector<std::vector<PrefillItem>> per_head(nh);
+    std::vector<int32_t> head_max(nh, 0);
+    for (int h = 0; h < nh; ++h) {
+      const HeadDesc& hd = pl.heads[h];
+      const int64_t C = hd.ctx_len - hd.q_start;
+      for (int64_t qt = 0; qt * T < C; ++qt) {
+        PrefillItem it{};
+        it.head = h;
+        it.n_rows = int32_t(std::min<int64_t>(T, C - qt * T));
+        it.q_row = int32_t(hd.q_row0 + qt * T);
+        it.p0 = int32_t(hd.q_start + qt * T);
+        const int64_t p1 = it.p0 + it.n_rows - 1;
+        int64_t v0, v1, v2, v3;
+        if (hd.kind == 0 || dense_masked) {
+          pages_touching(pl, h, 0, p1, &v0, &v1);
+          v2 = v3 = 0;
+        } else {
+          pages_touching(pl, h, 0, std::min<int64_t>(hd.sink, p1 + 1) - 1, &v0, &v1);
+          pages_touching(pl, h, std::max<int64_t>(hd.sink, int64_t(it.p0) - hd.window + 1), p1, &v2, &v3);
+        }
+        int64_t t0 = v0 / ppt, t1 = ceil_div(v1, ppt), t2 = v2 / ppt, t3 = ceil_div(v3, ppt);
+        if (v0 == v1) t0 = t1 = 0;
+        if (v2 == v3) t2 = t3 = 0;
+        if (t0 == t1) std::swap(t0, t2), std::swap(t1, t3);
+        if (t2 < t3 && t2 <= t1) t1 = std::max(t1, t3), t2 = t3 = 0;
+        it.t0 = int32_t(t0), it.t1 = int32_t(t1), it.t2 = int32_t(t2), it.t3 = int32_t(t3);
+        it.work = int32_t((t1 - t0) + (t3 - t2));
+        head_max[h] = std::max(head_max[h], it.work);
+        per_head[h].push_back(it);
+      }
+    }
+    // Heaviest heads first; within a head the heaviest query tiles first, the
+    // group's q-heads back to back so that they share KV tiles through L2.
+    std::vector<int> order(nh);
+    std::iota(order.begin(), order.end(), 0);
+    std::stable_sort(order.begin(), order.end(), [&](int a, int c) { return head_max[a] > head_max[c]; });
+    for (int h : order) {
+      auto& v = per_head[h];
+      std::stable_sort(v.begin(), v.end(), [](const PrefillItem& a, const PrefillItem& c) { return a.work > c.work; });
+      const int kv = pl.heads[h].kv;
+      for (const PrefillItem& it : v)
+        for (int g = 0; g < pl.group; ++g) {
+          PrefillItem x = it;
+          x.qh = kv * pl.group + g;
+          pl.prefill.push_back(x);
+        }
+    }
+  }
+  pl.n_partial_slots = n_slots;
+
+  // --- table blob --------------------------------------------------------------
+  TableHeader& H = pl.hdr;
+  H = TableHeader{};
+  H.magic = kTableMagic;
+  H.version = SEGPAGED_ABI_VERSION;
+  H.n_heads = nh;
+  H.n_vpages = int32_t(n_pages);
+  H.n_decode_items = int32_t(pl.decode_items.size());
+  H.n_decode_ctas = decode ? int32_t(pl.decode_cta_begin.size() - 1) : 0;
+  H.n_combine = int32_t(pl.combine.size());
+  H.n_prefill_items = int32_t(pl.prefill.size());
+  pl.blob.assign(sizeof(TableHeader), 0);
+  H.off_heads = append(pl.blob, pl.heads);
+  H.off_pages = append(pl.blob, pl.pages);
+  H.off_decode_items = append(pl.blob, pl.decode_items);
+  H.off_decode_cta = append(pl.blob, pl.decode_cta_begin);
+  H.off_combine = append(pl.blob, pl.combine);
+  H.off_prefill = append(pl.blob, pl.prefill);
+  align_to(pl.blob, 256);
+  std::memcpy(pl.blob.data(), &H, sizeof(H));
+
+  sp_sizes& z = pl.sizes;
+  z = sp_sizes{};
+  z.num_pages = n_pages;
+  z.pool_pages = p.first_page + max_id + 1;
+  z.page_bytes = int64_t(P) * D * pl.elem_bytes;
+  z.table_bytes = int64_t(pl.blob.size());
+  const int64_t partial = int64_t(n_slots) * pl.group * (D + 2) * 4;
+  z.workspace_bytes = kStatusBytes + ceil_div(partial, 256) * 256;
+  z.stored_token_heads = stored;
+  z.dense_token_heads = dense_rows;
+  z.visible_pairs = visible;
+  z.num_queries = qrow[B];
+  z.is_decode = decode ? 1 : 0;
+  z.num_decode_ctas = H.n_decode_ctas;
+  z.num_prefill_items = H.n_prefill_items;
+  return SP_OK;
+}
+
+}  // namespace
+}  // namespace sp
+
+extern "C" {
+
+const char* segpaged_last_error(void) { return sp::g_last_error.c_str(); }
+
+int32_t segpaged_abi_version(void) { return SEGPAGED_ABI_VERSION; }
+
+const char* segpaged_status_string(sp_status st) {
+  switch (st) {
+    case SP_OK: return "SP_OK";
+    case SP_ERR_INVALID_ARG: return "SP_ERR_INVALID_ARG";
+    case SP_ERR_UNSUPPORTED: return "SP_ERR_UNSUPPORTED";
+    case SP_ERR_WORKSPACE: return "SP_ERR_WORKSPACE";
+    case SP_ERR_CUDA: return "SP_ERR_CUDA";
+    case SP_ERR_DEVICE_CHECK: return "SP_ERR_DEVICE_CHECK";
+  }
+  return "unknown sp_status";
+}
+
+sp_status segpaged_plan_create(const sp_problem* problem, sp_plan** out) {
+  if (!problem || !out) return sp::fail(SP_ERR_INVALID_ARG, "problem and out must be non-NULL");
+  *out = nullptr;
+  try {
+    sp_status st = sp::validate(*problem);
+    if (st != SP_OK) return st;
+    auto* pl = new sp_plan();
+    pl->prob = *problem;
+    const int B = problem->batch, nh = problem->batch * problem->num_kv_heads;
+    pl->ctx_len.assign(problem->ctx_len, problem->ctx_len + B);
+    pl->q_start.assign(problem->q_start, problem->q_start + B);
+    pl->policy.assign(problem->policy, problem->policy + nh);
+    st = sp::plan_build(*pl);
+    pl->prob.ctx_len = pl->prob.q_start = nullptr;
+    pl->prob.policy = nullptr;
+    pl->prob.page_ids = nullptr;
+    if (st != SP_OK) {
+      delete pl;
+      return st;
+    }
+    *out = pl;
+    return SP_OK;
+  } catch (const std::bad_alloc&) {
+    return sp::fail(SP_ERR_INVALID_ARG, "out of host memory while planning");
+  } catch (...) {
+    return sp::fail(SP_ERR_INVALID_ARG, "unexpected error while planning");
+  }
+}
+
+void segpaged_plan_destroy(sp_plan* plan) { delete plan; }
+
+sp_status segpaged_plan_sizes(const sp_plan* plan, sp_sizes* out) {
+  if (!plan || !out) return sp::fail(SP_ERR_INVALID_ARG, "plan and out must be non-NULL");
+  *out = plan->sizes;
+  return SP_OK;
+}
+
+sp_status segpaged_plan_head_segments(const sp_plan* plan, int32_t b, int32_t kv, sp_segment* segs,
+                                      int32_t max, int32_t* count) {
+  if (!plan || !count || (max > 0 && !segs)) return sp::fail(SP_ERR_INVALID_ARG, "NULL argument");
+  if (b < 0 || b >= plan->prob.batch || kv < 0 || kv >= plan->prob.num_kv_heads)
+    return sp::fail(SP_ERR_INVALID_ARG, "(b, kv) out of range");
+  const int h = b * plan->prob.num_kv_heads + kv;
+  const int n = plan->seg_begin[h + 1] - plan->seg_begin[h];
+  *count = n;
+  for (int i = 0; i < n && i < max; ++i) segs[i] = plan->segments[plan->seg_begin[h] + i];
+  return SP_OK;
+}
+
+sp_status segpaged_plan_head_pages(const sp_plan* plan, int32_t b, int32_t kv, int64_t* page_ids,
+                                   int32_t max, int32_t* count) {
+  if (!plan || !count || (max > 0 && !page_ids)) return sp::fail(SP_ERR_INVALID_ARG, "NULL argument");
+  if (b < 0 || b >= plan->prob.batch || kv < 0 || kv >= plan->prob.num_kv_heads)
+    return sp::fail(SP_ERR_INVALID_ARG, "(b, kv) out of range");
+  const sp::HeadDesc& hd = plan->heads[b * plan->prob.num_kv_heads + kv];
+  *count = hd.n_vpages;
+  for (int i = 0; i < hd.n_vpages && i < max; ++i) page_ids[i] = plan->pages[hd.vpage_begin + i].phys;
+  return SP_OK;
+}
+
+}  // extern "C"

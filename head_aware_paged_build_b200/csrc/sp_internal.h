@@ -1,0 +1,126 @@
+// Internal layout of the SegmentPageTable blob and of the plan, shared by the
+// host planner and the CUDA kernels of libsegpaged.so.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "segpaged.h"
+
+namespace sp {
+
+constexpr int32_t kTableMagic = 0x53504731;  // "SPG1"
+constexpr int kStatusBytes = 256;            // workspace prefix holding the status word
+constexpr int kPrefillTileTokensBf16 = 128;  // KV / query tile of the tcgen05 prefill kernel
+constexpr int kPrefillTileTokensF32 = 64;    // KV / query tile of the fp32 prefill kernel
+constexpr int kMaxGroup = 16;                // q-heads per kv-head handled by one decode CTA
+
+// Device status codes (workspace word 0); the first error sticks.
+enum DeviceCode : int32_t {
+  kDevOk = 0,
+  kDevTimeoutFull = 1,     // a consumer gave up waiting for a page / tile copy
+  kDevTimeoutEmpty = 2,    // the producer gave up waiting for a free stage
+  kDevTimeoutMma = 3,      // a wait on a tensor-core commit ran out
+  kDevTimeoutSoftmax = 4,  // the MMA issuer gave up waiting for P
+  kDevBadPage = 5,         // a page id outside the pool (debug builds)
+};
+
+// One (sequence, kv-head).  Kinds are resolved: 0 reads the whole causal
+// context, 1 is local (sink + window).
+struct alignas(16) HeadDesc {
+  int32_t kind;
+  int32_t sink;
+  int32_t window;
+  int32_t ctx_len;
+  int32_t q_start;
+  int32_t vpage_begin;  // first entry of this head in the page array
+  int32_t n_vpages;
+  int32_t mask_local;   // 1: kernels apply the local mask per element (dense-masked baseline)
+  int32_t b;
+  int32_t kv;
+  int32_t q_row0;       // first row of sequence b in the varlen query / output arrays
+  int32_t ctx_row0;     // L_0 + ... + L_{b-1}: first token row of sequence b when packed
+};
+static_assert(sizeof(HeadDesc) == 48, "HeadDesc layout");
+
+// One page of a head, in the head's position order.
+struct alignas(16) PageDesc {
+  int32_t phys;       // physical page id in the pools
+  int32_t abs_start;  // absolute position held by slot 0
+  int32_t nvalid;     // slots [0, nvalid) hold positions abs_start .. abs_start + nvalid - 1
+  int32_t head;       // owning HeadDesc index
+};
+static_assert(sizeof(PageDesc) == 16, "PageDesc layout");
+
+// A run of consecutive pages of one head processed by one decode CTA.
+struct alignas(16) DecodeItem {
+  int32_t head;
+  int32_t vp_begin;  // global page-array indices [vp_begin, vp_end)
+  int32_t vp_end;
+  int32_t slot;      // partial-result slot in the workspace, or -1: the item covers the head
+};
+
+// A head whose decode result is split across several items.
+struct alignas(16) CombineItem {
+  int32_t head;
+  int32_t slot_begin;
+  int32_t n_slots;
+  int32_t pad;
+};
+
+// One prefill work unit: a tile of query rows of one q-head.  KV tiles (of the
+// kernel's tile size, counted in the head's page list) are visited in
+// [t0, t1) then [t2, t3).
+struct alignas(16) PrefillItem {
+  int32_t head;
+  int32_t qh;      // absolute q-head index
+  int32_t q_row;   // first varlen row of the tile
+  int32_t n_rows;  // rows in the tile (<= tile size)
+  int32_t p0;      // absolute position of the first row
+  int32_t t0, t1, t2, t3;
+  int32_t work;    // visited KV tiles
+  int32_t pad0, pad1;
+};
+static_assert(sizeof(PrefillItem) == 48, "PrefillItem layout");
+
+struct alignas(16) TableHeader {
+  int32_t magic;
+  int32_t version;
+  int32_t n_heads;
+  int32_t n_vpages;
+  int32_t n_decode_items;
+  int32_t n_decode_ctas;
+  int32_t n_combine;
+  int32_t n_prefill_items;
+  int64_t off_heads, off_pages, off_decode_items, off_decode_cta, off_combine, off_prefill;
+};
+
+}  // namespace sp
+
+// The plan: a host copy of the problem plus the table blob.
+struct sp_plan {
+  sp_problem prob{};                      // pointers inside are cleared after copying
+  std::vector<int32_t> ctx_len, q_start;
+  std::vector<sp_head_policy> policy;
+  std::vector<sp_segment> segments;       // per head: up to two, flattened
+  std::vector<int32_t> seg_begin;         // [n_heads + 1]
+  std::vector<sp::HeadDesc> heads;
+  std::vector<sp::PageDesc> pages;
+  std::vector<sp::DecodeItem> decode_items;
+  std::vector<int32_t> decode_cta_begin;  // [n_ctas + 1] item ranges per CTA
+  std::vector<sp::CombineItem> combine;
+  std::vector<sp::PrefillItem> prefill;
+  std::vector<uint8_t> blob;              // header + arrays, 256-byte aligned sections
+  sp::TableHeader hdr{};
+  sp_sizes sizes{};
+  int32_t group = 1;
+  int32_t elem_bytes = 4;
+  int32_t prefill_tile = 0;
+  int32_t n_partial_slots = 0;
+};
+
+namespace sp {
+void set_error(const std::string& msg);
+sp_status fail(sp_status st, const std::string& msg);
+}  // namespace sp

@@ -1,0 +1,107 @@
+"""PyTorch-facing wrapper of one SegPaged layer (buffers + calls, nothing else).
+
+``SegPagedLayer`` owns the device buffers a plan needs (table blob, K/V
+pools, workspace) as PyTorch tensors and forwards to the C ABI.  It performs
+no arithmetic of the method: planning, packing and attention all run in
+libsegpaged.so.
+"""
+from __future__ import annotations
+
+from typing import Sequence
+
+import torch
+
+from . import segpaged as S
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class SegPagedLayer:
+    """Plan + device buffers of one attention layer's batch.
+
+    ``policy`` holds ``(kind, sink, window)`` per (sequence, kv-head) with kind
+    in {"global", "local", "dense"}; ``q_start[b]`` is the position of the
+    first query of sequence b (``ctx_len[b] - 1`` for decode).
+    """
+
+    def __init__(self, *, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, page_size: int,
+                 dtype: str, ctx_len: Sequence[int], q_start: Sequence[int],
+                 policy: Sequence[tuple[str, int, int]], device="cuda", flags: int = 0,
+                 page_ids: Sequence[int] | None = None, first_page: int = 0, target_ctas: int = 0,
+                 pools: tuple[torch.Tensor, torch.Tensor] | None = None):
+        self.dtype = dtype
+        self.torch_dtype = {"f32": torch.float32, "bf16": torch.bfloat16}[dtype]
+        self.num_q_heads, self.num_kv_heads, self.head_dim = num_q_heads, num_kv_heads, head_dim
+        self.device = torch.device(device)
+        self.problem = S.make_problem(batch, num_q_heads, num_kv_heads, head_dim, page_size, dtype, ctx_len,
+                                      q_start, policy, first_page, page_ids, target_ctas, flags)
+        self.plan = S.segpaged_plan_create(self.problem)
+        self.sizes = S.segpaged_plan_sizes(self.plan)
+        z = self.sizes
+        self.table = torch.empty(z.table_bytes, dtype=torch.uint8, device=self.device)
+        S.segpaged_table_write(self.plan, self.table.data_ptr(), z.table_bytes, _stream(None))
+        if pools is None:
+            nbytes = z.pool_pages * z.page_bytes
+            self.k_pool = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=self.device)
+            self.v_pool = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=self.device)
+        else:
+            self.k_pool, self.v_pool = pools
+        self.workspace = torch.zeros(z.workspace_bytes, dtype=torch.uint8, device=self.device)
+
+    # -- calls --------------------------------------------------------------
+    def build(self, k_dense: torch.Tensor, v_dense: torch.Tensor, varlen: bool = False, stream=None) -> None:
+        """Pack dense K/V ([B, Hkv, Lmax, d], or varlen [sum L, Hkv, d] with varlen=True)."""
+        if varlen:
+            ss, sh, st = S.SP_VARLEN, k_dense.stride(1), k_dense.stride(0)
+        else:
+            ss, sh, st = k_dense.stride(0), k_dense.stride(1), k_dense.stride(2)
+        assert k_dense.stride() == v_dense.stride() and k_dense.stride(-1) == 1
+        S.build_segpaged_cache(self.plan, self.table.data_ptr(), k_dense.data_ptr(), v_dense.data_ptr(), ss, sh,
+                               st, self.k_pool.data_ptr(), self.v_pool.data_ptr(), _stream(stream))
+
+    def gather(self, k_out: torch.Tensor, v_out: torch.Tensor, varlen: bool = False, stream=None) -> None:
+        if varlen:
+            ss, sh, st = S.SP_VARLEN, k_out.stride(1), k_out.stride(0)
+        else:
+            ss, sh, st = k_out.stride(0), k_out.stride(1), k_out.stride(2)
+        S.segpaged_gather(self.plan, self.table.data_ptr(), self.k_pool.data_ptr(), self.v_pool.data_ptr(),
+                          k_out.data_ptr(), v_out.data_ptr(), ss, sh, st, _stream(stream))
+
+    def attention(self, q: torch.Tensor, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                  scale: float = 0.0, with_lse: bool = True, stream=None):
+        """q: [sum C_b, Hq, d] contiguous; returns (out, lse)."""
+        assert q.is_contiguous() and q.dtype == self.torch_dtype
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None and with_lse:
+            lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device)
+        S.segpaged_attention(self.plan, self.table.data_ptr(), self.k_pool.data_ptr(), self.v_pool.data_ptr(),
+                             q.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None, scale,
+                             self.workspace.data_ptr(), self.workspace.numel(), _stream(stream))
+        return out, lse
+
+    def device_status(self, stream=None) -> int:
+        return S.segpaged_read_device_status(self.workspace.data_ptr(), _stream(stream))
+
+    def close(self) -> None:
+        if getattr(self, "plan", None):
+            S.segpaged_plan_destroy(self.plan)
+            self.plan = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def layer_for(prob, device="cuda", flags: int = 0, **kw) -> SegPagedLayer:
+    """A SegPagedLayer for a ``workloads.Problem``."""
+    wl = prob.wl
+    return SegPagedLayer(batch=wl.batch, num_q_heads=wl.num_q_heads, num_kv_heads=wl.num_kv_heads,
+                         head_dim=wl.head_dim, page_size=wl.page_size, dtype=wl.dtype, ctx_len=prob.ctx_lens,
+                         q_start=prob.q_starts, policy=wl.policy, device=device, flags=flags, **kw)

@@ -1,0 +1,226 @@
+"""Python binding of libsegpaged.so (ctypes; argument marshalling only).
+
+Every function here has the name of a C entry point in ``include/segpaged.h``
+and forwards to it; no step of the attention path runs in Python.  Device
+buffers are passed as raw pointers (``int`` addresses, e.g. ``tensor.data_ptr()``)
+and streams as ``cudaStream_t`` handles (``torch.cuda.Stream.cuda_stream``).
+
+Loading fails loudly when the compiled library is missing: there is no CPU
+or library fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+from typing import Sequence
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libsegpaged.so"
+
+SP_OK, SP_ERR_INVALID_ARG, SP_ERR_UNSUPPORTED, SP_ERR_WORKSPACE, SP_ERR_CUDA, SP_ERR_DEVICE_CHECK = range(6)
+SP_GLOBAL, SP_LOCAL, SP_DENSE, SP_RETRIEVAL = range(4)
+SP_F32, SP_BF16 = 0, 1
+SP_FLAG_DENSE_MASKED = 1
+SP_VARLEN = -1
+KIND_CODES = {"global": SP_GLOBAL, "local": SP_LOCAL, "dense": SP_DENSE, "retrieval": SP_RETRIEVAL}
+DTYPE_CODES = {"f32": SP_F32, "bf16": SP_BF16}
+
+# every symbol include/segpaged.h declares
+EXPORTED = ("segpaged_plan_create", "segpaged_plan_destroy", "segpaged_plan_sizes",
+            "segpaged_plan_head_segments", "segpaged_plan_head_pages", "segpaged_table_write",
+            "build_segpaged_cache", "segpaged_gather", "segpaged_attention",
+            "segpaged_read_device_status", "segpaged_clear_device_status", "segpaged_status_string",
+            "segpaged_last_error", "segpaged_abi_version")
+
+
+class SegPagedError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {status_name(status)}: {detail}")
+
+
+class sp_head_policy(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("sink", ctypes.c_int32), ("window", ctypes.c_int32)]
+
+
+class sp_problem(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("ctx_len", ctypes.POINTER(ctypes.c_int32)), ("q_start", ctypes.POINTER(ctypes.c_int32)),
+                ("policy", ctypes.POINTER(sp_head_policy)), ("first_page", ctypes.c_int64),
+                ("page_ids", ctypes.POINTER(ctypes.c_int32)), ("target_ctas", ctypes.c_int32),
+                ("flags", ctypes.c_uint32)]
+
+
+class sp_sizes(ctypes.Structure):
+    _fields_ = [("num_pages", ctypes.c_int64), ("pool_pages", ctypes.c_int64), ("page_bytes", ctypes.c_int64),
+                ("table_bytes", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64),
+                ("stored_token_heads", ctypes.c_int64), ("dense_token_heads", ctypes.c_int64),
+                ("visible_pairs", ctypes.c_int64), ("num_queries", ctypes.c_int64), ("is_decode", ctypes.c_int32),
+                ("num_decode_ctas", ctypes.c_int32), ("num_prefill_items", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_ if name != "reserved"}
+
+
+class sp_segment(ctypes.Structure):
+    _fields_ = [("abs_start", ctypes.c_int32), ("length", ctypes.c_int32), ("first_page_index", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load(path: Path | str | None = None) -> ctypes.CDLL:
+    """Load libsegpaged.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = Path(path) if path else LIB_PATH
+    if not p.exists():
+        raise ImportError(f"{p} is missing: build it with head_aware_paged_build_b200.build_ext.build() "
+                          "(there is no fallback path)")
+    lib = ctypes.CDLL(str(p))
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "segpaged_plan_create": ([ctypes.POINTER(sp_problem), ctypes.POINTER(vp)], i32),
+        "segpaged_plan_destroy": ([vp], None),
+        "segpaged_plan_sizes": ([vp, ctypes.POINTER(sp_sizes)], i32),
+        "segpaged_plan_head_segments": ([vp, i32, i32, ctypes.POINTER(sp_segment), i32, ctypes.POINTER(i32)], i32),
+        "segpaged_plan_head_pages": ([vp, i32, i32, ctypes.POINTER(i64), i32, ctypes.POINTER(i32)], i32),
+        "segpaged_table_write": ([vp, vp, sz, vp], i32),
+        "build_segpaged_cache": ([vp, vp, vp, vp, i64, i64, i64, vp, vp, vp], i32),
+        "segpaged_gather": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
+        "segpaged_attention": ([vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp], i32),
+        "segpaged_read_device_status": ([vp, ctypes.POINTER(i32), vp], i32),
+        "segpaged_clear_device_status": ([vp, vp], i32),
+        "segpaged_status_string": ([i32], ctypes.c_char_p),
+        "segpaged_last_error": ([], ctypes.c_char_p),
+        "segpaged_abi_version": ([], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_name(st: int) -> str:
+    return load().segpaged_status_string(st).decode()
+
+
+def last_error() -> str:
+    return load().segpaged_last_error().decode()
+
+
+def _check(st: int, where: str) -> None:
+    if st != SP_OK:
+        raise SegPagedError(st, where, last_error())
+
+
+# ---------------------------------------------------------------------------
+# Thin wrappers with the C names
+# ---------------------------------------------------------------------------
+
+def make_problem(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, page_size: int, dtype: str,
+                 ctx_len: Sequence[int], q_start: Sequence[int], policy: Sequence[tuple[str, int, int]],
+                 first_page: int = 0, page_ids: Sequence[int] | None = None, target_ctas: int = 0,
+                 flags: int = 0):
+    """Build an ``sp_problem`` plus the host arrays it points to (kept alive in the result)."""
+    B = batch
+    ctx = (ctypes.c_int32 * B)(*ctx_len)
+    q0 = (ctypes.c_int32 * B)(*q_start)
+    pol = (sp_head_policy * len(policy))(*[sp_head_policy(KIND_CODES[k] if isinstance(k, str) else k, s, w)
+                                           for k, s, w in policy])
+    ids = (ctypes.c_int32 * len(page_ids))(*page_ids) if page_ids is not None else None
+    prob = sp_problem(B, num_q_heads, num_kv_heads, head_dim, page_size,
+                      DTYPE_CODES[dtype] if isinstance(dtype, str) else dtype,
+                      ctx, q0, pol, first_page,
+                      ctypes.cast(ids, ctypes.POINTER(ctypes.c_int32)) if ids is not None else None,
+                      target_ctas, flags)
+    prob._keep = (ctx, q0, pol, ids)
+    return prob
+
+
+def segpaged_plan_create(problem: sp_problem) -> int:
+    out = ctypes.c_void_p()
+    _check(load().segpaged_plan_create(ctypes.byref(problem), ctypes.byref(out)), "segpaged_plan_create")
+    return out.value
+
+
+def segpaged_plan_create_status(problem: sp_problem) -> tuple[int, int | None]:
+    """Like segpaged_plan_create but returns (status, plan) instead of raising."""
+    out = ctypes.c_void_p()
+    st = load().segpaged_plan_create(ctypes.byref(problem), ctypes.byref(out))
+    return st, out.value
+
+
+def segpaged_plan_destroy(plan: int) -> None:
+    load().segpaged_plan_destroy(plan)
+
+
+def segpaged_plan_sizes(plan: int) -> sp_sizes:
+    z = sp_sizes()
+    _check(load().segpaged_plan_sizes(plan, ctypes.byref(z)), "segpaged_plan_sizes")
+    return z
+
+
+def segpaged_plan_head_segments(plan: int, b: int, kv: int) -> list[tuple[int, int, int, int]]:
+    n = ctypes.c_int32()
+    segs = (sp_segment * 4)()
+    _check(load().segpaged_plan_head_segments(plan, b, kv, segs, 4, ctypes.byref(n)), "segpaged_plan_head_segments")
+    return [(s.abs_start, s.length, s.first_page_index, s.num_pages) for s in segs[: n.value]]
+
+
+def segpaged_plan_head_pages(plan: int, b: int, kv: int) -> list[int]:
+    n = ctypes.c_int32()
+    _check(load().segpaged_plan_head_pages(plan, b, kv, None, 0, ctypes.byref(n)), "segpaged_plan_head_pages")
+    ids = (ctypes.c_int64 * max(1, n.value))()
+    _check(load().segpaged_plan_head_pages(plan, b, kv, ids, n.value, ctypes.byref(n)), "segpaged_plan_head_pages")
+    return list(ids[: n.value])
+
+
+def segpaged_table_write(plan: int, d_table: int, nbytes: int, stream: int = 0) -> None:
+    _check(load().segpaged_table_write(plan, d_table, nbytes, stream), "segpaged_table_write")
+
+
+def build_segpaged_cache(plan: int, d_table: int, k_dense: int, v_dense: int, stride_seq: int, stride_head: int,
+                         stride_tok: int, k_pool: int, v_pool: int, stream: int = 0) -> None:
+    _check(load().build_segpaged_cache(plan, d_table, k_dense, v_dense, stride_seq, stride_head, stride_tok,
+                                       k_pool, v_pool, stream), "build_segpaged_cache")
+
+
+def segpaged_gather(plan: int, d_table: int, k_pool: int, v_pool: int, k_out: int, v_out: int, stride_seq: int,
+                    stride_head: int, stride_tok: int, stream: int = 0) -> None:
+    _check(load().segpaged_gather(plan, d_table, k_pool, v_pool, k_out, v_out, stride_seq, stride_head,
+                                  stride_tok, stream), "segpaged_gather")
+
+
+def segpaged_attention(plan: int, d_table: int, k_pool: int, v_pool: int, q: int, out: int, lse: int | None,
+                       softmax_scale: float, workspace: int, workspace_bytes: int, stream: int = 0) -> None:
+    _check(load().segpaged_attention(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale, workspace,
+                                     workspace_bytes, stream), "segpaged_attention")
+
+
+def segpaged_attention_status(*args) -> int:
+    """Like segpaged_attention but returns the status code instead of raising."""
+    return load().segpaged_attention(*args)
+
+
+def segpaged_read_device_status(workspace: int, stream: int = 0) -> int:
+    code = ctypes.c_int32()
+    st = load().segpaged_read_device_status(workspace, ctypes.byref(code), stream)
+    if st not in (SP_OK, SP_ERR_DEVICE_CHECK):
+        _check(st, "segpaged_read_device_status")
+    return code.value
+
+
+def segpaged_clear_device_status(workspace: int, stream: int = 0) -> None:
+    _check(load().segpaged_clear_device_status(workspace, stream), "segpaged_clear_device_status")
+
+
+def segpaged_abi_version() -> int:
+    return load().segpaged_abi_version()

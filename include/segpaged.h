@@ -1,0 +1,221 @@
+/*
+ * segpaged.h — C ABI of libsegpaged.so, head-aware paged KV attention
+ * (SegPagedAttention) for NVIDIA B200 (sm_100a).
+ *
+ * The KV cache is paged per (sequence, kv-head, segment).  Every kv-head
+ * follows its own policy: a GLOBAL head stores and reads its whole causal
+ * context; a LOCAL head stores and reads only the first `sink` tokens of the
+ * sequence plus its `window` most recent tokens.  Attention evaluates every
+ * (query-head, kv-head) pair over exactly the tokens that head stores, with no
+ * mask over tokens it cannot see ("SegPagedAttention runtime design", §1 why
+ * heads see different contexts, §3 per-head page tables, §4 mask-free fused
+ * kernel; "RedKnot head classification", four head kinds).
+ *
+ * Conventions shared by every call:
+ *  - Device memory (K/V pools, the table blob, workspace, Q/K/V/O tensors) is
+ *    owned by the caller.  Pointers are borrowed for the duration of the call.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Device calls only enqueue work and return; nothing synchronises
+ *    except segpaged_read_device_status.
+ *  - Every argument and layout error is detected on the host before any launch
+ *    and leaves every output untouched.  No C++ exception crosses the ABI.
+ *    segpaged_last_error() returns a message for the calling thread's last
+ *    failure.
+ *  - Positions are 0-based absolute positions in a sequence.  Query q-head h
+ *    uses kv-head h / (num_q_heads / num_kv_heads).
+ *  - Supported: head_dim 64 or 128; dtype fp32 with page size 16 or 64; dtype
+ *    bf16 with page size 64; num_q_heads / num_kv_heads <= 16.  Anything else
+ *    returns SP_ERR_UNSUPPORTED.
+ */
+#ifndef SEGPAGED_H_
+#define SEGPAGED_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SP_API __attribute__((visibility("default")))
+#else
+#define SP_API
+#endif
+
+#define SEGPAGED_ABI_VERSION 1
+
+/* stride_seq value selecting sequences packed back to back (varlen). */
+#define SP_VARLEN (-1)
+
+typedef enum {
+  SP_OK = 0,
+  SP_ERR_INVALID_ARG = 1,  /* malformed sizes, positions, policies, pointers or strides */
+  SP_ERR_UNSUPPORTED = 2,  /* valid request outside the supported shapes / kinds / dtypes */
+  SP_ERR_WORKSPACE = 3,    /* table or workspace buffer smaller than the plan needs */
+  SP_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  SP_ERR_DEVICE_CHECK = 5  /* a kernel recorded an error in the workspace status word */
+} sp_status;
+
+/* Head kinds ("RedKnot head classification", four-kind table).  DENSE reads
+ * the full causal context like GLOBAL (its RoPE re-alignment belongs to KV
+ * reuse, outside attention).  RETRIEVAL (top-p token selection) is not
+ * implemented: the pages give no scoring rule; it returns SP_ERR_UNSUPPORTED. */
+typedef enum { SP_GLOBAL = 0, SP_LOCAL = 1, SP_DENSE = 2, SP_RETRIEVAL = 3 } sp_kind;
+
+typedef enum { SP_F32 = 0, SP_BF16 = 1 } sp_dtype;
+
+/* Problem flags. */
+enum {
+  /* Dense-plus-mask baseline: every head stores its whole context [0, L) and
+   * the kernels visit every causal tile, masking LOCAL heads per element
+   * ("SegPagedAttention runtime design", §4 verify_against_dense and §5: the
+   * dense baseline the speedups are quoted against). */
+  SP_FLAG_DENSE_MASKED = 1u
+};
+
+/* Policy of one (sequence, kv-head).  `sink` >= 0 and `window` >= 1 are read
+ * for SP_LOCAL only. */
+typedef struct {
+  int32_t kind;
+  int32_t sink;
+  int32_t window;
+} sp_head_policy;
+
+/* One attention layer's batch.  All arrays are host memory, copied by
+ * segpaged_plan_create.
+ *   ctx_len[b]  L_b >= 1, tokens of sequence b in the cache (queries included)
+ *   q_start[b]  q0_b in [0, L_b): the call's queries sit at q0_b .. L_b - 1, so
+ *               C_b = L_b - q0_b queries; every C_b == 1 makes a decode plan.
+ *   policy      [batch * num_kv_heads], (b, kv) order
+ *   first_page  physical page id of the plan's first page, so that several
+ *               layers' plans can share one pool
+ *   page_ids    NULL, or [num_pages] distinct non-negative ids (logical page i
+ *               goes to physical page first_page + page_ids[i]); num_pages is
+ *               reported by segpaged_plan_sizes of a plan made with NULL
+ *   target_ctas decode work is split into this many equal page ranges; 0 picks
+ *               2 x 148 (two CTAs on each B200 SM)
+ */
+typedef struct {
+  int32_t batch;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t page_size;
+  int32_t dtype; /* sp_dtype */
+  const int32_t* ctx_len;
+  const int32_t* q_start;
+  const sp_head_policy* policy;
+  int64_t first_page;
+  const int32_t* page_ids;
+  int32_t target_ctas;
+  uint32_t flags;
+} sp_problem;
+
+typedef struct {
+  int64_t num_pages;          /* pages the plan owns in each of the K and V pools */
+  int64_t pool_pages;         /* pages each pool must hold: first_page + max id + 1 */
+  int64_t page_bytes;         /* bytes of one page = page_size * head_dim * element size */
+  int64_t table_bytes;        /* size of the device table blob */
+  int64_t workspace_bytes;    /* workspace segpaged_attention needs (>= 256) */
+  int64_t stored_token_heads; /* (position, kv-head) rows held in the cache */
+  int64_t dense_token_heads;  /* sum over (b, kv) of L_b: rows a dense cache holds */
+  int64_t visible_pairs;      /* sum over (b, q-head, query p) of |visible set of p| */
+  int64_t num_queries;        /* sum_b C_b */
+  int32_t is_decode;          /* 1 if every C_b == 1 */
+  int32_t num_decode_ctas;    /* decode grid size (0 for prefill plans) */
+  int32_t num_prefill_items;  /* prefill grid size (0 for decode plans) */
+  int32_t reserved;
+} sp_sizes;
+
+/* One contiguous run of stored positions of a head; it starts on a fresh page. */
+typedef struct {
+  int32_t abs_start; /* first absolute position */
+  int32_t length;    /* number of positions */
+  int32_t first_page_index; /* index into the head's page list */
+  int32_t num_pages;
+} sp_segment;
+
+typedef struct sp_plan sp_plan;
+
+/* Build the SegmentPageTable of a batch ("SegPagedAttention runtime design",
+ * §3 SegmentPageTable: page ids per head segment plus per-head policy).  Host
+ * only, no CUDA call.  For each (b, kv): GLOBAL/DENSE keep one segment
+ * [0, L); LOCAL keeps [0, min(sink, L)) and [max(sink, q0 - window + 1), L),
+ * the union of what the call's queries see (merged when they touch).  Each
+ * segment starts on a fresh page.  The plan also holds the decode split list
+ * and the prefill tile list, so that no layout work happens per attention
+ * call (same page, §5: layout computed on every call cost a 0.70x slowdown).
+ * The plan is immutable and may be shared by several streams. */
+SP_API sp_status segpaged_plan_create(const sp_problem* problem, sp_plan** out);
+SP_API void segpaged_plan_destroy(sp_plan* plan);
+SP_API sp_status segpaged_plan_sizes(const sp_plan* plan, sp_sizes* out);
+
+/* Inspect the segments / physical page ids of (b, kv).  *count receives the
+ * number available; at most `max` are written. */
+SP_API sp_status segpaged_plan_head_segments(const sp_plan* plan, int32_t b, int32_t kv,
+                                      sp_segment* segs, int32_t max, int32_t* count);
+SP_API sp_status segpaged_plan_head_pages(const sp_plan* plan, int32_t b, int32_t kv, int64_t* page_ids,
+                                   int32_t max, int32_t* count);
+
+/* Copy the plan's table blob to `d_table` (device, >= table_bytes, 16-byte
+ * aligned) with an asynchronous host-to-device copy on `stream`. */
+SP_API sp_status segpaged_table_write(const sp_plan* plan, void* d_table, size_t bytes, void* stream);
+
+/* build_segpaged_cache ("SegPagedAttention runtime design", §3: build the
+ * per-head store from dense KV, keeping only the tokens each head can see).
+ * Copies, bit for bit, every stored (b, kv, position) row of the dense K and
+ * V into the pools; unused slots of a segment's last page are zeroed.
+ *   k_dense, v_dense  device, element (b, kv, t, i) at
+ *                     base + seq_off(b) + kv*stride_head + t*stride_tok + i
+ *                     (elements), with seq_off(b) = b*stride_seq, or, when
+ *                     stride_seq == SP_VARLEN, (L_0 + ... + L_{b-1})*stride_tok
+ *                     (sequences packed back to back in token order).
+ *                     Covers [B,Hkv,Lmax,d] (stride_tok = d) and varlen
+ *                     [sum L, Hkv, d] (stride_tok = Hkv*d, SP_VARLEN) layouts.
+ *   k_pool, v_pool    device, pool_pages * page_bytes each, 16-byte aligned.
+ * Base pointers and strides must give 16-byte aligned rows. */
+SP_API sp_status build_segpaged_cache(const sp_plan* plan, const void* d_table, const void* k_dense,
+                               const void* v_dense, int64_t stride_seq, int64_t stride_head,
+                               int64_t stride_tok, void* k_pool, void* v_pool, void* stream);
+
+/* Inverse of build_segpaged_cache, for checking: writes each stored row back
+ * into dense-shaped k_out / v_out (same addressing rules); rows that are not
+ * stored are left untouched. */
+SP_API sp_status segpaged_gather(const sp_plan* plan, const void* d_table, const void* k_pool,
+                          const void* v_pool, void* k_out, void* v_out, int64_t stride_seq,
+                          int64_t stride_head, int64_t stride_tok, void* stream);
+
+/* segpaged_attention ("SegPagedAttention runtime design", §4, the paper's
+ * Algorithm 2: read each head's true KV length from the page table, evaluate
+ * all (query-head, kv-head) pairs in one launch at their own lengths, no
+ * mask over invisible KV).
+ *   q    device [sum_b C_b, num_q_heads, head_dim], rows in sequence order,
+ *        row i of sequence b at position q0_b + i; dtype of the plan
+ *   out  device, same shape and dtype as q
+ *   lse  device [sum_b C_b, num_q_heads] fp32 natural-log sum-exp, or NULL
+ *   softmax_scale  <= 0 selects 1/sqrt(head_dim)
+ *   workspace      device, >= workspace_bytes, 256-byte aligned; its first
+ *                  256 bytes hold the device status word
+ * Decode plans run a split-KV kernel over each head's own pages plus a
+ * combine pass; prefill plans run one tile kernel (tcgen05 for bf16). */
+SP_API sp_status segpaged_attention(const sp_plan* plan, const void* d_table, const void* k_pool,
+                             const void* v_pool, const void* q, void* out, float* lse,
+                             float softmax_scale, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* Device status word: kernels never trap; a failed device-side check or a
+ * bounded wait that ran out records a non-zero code.  read synchronises
+ * `stream` and returns the code in *code (0 = no error); clear zeroes it. */
+SP_API sp_status segpaged_read_device_status(const void* workspace, int32_t* code, void* stream);
+SP_API sp_status segpaged_clear_device_status(void* workspace, void* stream);
+
+SP_API const char* segpaged_status_string(sp_status status);
+SP_API const char* segpaged_last_error(void);
+SP_API int32_t segpaged_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEGPAGED_H_ */

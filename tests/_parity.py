@@ -1,0 +1,79 @@
+"""Helpers of the GPU parity tests: run the oracle on the exact inputs the GPU used."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle
+
+# Tolerances of the attention outputs against the fp64 oracle: per-head
+# cosine >= 0.99998 ("SegPagedAttention runtime design", §4 verify_against_dense)
+# and a max absolute error of 1e-5 for fp32 inputs, 2e-2 for bf16 inputs (fp32
+# accumulation in both).  LSE: 1e-5 (fp32); 2e-3 (bf16): scores are exact
+# products of bf16 values summed in fp32 (relative error ~d * 2^-24) and the
+# softmax sums use the unrounded fp32 weights, so the bf16 LSE error is set by
+# fp32 accumulation and the SFU exp2, far below 2e-3 at |s| < 60.
+TOL = {"f32": dict(cos=0.99998, abs=1e-5, lse=1e-5), "bf16": dict(cos=0.99998, abs=2e-2, lse=2e-3)}
+
+
+def oracle_rows(prob, q_host, k_host, v_host, b, h, rows=None):
+    """Oracle output for (sequence b, q-head h) at varlen rows `rows` (indices within the sequence)."""
+    wl = prob.wl
+    kv = h // wl.group
+    kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+    L, q0 = prob.ctx_lens[b], prob.q_starts[b]
+    C = L - q0
+    rows = np.arange(C) if rows is None else np.asarray(rows)
+    off = prob.q_offsets[b]
+    q = q_host[off + rows, h].double().numpy()
+    k = k_host[b, kv, :L].double().numpy()
+    v = v_host[b, kv, :L].double().numpy()
+    return oracle.attention_rows(q, q0 + rows, k, v, kind, s, w)
+
+
+def compare(prob, q_host, k_host, v_host, out, lse, rows_per_seq=None, heads=None):
+    """Compare GPU out / lse (device or host tensors) with the oracle.
+
+    Returns dict(min_cos, max_abs, max_lse, worst) over the checked (b, h).
+    """
+    wl = prob.wl
+    out_h = out.float().cpu()
+    lse_h = lse.float().cpu() if lse is not None else None
+    heads = range(wl.num_q_heads) if heads is None else heads
+    min_cos, max_abs, max_lse, worst = 1.0, 0.0, 0.0, None
+    for b in range(wl.batch):
+        rows = None if rows_per_seq is None else rows_per_seq[b]
+        C = prob.ctx_lens[b] - prob.q_starts[b]
+        ridx = np.arange(C) if rows is None else np.asarray(rows)
+        off = prob.q_offsets[b]
+        for h in heads:
+            o_ref, l_ref = oracle_rows(prob, q_host, k_host, v_host, b, h, ridx)
+            o = out_h[off + ridx, h].double().numpy()
+            a, r = o.ravel(), o_ref.ravel()
+            cos = float(a @ r / (np.linalg.norm(a) * np.linalg.norm(r)))
+            err = float(np.max(np.abs(o - o_ref)))
+            if cos < min_cos:
+                min_cos, worst = cos, (b, h)
+            max_abs = max(max_abs, err)
+            if lse_h is not None:
+                max_lse = max(max_lse, float(np.max(np.abs(lse_h[off + ridx, h].double().numpy() - l_ref))))
+    return dict(min_cos=min_cos, max_abs=max_abs, max_lse=max_lse, worst=worst)
+
+
+def assert_close(res, dtype):
+    tol = TOL[dtype]
+    assert res["min_cos"] >= tol["cos"], res
+    assert res["max_abs"] <= tol["abs"], res
+    assert res["max_lse"] <= tol["lse"], res
+
+
+def sample_rows(C: int, page: int = 64, n_random: int = 16, seed: int = 0) -> np.ndarray:
+    """First / last rows, rows around multiples of 128, and seeded random rows of a chunk."""
+    rng = np.random.default_rng(seed)
+    pick = {0, 1, C - 1, C - 2}
+    for m in range(128, C, 128):
+        pick.update((m - 1, m, m + 1))
+    pick.update(int(x) for x in rng.integers(0, C, n_random))
+    return np.array(sorted(x for x in pick if 0 <= x < C))

@@ -1,0 +1,215 @@
+"""C-ABI library and host planner tests (no GPU: only host-side entry points run)."""
+from __future__ import annotations
+
+import re
+from pathlib import Path
+
+import numpy as np
+import pytest
+
+import oracle
+from head_aware_paged_build_b200 import build_ext
+from head_aware_paged_build_b200 import segpaged as S
+from head_aware_paged_build_b200 import workloads as W
+
+ROOT = Path(__file__).resolve().parent.parent
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build_ext.build()
+    return S.load()
+
+
+def header_symbols():
+    text = (ROOT / "include" / "segpaged.h").read_text()
+    return re.findall(r"SP_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_library_exports_every_header_symbol():
+    names = header_symbols()
+    assert len(names) == len(S.EXPORTED) and set(names) == set(S.EXPORTED)
+    lib = S.load()
+    for n in names:
+        assert getattr(lib, n) is not None
+    assert S.segpaged_abi_version() == 1
+    assert S.status_name(S.SP_ERR_WORKSPACE) == "SP_ERR_WORKSPACE"
+
+
+def plan_for(prob, **kw):
+    wl = prob.wl
+    p = S.make_problem(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.page_size, wl.dtype,
+                       prob.ctx_lens, prob.q_starts, wl.policy, **kw)
+    return S.segpaged_plan_create(p), p
+
+
+def oracle_stored(prob, dense_masked=False):
+    wl = prob.wl
+    n = 0
+    for b in range(wl.batch):
+        for kv in range(wl.num_kv_heads):
+            kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+            if dense_masked:
+                kind = "global"
+            n += int(oracle.stored_mask(kind, s, w, prob.ctx_lens[b], prob.q_starts[b]).sum())
+    return n
+
+
+@pytest.mark.parametrize("name", ["tiny", "mistral"])
+@pytest.mark.parametrize("mode", ["decode", "prefill"])
+def test_plan_sizes_match_oracle(name, mode):
+    wl = W.ALL[name]()
+    prob = wl.decode_problem() if mode == "decode" else wl.prefill_problem()
+    plan, _ = plan_for(prob)
+    try:
+        z = S.segpaged_plan_sizes(plan)
+        assert z.stored_token_heads == oracle_stored(prob)
+        assert z.dense_token_heads == sum(prob.ctx_lens) * wl.num_kv_heads
+        pairs = 0
+        for b in range(wl.batch):
+            for kv in range(wl.num_kv_heads):
+                kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+                pairs += oracle.visible_pairs(kind, s, w, prob.ctx_lens[b], prob.q_starts[b])
+        assert z.visible_pairs == pairs * wl.group
+        assert z.is_decode == (mode == "decode")
+        assert z.num_queries == prob.total_queries
+        elem = 2 if wl.dtype == "bf16" else 4
+        assert z.page_bytes == wl.page_size * wl.head_dim * elem
+        assert z.workspace_bytes >= 256 and z.workspace_bytes % 256 == 0
+    finally:
+        S.segpaged_plan_destroy(plan)
+
+
+def test_plan_sizes_of_large_layers_closed_form():
+    """Llama-70B-shaped: 721,120 stored token-heads at decode, 950,440 for the 4096-query chunk."""
+    for prob, want in ((W.llama().decode_problem(), 721_120), (W.llama().prefill_problem(), 950_440),
+                       (W.mha().decode_problem(), 4 * (8 * 131072 + 56 * 132))):
+        plan, _ = plan_for(prob)
+        z = S.segpaged_plan_sizes(plan)
+        assert z.stored_token_heads == want
+        S.segpaged_plan_destroy(plan)
+    wl = W.llama()
+    plan, _ = plan_for(wl.prefill_problem())
+    z = S.segpaged_plan_sizes(plan)
+    # visible FLOPs of the 4096-query chunk: 4 d sum |V(p)| = 1.1824e13
+    assert 4 * 128 * z.visible_pairs == pytest.approx(1.1824e13, rel=1e-4)
+    S.segpaged_plan_destroy(plan)
+
+
+def _random_policy_cases(n=60, seed=0):
+    rng = np.random.default_rng(seed)
+    for _ in range(n):
+        L = int(rng.integers(1, 300))
+        q0 = int(rng.integers(0, L))
+        kind = ["global", "local", "dense"][int(rng.integers(0, 3))]
+        s = int(rng.integers(0, 40))
+        w = int(rng.integers(1, 120))
+        yield L, q0, kind, s, w
+
+
+@pytest.mark.parametrize("page", [16, 64])
+@pytest.mark.parametrize("dense_masked", [False, True])
+def test_segments_hold_exactly_the_oracle_stored_set(page, dense_masked):
+    for L, q0, kind, s, w in _random_policy_cases(seed=page + dense_masked):
+        p = S.make_problem(1, 1, 1, 64, page, "f32", [L], [q0], [(kind, s, w)],
+                           flags=S.SP_FLAG_DENSE_MASKED if dense_masked else 0)
+        plan = S.segpaged_plan_create(p)
+        segs = S.segpaged_plan_head_segments(plan, 0, 0)
+        pages = S.segpaged_plan_head_pages(plan, 0, 0)
+        S.segpaged_plan_destroy(plan)
+        held = np.zeros(L, bool)
+        next_page = 0
+        for start, length, first_page, npages in segs:
+            assert length >= 1 and not held[start:start + length].any()
+            held[start:start + length] = True
+            assert first_page == next_page and npages == -(-length // page)
+            next_page += npages
+        assert len(pages) == next_page
+        want = oracle.stored_mask("global" if dense_masked else kind, s, w, L, q0)
+        assert np.array_equal(held, want), (L, q0, kind, s, w, segs)
+
+
+def test_page_ids_first_page_and_permutation():
+    wl = W.tiny()
+    prob = wl.decode_problem()
+    plan, _ = plan_for(prob)
+    n = S.segpaged_plan_sizes(plan).num_pages
+    S.segpaged_plan_destroy(plan)
+    perm = list(np.random.default_rng(3).permutation(n))
+    plan, _ = plan_for(prob, first_page=7, page_ids=perm)
+    z = S.segpaged_plan_sizes(plan)
+    assert z.pool_pages == 7 + n and z.num_pages == n
+    got = S.segpaged_plan_head_pages(plan, 0, 0) + S.segpaged_plan_head_pages(plan, 0, 1)
+    assert got == [7 + int(x) for x in perm]
+    S.segpaged_plan_destroy(plan)
+    bad = S.make_problem(1, 4, 2, 64, 16, "f32", prob.ctx_lens, prob.q_starts, wl.policy,
+                         page_ids=[0] * n)
+    st, _ = S.segpaged_plan_create_status(bad)
+    assert st == S.SP_ERR_INVALID_ARG and "distinct" in S.last_error()
+
+
+BASE = dict(batch=1, num_q_heads=4, num_kv_heads=2, head_dim=64, page_size=16, dtype="f32", ctx_len=[100],
+            q_start=[99], policy=[("global", 0, 0), ("local", 4, 8)])
+
+
+@pytest.mark.parametrize("change,code", [
+    (dict(batch=0, ctx_len=[], q_start=[], policy=[]), S.SP_ERR_INVALID_ARG),
+    (dict(ctx_len=[0], q_start=[0]), S.SP_ERR_INVALID_ARG),
+    (dict(q_start=[100]), S.SP_ERR_INVALID_ARG),
+    (dict(q_start=[-1]), S.SP_ERR_INVALID_ARG),
+    (dict(policy=[("global", 0, 0), ("local", 4, 0)]), S.SP_ERR_INVALID_ARG),
+    (dict(policy=[("global", 0, 0), ("local", -1, 8)]), S.SP_ERR_INVALID_ARG),
+    (dict(policy=[("global", 0, 0), (7, 0, 8)]), S.SP_ERR_INVALID_ARG),
+    (dict(policy=[("global", 0, 0), ("retrieval", 0, 0)]), S.SP_ERR_UNSUPPORTED),
+    (dict(head_dim=96), S.SP_ERR_UNSUPPORTED),
+    (dict(dtype=5), S.SP_ERR_UNSUPPORTED),
+    (dict(dtype="bf16"), S.SP_ERR_UNSUPPORTED),  # bf16 needs page 64
+    (dict(page_size=32), S.SP_ERR_UNSUPPORTED),
+    (dict(num_q_heads=5), S.SP_ERR_UNSUPPORTED),
+    (dict(num_q_heads=34, num_kv_heads=2), S.SP_ERR_UNSUPPORTED),
+])
+def test_plan_validation_errors(change, code):
+    args = dict(BASE)
+    args.update(change)
+    p = S.make_problem(**args)
+    st, plan = S.segpaged_plan_create_status(p)
+    assert st == code, S.last_error()
+    assert not plan
+    assert S.last_error()
+
+
+def test_unknown_flag_and_negative_first_page_rejected():
+    for kw in (dict(flags=4), dict(first_page=-1), dict(target_ctas=-2)):
+        p = S.make_problem(**BASE, **kw)
+        st, _ = S.segpaged_plan_create_status(p)
+        assert st == S.SP_ERR_INVALID_ARG
+
+
+def test_decode_split_uses_target_ctas():
+    wl = W.mistral()
+    prob = wl.decode_problem()
+    for target, want in ((0, 296), (10, 10), (100000, None)):
+        plan, _ = plan_for(prob, target_ctas=target)
+        z = S.segpaged_plan_sizes(plan)
+        assert z.num_decode_ctas == (want if want is not None else z.num_pages)
+        S.segpaged_plan_destroy(plan)
+
+
+def test_device_calls_reject_bad_arguments_before_launch():
+    """Host-side checks run before any CUDA call, so they work without a GPU."""
+    wl = W.tiny()
+    plan, _ = plan_for(wl.decode_problem())
+    z = S.segpaged_plan_sizes(plan)
+    lib = S.load()
+    # NULL table / misaligned pointers / short workspace never reach CUDA
+    assert lib.segpaged_attention(plan, None, 16, 16, 16, 16, None, 0.0, 256, z.workspace_bytes, None) \
+        == S.SP_ERR_INVALID_ARG
+    assert lib.segpaged_attention(plan, 256, 16, 16, 16, 16, None, 0.0, 256, 1, None) == S.SP_ERR_WORKSPACE
+    assert lib.segpaged_attention(plan, 256, 16, 16, 17, 16, None, 0.0, 256, z.workspace_bytes, None) \
+        == S.SP_ERR_INVALID_ARG
+    assert lib.segpaged_attention(plan, 256, 16, 16, 16, 16, None, float("nan"), 256, z.workspace_bytes, None) \
+        == S.SP_ERR_INVALID_ARG
+    assert lib.build_segpaged_cache(plan, 256, 16, 16, -5, 0, 64, 16, 16, None) == S.SP_ERR_INVALID_ARG
+    assert lib.build_segpaged_cache(plan, 256, 16, 16, 0, 0, 3, 16, 16, None) == S.SP_ERR_INVALID_ARG
+    assert lib.segpaged_table_write(plan, 256, 8, None) == S.SP_ERR_WORKSPACE
+    S.segpaged_plan_destroy(plan)

@@ -1,0 +1,110 @@
+"""build_segpaged_cache / segpaged_gather: bit-exact against the oracle's stored set."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from head_aware_paged_build_b200 import segpaged as S
+from head_aware_paged_build_b200 import workloads as W
+from head_aware_paged_build_b200.runtime import layer_for
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    S.load()
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    return t.view(torch.int16) if t.element_size() == 2 else t.view(torch.int32)
+
+
+def check_pack(prob, flags=0, **kw):
+    """Pack, gather into a sentinel-filled dense buffer, and compare bit for bit."""
+    wl = prob.wl
+    k, v = W.dense_kv(prob)
+    kd, vd = k.cuda(), v.cuda()
+    layer = layer_for(prob, flags=flags, **kw)
+    layer.build(kd, vd)
+    ko = torch.full_like(kd, float("nan"))
+    vo = torch.full_like(vd, float("nan"))
+    layer.gather(ko, vo)
+    torch.cuda.synchronize()
+    kb, vb, kob, vob = _bits(k), _bits(v), _bits(ko.cpu()), _bits(vo.cpu())
+    sentinel = _bits(torch.full((1,), float("nan"), dtype=k.dtype))[0]
+    dense_masked = bool(flags & S.SP_FLAG_DENSE_MASKED)
+    stored_total = 0
+    for b in range(wl.batch):
+        L, q0 = prob.ctx_lens[b], prob.q_starts[b]
+        for kv in range(wl.num_kv_heads):
+            kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+            m = oracle.stored_mask("global" if dense_masked else kind, s, w, L, q0)
+            mt = torch.from_numpy(m)
+            stored_total += int(m.sum())
+            assert torch.equal(kob[b, kv, :L][mt], kb[b, kv, :L][mt]), (b, kv)
+            assert torch.equal(vob[b, kv, :L][mt], vb[b, kv, :L][mt]), (b, kv)
+            assert bool((kob[b, kv, :L][~mt] == sentinel).all()), (b, kv)
+            assert bool((vob[b, kv, :L][~mt] == sentinel).all()), (b, kv)
+    assert stored_total == layer.sizes.stored_token_heads
+    return layer
+
+
+@pytest.mark.parametrize("name", ["tiny", "mistral"])
+@pytest.mark.parametrize("mode", ["decode", "prefill"])
+def test_pack_gather_bit_exact(name, mode):
+    wl = W.ALL[name]()
+    check_pack(wl.decode_problem() if mode == "decode" else wl.prefill_problem())
+
+
+def test_pack_dense_masked_keeps_everything():
+    check_pack(W.mistral().decode_problem(), flags=S.SP_FLAG_DENSE_MASKED)
+
+
+def test_pack_with_permuted_pages_and_offset_pool():
+    prob = W.tiny().decode_problem()
+    n = layer_for(prob).sizes.num_pages
+    perm = list(np.random.default_rng(1).permutation(n) * 2)  # sparse ids in a larger pool
+    check_pack(prob, first_page=3, page_ids=perm)
+
+
+@pytest.mark.parametrize("dtype,page,d", [("f32", 16, 64), ("f32", 64, 128), ("bf16", 64, 64), ("bf16", 64, 128)])
+def test_pack_ragged_edge_policies(dtype, page, d):
+    """Ragged lengths, partial pages, sink >= L, sink 0, window 1, windows wider than the context."""
+    lens = (1, 5, 63, 64, 65, 200, 130)
+    pol = []
+    for b, L in enumerate(lens):
+        pol += [("global", 0, 0), ("local", 4, 1), ("local", 0, 7), ("local", 70, 3), ("dense", 0, 0),
+                ("local", 3, 1000)]
+    wl = W.custom("edge", 11, len(lens), 6, 6, d, dtype, page, lens, pol, chunk=37)
+    check_pack(wl.decode_problem())
+    check_pack(wl.prefill_problem())
+
+
+def test_pack_varlen_layout_matches_padded():
+    wl = W.custom("var", 12, 3, 4, 2, 64, "bf16", 64, (100, 257, 64),
+                  [("global", 0, 0), ("local", 4, 16)] * 3)
+    prob = wl.decode_problem()
+    k, v = W.dense_kv(prob)
+    # varlen [sum L, Hkv, d]
+    kvar = torch.cat([k[b, :, :L].transpose(0, 1) for b, L in enumerate(prob.ctx_lens)]).contiguous().cuda()
+    vvar = torch.cat([v[b, :, :L].transpose(0, 1) for b, L in enumerate(prob.ctx_lens)]).contiguous().cuda()
+    a = layer_for(prob)
+    a.build(k.cuda(), v.cuda())
+    bl = layer_for(prob)
+    bl.build(kvar, vvar, varlen=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a.k_pool, bl.k_pool) and torch.equal(a.v_pool, bl.v_pool)
+    ko, vo = torch.zeros_like(kvar), torch.zeros_like(vvar)
+    bl.gather(ko, vo, varlen=True)
+    torch.cuda.synchronize()
+    for b, L in enumerate(prob.ctx_lens):
+        off = sum(prob.ctx_lens[:b])
+        for kv in range(2):
+            kind, s, w = wl.policy[b * 2 + kv]
+            m = torch.from_numpy(oracle.stored_mask(kind, s, w, L, L - 1)).cuda()
+            assert torch.equal(ko[off:off + L, kv][m], kvar[off:off + L, kv][m])
+            assert torch.equal(vo[off:off + L, kv][m], vvar[off:off + L, kv][m])
