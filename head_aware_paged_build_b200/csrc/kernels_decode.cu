@@ -119,7 +119,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
 
     for (int g = item.vp_begin; g < item.vp_end; ++g, ++k) {
       const int s = k % NST;
-      if (ok && !mbar_wait(&full[s], (k / NST) & 1)) {
+      // ldmatrix / mma.sync are warp-collective: the wait outcome is voted so the
+      // whole warp takes the same branch.
+      if (ok && !__all_sync(0xffffffffu, mbar_wait(&full[s], (k / NST) & 1))) {
         record_error(a.status, kDevTimeoutFull);
         ok = false;
       }
