@@ -1,0 +1,425 @@
+"""Benchmark of the SegPaged hot path on synthetic layers (one JSON line).
+
+One step = one pass of the whole path over one batch: build_segpaged_cache
+for the decode layout, decode attention, build_segpaged_cache for the
+prefill-chunk layout, prefill attention.  Inputs are resident in HBM; L2 is
+flushed (256 MB written, then 512 MB read so no dirty line is written back
+inside a timed kernel) before every timed kernel; each kernel is timed with
+CUDA events on the stream it is launched on.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama|mistral|mha|ragged]
+    python bench.py --impl reference ...   # the CPU oracle, timed on the host cores
+
+Under torchrun each rank runs its own batch (a different seed) on its own GPU:
+weak scaling with no collective on the data path; the timing is the max over
+ranks.  `value` is the decode visible-KV throughput; prefill TFLOP/s, the
+packing rate and the dense-plus-mask variant are reported beside it.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "SegPaged decode visible-KV GB/s (% HBM peak); prefill visible TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def peaks() -> dict:
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def workload(name: str, rank: int):
+    from head_aware_paged_build_b200 import workloads as W
+    wl = W.ALL[name]()
+    # weak scaling: every rank runs the same layer shape on its own batch
+    return dataclasses.replace(wl, seed=wl.seed + 7919 * rank) if rank else wl
+
+
+def config_of(wl, n_gpus: int) -> dict:
+    kinds = {}
+    for k, s, w in wl.policy:
+        kinds[k] = kinds.get(k, 0) + 1
+    loc = next(((s, w) for k, s, w in wl.policy if k == "local"), None)
+    return {
+        "workload": {"llama": "Llama-70B-shaped layer, 32K context", "mistral": "Mistral-7B-shaped layer, 8K context",
+                     "mha": "MHA-style layer, 128K context", "ragged": "ragged decode batch"}.get(
+                         wl.name.split("_")[0], wl.name),
+        "batch": wl.batch, "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+        "context": max(wl.ctx_lens), "page_size": wl.page_size, "prefill_chunk": wl.prefill_chunk,
+        "heads": {"global": kinds.get("global", 0), "local": kinds.get("local", 0)},
+        "local_sink_window": list(loc) if loc else None,
+        "inputs": "i.i.d. N(0,1) bf16, per-rank seed",
+        "l2": "flushed before every timed kernel (256 MB write + 512 MB read)",
+        "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def kernel_traffic(kernel: str, source: Path) -> int | None:
+    """DRAM bytes per launch from the last ncu capture, if the kernel source is unchanged since."""
+    p = ROOT / "profiles" / "traffic.json"
+    if not p.exists():
+        return None
+    rec = json.loads(p.read_text()).get(kernel)
+    if not rec:
+        return None
+    sha = hashlib.sha256(source.read_bytes()).hexdigest()[:16]
+    return int(rec["bytes_per_launch"]) if rec.get("source_sha16") == sha else None
+
+
+def run_ours(args) -> None:
+    import torch
+    import torch.distributed as dist
+
+    from head_aware_paged_build_b200 import workloads as W
+    from head_aware_paged_build_b200.runtime import layer_for
+    from head_aware_paged_build_b200 import segpaged as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = workload(args.workload, rank)
+    dec, pre = wl.decode_problem(), wl.prefill_problem()
+    k, v = W.dense_kv(dec, device=dev, gen_device=dev)
+    qd = W.queries(dec, device=dev, gen_device=dev)
+    qp = W.queries(pre, device=dev, gen_device=dev)
+    Ld = layer_for(dec, device=dev)
+    Lp = layer_for(pre, device=dev)
+    od, lsed = torch.empty_like(qd), torch.empty(qd.shape[:2], dtype=torch.float32, device=dev)
+    op, lsep = torch.empty_like(qp), torch.empty(qp.shape[:2], dtype=torch.float32, device=dev)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(128 << 20, dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_w.zero_()
+        flush_r.sum()
+
+    calls = [lambda: Ld.build(k, v), lambda: Ld.attention(qd, od, lsed), lambda: Lp.build(k, v),
+             lambda: Lp.attention(qp, op, lsep)]
+    names = ["pack_decode", "decode", "pack_prefill", "prefill"]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in calls]
+
+    def step(record: bool):
+        for i, c in enumerate(calls):
+            flush()
+            if record:
+                ev[i][0].record()
+            c()
+            if record:
+                ev[i][1].record()
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    for lay in (Ld, Lp):
+        assert lay.device_status() == 0, "device status word set during warm-up"
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    totals = [0.0] * len(calls)
+    wall0 = time.perf_counter()
+    for _ in range(args.steps):
+        step(True)
+        torch.cuda.synchronize()
+        for i in range(len(calls)):
+            totals[i] += ev[i][0].elapsed_time(ev[i][1])
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    t = torch.tensor([x / args.steps for x in totals], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = dict(zip(names, t.tolist()))
+
+    # ---- dense-plus-mask variant (same kernels, every head stores its whole context) ----
+    Ldm = layer_for(dec, device=dev, flags=S.SP_FLAG_DENSE_MASKED)
+    Lpm = layer_for(pre, device=dev, flags=S.SP_FLAG_DENSE_MASKED)
+    Ldm.build(k, v)
+    Lpm.build(k, v)
+    dm = {}
+    for nm, fn in (("decode", lambda: Ldm.attention(qd, od, lsed)), ("prefill", lambda: Lpm.attention(qp, op, lsep))):
+        fn()
+        vals = []
+        for _ in range(3 if nm == "prefill" else 10):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            vals.append(e0.elapsed_time(e1))
+        dm[nm] = statistics.median(vals)
+    dmt = torch.tensor([dm["decode"], dm["prefill"]], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(dmt, op=dist.ReduceOp.MAX)
+    dm = dict(zip(("decode", "prefill"), dmt.tolist()))
+    del Ldm, Lpm
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = run_e2e(args, dev, Ld, k, v, qd, od, lsed, world)
+
+    zd, zp = Ld.sizes, Lp.sizes
+    eb = 2
+    vis_dec = zd.stored_token_heads * 2 * wl.head_dim * eb          # K + V rows the decode must read
+    flops_pre = 4 * wl.head_dim * zp.visible_pairs                  # QK^T + PV on visible pairs
+    pack_bytes = lambda z: z.stored_token_heads * 2 * wl.head_dim * eb + 2 * z.num_pages * z.page_bytes
+    pk = peaks()
+    dec_gbs = world * vis_dec / (ms["decode"] * 1e-3) / 1e9
+    pre_tflops = world * flops_pre / (ms["prefill"] * 1e-3) / 1e12
+    launches_per_step = 1 + zd.kernel_launches() + 1 + zp.kernel_launches()
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    per_launch_pre = flops_pre / (ms["prefill"] * 1e-3) / 1e12
+    csrc = ROOT / "head_aware_paged_build_b200" / "csrc"
+    line = {
+        "metric": METRIC,
+        "value": round(dec_gbs, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(sum(ms.values()), 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": config_of(wl, world),
+        "decode": {"ms": round(ms["decode"], 5), "visible_kv_bytes": vis_dec, "GB/s": round(dec_gbs, 1),
+                   "frac_hbm": round(dec_gbs / world / pk["hbm_gbs"], 4), "launches": zd.kernel_launches()},
+        "prefill": {"ms": round(ms["prefill"], 4), "visible_flops": flops_pre, "TFLOP/s": round(pre_tflops, 1),
+                    "frac_bf16_burst": round(pre_tflops / world / pk["bf16_tflops"], 4),
+                    "frac_bf16_sustained": round(pre_tflops / world / pk["bf16_tflops_sustained"], 4)},
+        "pack": {"decode_ms": round(ms["pack_decode"], 5), "prefill_ms": round(ms["pack_prefill"], 5),
+                 "decode_GB/s": round(pack_bytes(zd) / (ms["pack_decode"] * 1e-3) / 1e9, 1),
+                 "prefill_GB/s": round(pack_bytes(zp) / (ms["pack_prefill"] * 1e-3) / 1e9, 1)},
+        "dense_masked": {"decode_ms": round(dm["decode"], 5), "prefill_ms": round(dm["prefill"], 4),
+                         "decode_skip": round(dm["decode"] / ms["decode"], 3),
+                         "prefill_skip": round(dm["prefill"] / ms["prefill"], 3),
+                         "kv_saving": round(1 - zd.stored_token_heads / zd.dense_token_heads, 4)},
+        "roofline": {"kernel": "prefill_tc_kernel", "bound": "tensor", "achieved": round(per_launch_pre, 1),
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(per_launch_pre / pk["bf16_tflops"], 4),
+                     "peak_source": f"{pk['source']} bf16 burst",
+                     "traffic": kernel_traffic("prefill_tc_kernel", csrc / "kernels_prefill_tc.cu")},
+        "roofline_decode": {"kernel": "decode_bf16_kernel + combine_kernel", "bound": "hbm",
+                            "achieved": round(vis_dec / (ms["decode"] * 1e-3) / 1e9, 1), "peak": pk["hbm_gbs"],
+                            "unit": "GB/s", "frac": round(vis_dec / (ms["decode"] * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                            "peak_source": f"{pk['source']} HBM copy",
+                            "traffic": kernel_traffic("decode_bf16_kernel", csrc / "kernels_decode.cu")},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "wall_s_timed": round(wall, 3),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, dec, k, v, qd, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, dev, layer, k, v, qd, od, lsed, world) -> dict:
+    """Decode through the public API with the step's inputs copied from pinned host memory."""
+    import torch
+    kh, vh, qh = (t.cpu().pin_memory() for t in (k, v, qd))
+    oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    lh = torch.empty(lsed.shape, dtype=lsed.dtype).pin_memory()
+    kd, vd, qdd = torch.empty_like(k), torch.empty_like(v), torch.empty_like(qd)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    for i in range(args.warmup + max(3, args.steps // 4)):
+        e0.record(s)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        qdd.copy_(qh, non_blocking=True)
+        layer.build(kd, vd)
+        layer.attention(qdd, od, lsed)
+        oh.copy_(od, non_blocking=True)
+        lh.copy_(lsed, non_blocking=True)
+        e1.record(s)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    t = torch.tensor([statistics.median(times)], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    vis = layer.sizes.stored_token_heads * 2 * k.shape[-1] * k.element_size()
+    h2d = (kh.numel() + vh.numel()) * kh.element_size() + qh.numel() * qh.element_size()
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+    return {"value": round(world * vis / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "path": "pinned host K/V/Q -> build_segpaged_cache -> segpaged_attention (decode) -> host O, LSE"}
+
+
+def oracle_decode_sample(wl, dec, k, v, qd, budget_s: float, max_heads: int | None = None) -> tuple[float, int, int]:
+    """Run the CPU oracle on whole (sequence, kv-head) groups until the time budget is spent.
+
+    Returns (seconds spent inside the oracle, visible KV bytes covered, groups done).
+    """
+    import oracle
+
+    spent, vis, groups = 0.0, 0, 0
+    order = [(b, kv) for b in range(wl.batch) for kv in range(wl.num_kv_heads)]
+    for b, kv in order:
+        if spent >= budget_s or (max_heads is not None and groups >= max_heads):
+            break
+        L = dec.ctx_lens[b]
+        kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+        kk = k[b, kv, :L].double().cpu().numpy()
+        vv = v[b, kv, :L].double().cpu().numpy()
+        qq = qd[b, kv * wl.group:(kv + 1) * wl.group].double().cpu().numpy()
+        t0 = time.perf_counter()
+        # the group's q-heads share the kv-head: one call, one query row per q-head (OpenMP over rows)
+        oracle.attention_rows(qq, [L - 1] * wl.group, kk, vv, kind, s, w)
+        spent += time.perf_counter() - t0
+        vis += int(oracle.stored_mask(kind, s, w, L, L - 1).sum()) * 2 * wl.head_dim * 2
+        groups += 1
+    return spent, vis, groups
+
+
+def cpu_baseline(wl, dec, k, v, qd, budget_s: float) -> dict:
+    import oracle
+    spent, vis, groups = oracle_decode_sample(wl, dec, k, v, qd, budget_s)
+    return {"value": round(vis / spent / 1e9, 4), "unit": "GB/s", "cores": min(oracle.num_threads(), wl.group),
+            "kind": "oracle",
+            "seconds": round(spent, 2),
+            "sample": f"decode of {groups} of {wl.batch * wl.num_kv_heads} (sequence, kv-head) groups, "
+                      f"all {wl.group} q-heads each (fp64 dense attention with explicit mask)"}
+
+
+def run_reference(args) -> None:
+    """The oracle as the reference arm: decode visible-KV GB/s of the fp64 CPU oracle."""
+    import torch
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from head_aware_paged_build_b200 import workloads as W
+
+    wl = workload(args.workload, 0)
+    dec = wl.decode_problem()
+    # inputs on the host (CPU generator): the oracle never touches the GPU
+    k, v = W.dense_kv(dec)
+    qd = W.queries(dec)
+    per_step = max(1, wl.num_kv_heads // 2)
+    for _ in range(args.warmup):
+        oracle_decode_sample(wl, dec, k, v, qd, 1e9, max_heads=1)
+    spent = vis = 0.0
+    t_steps = []
+    for _ in range(args.steps):
+        s, b, _ = oracle_decode_sample(wl, dec, k, v, qd, 1e9, max_heads=per_step)
+        spent += s
+        vis += b
+        t_steps.append(s)
+    value = vis / spent / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * spent / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, 1),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": min(oracle.num_threads(), wl.group),
+                         "kind": "oracle",
+                         "sample": f"per step: decode of {per_step} (sequence, kv-head) groups of sequence 0 "
+                                   f"(all {wl.group} q-heads each), fp64 dense attention with explicit mask"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="llama", choices=("llama", "mistral", "mha"))
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="time budget of the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -311,6 +311,7 @@ sp_status plan_build(sp_plan& pl) {
   z.is_decode = decode ? 1 : 0;
   z.num_decode_ctas = H.n_decode_ctas;
   z.num_prefill_items = H.n_prefill_items;
+  z.num_combine = H.n_combine;
   return SP_OK;
 }
 

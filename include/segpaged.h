@@ -125,7 +125,7 @@ typedef struct {
   int32_t is_decode;          /* 1 if every C_b == 1 */
   int32_t num_decode_ctas;    /* decode grid size (0 for prefill plans) */
   int32_t num_prefill_items;  /* prefill grid size (0 for decode plans) */
-  int32_t reserved;
+  int32_t num_combine;        /* decode heads split across CTAs (> 0: a combine pass runs) */
 } sp_sizes;
 
 /* One contiguous run of stored positions of a head; it starts on a fresh page. */
