@@ -115,6 +115,21 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+def reduce_max(values, world: int, device) -> list[float]:
+    """Element-wise max over ranks (the slowest rank sets every timing)."""
+    import torch
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank processed the same units in at most max_ms."""
+    return world * units_per_rank / (max_ms * 1e-3)
+
+
 def kernel_traffic(kernel: str, source: Path) -> int | None:
     """DRAM bytes per launch from the last ncu capture, if the kernel source is unchanged since."""
     p = ROOT / "profiles" / "traffic.json"
@@ -196,10 +211,7 @@ def run_ours(args) -> None:
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    t = torch.tensor([x / args.steps for x in totals], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = dict(zip(names, t.tolist()))
+    ms = dict(zip(names, reduce_max([x / args.steps for x in totals], world, dev)))
 
     # ---- dense-plus-mask variant (same kernels, every head stores its whole context) ----
     Ldm = layer_for(dec, device=dev, flags=S.SP_FLAG_DENSE_MASKED)
@@ -219,10 +231,7 @@ def run_ours(args) -> None:
             torch.cuda.synchronize()
             vals.append(e0.elapsed_time(e1))
         dm[nm] = statistics.median(vals)
-    dmt = torch.tensor([dm["decode"], dm["prefill"]], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(dmt, op=dist.ReduceOp.MAX)
-    dm = dict(zip(("decode", "prefill"), dmt.tolist()))
+    dm = dict(zip(("decode", "prefill"), reduce_max([dm["decode"], dm["prefill"]], world, dev)))
     del Ldm, Lpm
 
     # ---- end to end through the public API with host buffers ----
@@ -234,8 +243,8 @@ def run_ours(args) -> None:
     flops_pre = 4 * wl.head_dim * zp.visible_pairs                  # QK^T + PV on visible pairs
     pack_bytes = lambda z: z.stored_token_heads * 2 * wl.head_dim * eb + 2 * z.num_pages * z.page_bytes
     pk = peaks()
-    dec_gbs = world * vis_dec / (ms["decode"] * 1e-3) / 1e9
-    pre_tflops = world * flops_pre / (ms["prefill"] * 1e-3) / 1e12
+    dec_gbs = weak_rate(vis_dec, world, ms["decode"]) / 1e9
+    pre_tflops = weak_rate(flops_pre, world, ms["prefill"]) / 1e12
     launches_per_step = 1 + zd.kernel_launches() + 1 + zp.kernel_launches()
 
     if rank != 0:
@@ -314,15 +323,11 @@ def run_e2e(args, dev, layer, k, v, qd, od, lsed, world) -> dict:
         torch.cuda.synchronize()
         if i >= args.warmup:
             times.append(e0.elapsed_time(e1))
-    t = torch.tensor([statistics.median(times)], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = reduce_max([statistics.median(times)], world, dev)[0]
     vis = layer.sizes.stored_token_heads * 2 * k.shape[-1] * k.element_size()
     h2d = (kh.numel() + vh.numel()) * kh.element_size() + qh.numel() * qh.element_size()
     d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
-    return {"value": round(world * vis / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 3),
+    return {"value": round(weak_rate(vis, world, ms) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "path": "pinned host K/V/Q -> build_segpaged_cache -> segpaged_attention (decode) -> host O, LSE"}
 
