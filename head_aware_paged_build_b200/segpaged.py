@@ -29,7 +29,7 @@ DTYPE_CODES = {"f32": SP_F32, "bf16": SP_BF16}
 EXPORTED = ("segpaged_plan_create", "segpaged_plan_destroy", "segpaged_plan_sizes",
             "segpaged_plan_head_segments", "segpaged_plan_head_pages", "segpaged_table_write",
             "build_segpaged_cache", "segpaged_gather", "segpaged_attention",
-            "segpaged_read_device_status", "segpaged_clear_device_status", "segpaged_status_string",
+            "segpaged_attention_decode_noalloc", "segpaged_read_device_status", "segpaged_clear_device_status", "segpaged_status_string",
             "segpaged_last_error", "segpaged_abi_version")
 
 
@@ -99,6 +99,7 @@ def load(path: Path | str | None = None) -> ctypes.CDLL:
         "build_segpaged_cache": ([vp, vp, vp, vp, i64, i64, i64, vp, vp, vp], i32),
         "segpaged_gather": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
         "segpaged_attention": ([vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp], i32),
+        "segpaged_attention_decode_noalloc": ([vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp], i32),
         "segpaged_read_device_status": ([vp, ctypes.POINTER(i32), vp], i32),
         "segpaged_clear_device_status": ([vp, vp], i32),
         "segpaged_status_string": ([i32], ctypes.c_char_p),
@@ -209,6 +210,14 @@ def segpaged_attention(plan: int, d_table: int, k_pool: int, v_pool: int, q: int
                        softmax_scale: float, workspace: int, workspace_bytes: int, stream: int = 0) -> None:
     _check(load().segpaged_attention(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale, workspace,
                                      workspace_bytes, stream), "segpaged_attention")
+
+
+def segpaged_attention_decode_noalloc(plan: int, d_table: int, k_pool: int, v_pool: int, q: int, out: int,
+                                      lse: int | None, softmax_scale: float, d_status: int | None = None,
+                                      stream: int = 0) -> None:
+    """Decode attention with the library's built-in scratch (no workspace argument, no allocation)."""
+    _check(load().segpaged_attention_decode_noalloc(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale,
+                                                    d_status, stream), "segpaged_attention_decode_noalloc")
 
 
 def segpaged_attention_status(*args) -> int:

@@ -204,6 +204,33 @@ SP_API sp_status segpaged_attention(const sp_plan* plan, const void* d_table, co
                              float softmax_scale, void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/* segpaged_attention_decode_noalloc: decode attention that allocates nothing.
+ * (The paper has no counterpart; this is a deployment variant of the decode
+ * call above.)  Some callers cannot hand this library a workspace: engines
+ * whose device memory is divided into a fixed arena before serving starts,
+ * and latency-critical loops that must not call cudaMalloc because it can
+ * synchronise the device.  This call runs the same split-KV decode and
+ * combine kernels as segpaged_attention on a decode plan, but takes their
+ * scratch (status word + partial results) from a 4 MiB array built into the
+ * library's device image, one per GPU, held until the process exits.  It
+ * calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - Decode plans only (SP_ERR_UNSUPPORTED otherwise).  A plan whose
+ *     workspace_bytes exceed 4 MiB is rejected with SP_ERR_WORKSPACE before
+ *     any launch (lower target_ctas, or use segpaged_attention).
+ *   - It runs on the current CUDA device.  The first call on a device looks
+ *     up the array's device address (cudaGetSymbolAddress) with that device
+ *     current; make that first call before any stream capture.
+ *   - All calls on one GPU share the array and leave their contents in it.
+ *     Each call clears the status word; the partial results need no
+ *     clearing.  Calls whose kernels overlap on the GPU race on the array:
+ *     serialise them.
+ *   - d_status: NULL, or a device int32 the caller owns (and clears) that
+ *     receives the device status code instead of the built-in word.
+ * Other arguments as segpaged_attention. */
+SP_API sp_status segpaged_attention_decode_noalloc(const sp_plan* plan, const void* d_table, const void* k_pool,
+                                                   const void* v_pool, const void* q, void* out, float* lse,
+                                                   float softmax_scale, int32_t* d_status, void* stream);
+
 /* Device status word: kernels never trap; a failed device-side check or a
  * bounded wait that ran out records a non-zero code.  read synchronises
  * `stream` and returns the code in *code (0 = no error); clear zeroes it. */
