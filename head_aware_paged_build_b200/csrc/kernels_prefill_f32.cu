@@ -1,6 +1,7 @@
 // fp32 prefill: SIMT FP32-FMA kernel over the plan's prefill work list.
 //
-// One CTA per (q-head, 64-row query tile); thread r owns query row r.  KV
+// One CTA per (q-head, 64-row query tile) (the planner gives fp32 plans
+// single-tile items); thread r owns query row r.  KV
 // tiles of 64 tokens (the head's pages, in its position order) are staged in
 // shared memory; each thread scores the tile's keys for its row, masks them
 // (causal, and sink + window for local heads), and folds them into an online
@@ -30,12 +31,12 @@ __global__ void __launch_bounds__(kRows) prefill_f32_kernel(PrefillLaunch a) {
   const PrefillItem it = a.items[blockIdx.x];
   const HeadDesc hd = a.heads[it.head];
   const int r = threadIdx.x;
-  const bool active = r < it.n_rows;
-  const int p = it.p0 + r;
+  const bool active = r < it.n_rows[0];
+  const int p = it.p0[0] + r;
   const float* qg = static_cast<const float*>(a.q);
   for (int e = threadIdx.x; e < kRows * D; e += kRows) {
     const int rr = e / D, i = e % D;
-    qs[rr * (D + 1) + i] = rr < it.n_rows ? qg[(int64_t(it.q_row + rr) * a.num_q_heads + it.qh) * D + i] : 0.f;
+    qs[rr * (D + 1) + i] = rr < it.n_rows[0] ? qg[(int64_t(it.q_row[0] + rr) * a.num_q_heads + it.qh[0]) * D + i] : 0.f;
   }
   float acc[D];
 #pragma unroll
@@ -97,10 +98,10 @@ __global__ void __launch_bounds__(kRows) prefill_f32_kernel(PrefillLaunch a) {
     }
   }
   if (!active) return;
-  float* og = static_cast<float*>(a.out) + (int64_t(it.q_row + r) * a.num_q_heads + it.qh) * D;
+  float* og = static_cast<float*>(a.out) + (int64_t(it.q_row[0] + r) * a.num_q_heads + it.qh[0]) * D;
 #pragma unroll
   for (int i = 0; i < D; ++i) og[i] = acc[i] / l;
-  if (a.lse) a.lse[int64_t(it.q_row + r) * a.num_q_heads + it.qh] = (m + log2f(l)) * kLn2f;
+  if (a.lse) a.lse[int64_t(it.q_row[0] + r) * a.num_q_heads + it.qh[0]] = (m + log2f(l)) * kLn2f;
 }
 
 template <int D, int P>

@@ -1,26 +1,36 @@
 // bf16 prefill on 5th-generation tensor cores (tcgen05, sm_100a).
 //
-// One CTA per (q-head, 128-row query tile).  It visits only the KV tiles of
-// 128 tokens (two pages) that some row of the tile can see, in the head's
-// stored order: the sink tiles and the recent-window tiles of a local head,
-// the causal prefix of a global head ("SegPagedAttention runtime design", §4:
-// each (query-head, kv-head) pair runs over its own true length, no mask over
+// One CTA per work item: one or two 128-row query tiles of the same
+// (sequence, kv-head) — two q-heads of the GQA group at the same positions,
+// or neighbouring query tiles.  The CTA visits only the KV tiles of 128
+// tokens (two pages) that some row can see, in the head's stored order: the
+// sink tiles and the recent-window tiles of a local head, the causal prefix of
+// a global head ("SegPagedAttention runtime design", §4: every
+// (query-head, kv-head) pair runs over its own true length, with no mask over
 // invisible KV).  Only tiles that cross a boundary (causal diagonal, window
-// edge, sink page, a segment's partial last page) are masked per element.
+// edge, sink page, a segment's partial last page) are masked, per row, by
+// visible column intervals.
 //
-// Warp roles (192 threads):
-//   warp 0      producer: Q tile by TMA (128-byte swizzle), K and V pages by
-//               1-D bulk copies (pool pages are stored in the tensor cores'
-//               swizzled K-major operand layout, V transposed)
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T and O += P V as
-//               tcgen05.mma kind::f16, fp32 accumulators in TMEM
-//               (O: D columns, S: two buffers of 128 columns)
-//   warps 2-5   softmax: one query row per thread, S read with tcgen05.ld,
-//               online softmax in the log2 domain with a lazy rescale of O
-//               (only when the row maximum grows by more than 2^8), P
-//               written to shared memory as the bf16 A operand of P V;
-//               then the epilogue (O / l, LSE).
-// Every wait is bounded; a wait that runs out records a status code and the
+// Warp roles (320 threads):
+//   warp 0      producer: both Q tiles by TMA (128-byte swizzle); K and V
+//               pages by 1-D bulk copies (pool pages are stored in the tensor
+//               cores' swizzled K-major operand layout, V transposed), one
+//               K/V stage feeding both query tiles
+//   warp 1      TMEM owner and MMA issuer (one thread):
+//                 S_x = Q_x K^T       tcgen05.mma, A and B from shared memory
+//                 O_x += P_x V        tcgen05.mma, A (= P_x) from TMEM
+//               in the order S_A, S_B, then per KV tile j:
+//                 PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
+//               so that the tensor core alternates between the two tiles while
+//               their softmax warpgroups run
+//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: one row per
+//               thread; S read with tcgen05.ld, online softmax in the log2
+//               domain with a lazy rescale of O (only when the row maximum
+//               grows by more than 2^8), P written back as bf16 over the first
+//               64 columns of its own S buffer; then the epilogue (O / l, LSE).
+// The commit that signals S_x(j) also covers P_x(j-1) V, so a softmax thread
+// holding S_x(j) may rescale O_x and overwrite P_x with no further wait.
+// Every wait is bounded; a wait that runs out records a status code, and the
 // CTA drains its copies and MMAs, frees its TMEM and returns.
 #include <cuda.h>
 
@@ -34,26 +44,34 @@ namespace sp {
 namespace {
 
 constexpr int kTile = kPrefillTileTokensBf16;  // 128 query rows, 128 KV tokens
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by more than 2^8
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr uint32_t kFull = 0xffffffffu;
 
 template <int D, int NS>
 struct TcSmem {
-  static constexpr int kQ = D / 64 * 16384;  // [D/64][128 rows][128 B]
+  static constexpr int kQ = D / 64 * 16384;  // one query tile: [D/64][128 rows][128 B]
   static constexpr int kK = D / 64 * 16384;  // [D/64][128 tokens][128 B]
   static constexpr int kV = 2 * D * 128;     // [2 pages][D rows][64 tokens * 2 B]
   static constexpr int kStage = kK + kV;
-  static constexpr int kP = 2 * 16384;       // [2][128 rows][64 tokens * 2 B]
   static constexpr int kOffQ = 0;
-  static constexpr int kOffStage = kOffQ + kQ;
-  static constexpr int kOffP = kOffStage + NS * kStage;
-  static constexpr int kOffBar = kOffP + kP;
+  static constexpr int kOffStage = kOffQ + 2 * kQ;
+  static constexpr int kOffBar = kOffStage + NS * kStage;
   static constexpr int kBytes = kOffBar + 256 + 1024;  // barriers + 1 KB alignment slack
 };
 
-// Does every query row p in [p_first, p_last] see every slot of this page?
+struct Bars {
+  uint64_t q;
+  uint64_t o_done;
+  uint64_t done;
+  uint64_t pad;
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+};
+
+// Does every row p in [p_first, p_last] see every slot of this page?
 __device__ __forceinline__ bool page_fully_visible(const PageDesc& pg, bool exists, const HeadDesc& hd, int p_first,
                                                    int p_last) {
   if (!exists || pg.nvalid != 64) return false;
@@ -63,14 +81,22 @@ __device__ __forceinline__ bool page_fully_visible(const PageDesc& pg, bool exis
   return a1 < hd.sink || a0 > p_last - hd.window;
 }
 
-struct Bars {
-  uint64_t q;
-  uint64_t p_full;
-  uint64_t o_done;
-  uint64_t done;
-  uint64_t s_full[2];
-  uint64_t s_free[2];
-};
+// Slots of a page visible to row p: [0, h1) and [l2, h2) (possibly empty).
+__device__ __forceinline__ void visible_slots(const PageDesc& pg, bool exists, const HeadDesc& hd, int p, int& h1,
+                                              int& l2, int& h2) {
+  if (!exists) {
+    h1 = 0, l2 = 0, h2 = 0;
+    return;
+  }
+  const int causal = min(pg.nvalid, p - pg.abs_start + 1);  // positions <= p
+  if (hd.kind == 0) {
+    h1 = causal, l2 = 0, h2 = 0;
+  } else {
+    h1 = min(causal, hd.sink - pg.abs_start);           // sink run
+    l2 = max(0, p - hd.window + 1 - pg.abs_start);      // recent window
+    h2 = causal;
+  }
+}
 
 template <int D, int NS>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap,
@@ -80,7 +106,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem + Sm::kOffQ;
   uint8_t* stage_s = smem + Sm::kOffStage;
-  uint8_t* p_s = smem + Sm::kOffP;
   Bars* bars = reinterpret_cast<Bars*>(smem + Sm::kOffBar);
   uint64_t* kv_full = reinterpret_cast<uint64_t*>(bars + 1);
   uint64_t* kv_free = kv_full + NS;
@@ -92,15 +117,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   const HeadDesc hd = a.heads[it.head];
   const int n1 = it.t1 - it.t0;
   const int n = n1 + (it.t3 - it.t2);
+  const bool two = it.qh[1] >= 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q, 1);
-    mbar_init(&bars->p_full, 128);
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->done, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_full[x], 128);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -118,21 +143,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_o = tmem;          // O: columns [0, D)
-  const uint32_t t_s0 = tmem + 128;   // S buffers: [128, 256), [256, 384)
+  // TMEM columns: S/P of tile x at [128 x, 128 x + 128); O of tile x at 256 + x D
+  auto t_s = [&](int x) { return tmem + uint32_t(128 * x); };
+  auto t_o = [&](int x) { return tmem + uint32_t(256 + x * D); };
 
   auto fail = [&](int32_t code) {
     record_error(a.status, code);
     *abort_flag = 1;
   };
+  auto tile_of = [&](int j) { return j < n1 ? it.t0 + j : it.t2 + (j - n1); };
 
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
     if (lane == 0) {
       const uint8_t* kpool = static_cast<const uint8_t*>(a.kpool);
       const uint8_t* vpool = static_cast<const uint8_t*>(a.vpool);
-      mbar_arrive_expect_tx(&bars->q, Sm::kQ);
-      for (int h = 0; h < D / 64; ++h) tc::tma_load_3d(q_s + h * 16384, &qmap, h * 64, it.qh, it.q_row, &bars->q);
+      mbar_arrive_expect_tx(&bars->q, (two ? 2 : 1) * Sm::kQ);
+      for (int x = 0; x < (two ? 2 : 1); ++x)
+        for (int h = 0; h < D / 64; ++h)
+          tc::tma_load_3d(q_s + x * Sm::kQ + h * 16384, &qmap, h * 64, it.qh[x], it.q_row[x], &bars->q);
       int issued = 0;
       for (int j = 0; j < n && !*abort_flag; ++j) {
         const int st = j % NS;
@@ -140,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           fail(kDevTimeoutEmpty);
           break;
         }
-        const int t = j < n1 ? it.t0 + j : it.t2 + (j - n1);
+        const int t = tile_of(j);
         const int vp0 = 2 * t, vp1 = (2 * t + 1 < hd.n_vpages) ? 2 * t + 1 : 2 * t;
         const int64_t ph[2] = {a.pages[hd.vpage_begin + vp0].phys, a.pages[hd.vpage_begin + vp1].phys};
         uint8_t* k_s = stage_s + st * Sm::kStage;
@@ -164,40 +193,53 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     if (lane == 0) {
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128);
       constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D);
-      const uint32_t q_addr = smem_u32(q_s), p_addr = smem_u32(p_s), st_addr = smem_u32(stage_s);
-      bool ok = mbar_wait(&bars->q, 0);
+      const uint32_t q_addr = smem_u32(q_s), st_addr = smem_u32(stage_s);
+      auto issue_s = [&](int x, int st) {
+        const uint32_t qa = q_addr + x * Sm::kQ, ka = st_addr + st * Sm::kStage;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc::mma_bf16_ss(t_s(x), tc::smem_desc_sw128(qa + off), tc::smem_desc_sw128(ka + off), idesc_s, kk > 0);
+        }
+        tc::commit(&bars->s_full[x]);
+      };
+      auto issue_pv = [&](int x, int st, bool acc) {
+        const uint32_t va = st_addr + st * Sm::kStage + Sm::kK;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          tc::mma_bf16_ts(t_o(x), t_s(x) + kk * 8,
+                          tc::smem_desc_sw128(va + (kk >> 2) * (D * 128) + (kk & 3) * 32), idesc_o,
+                          (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&bars->q, 0) && mbar_wait(&kv_full[0], 0);
       if (!ok) fail(kDevTimeoutFull);
-      for (int j = 0; ok && j <= n; ++j) {
-        if (*abort_flag) break;
-        if (j < n) {
-          const int st = j % NS, b = j & 1;
-          if (!mbar_wait(&kv_full[st], (j / NS) & 1)) { fail(kDevTimeoutFull); break; }
-          if (j >= 2 && !mbar_wait(&bars->s_free[b], ((j >> 1) - 1) & 1)) { fail(kDevTimeoutSoftmax); break; }
-          tc::fence_after_sync();
-          const uint32_t k_addr = st_addr + st * Sm::kStage;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc::mma_bf16_ss(t_s0 + b * 128, tc::smem_desc_sw128(q_addr + off), tc::smem_desc_sw128(k_addr + off),
-                            idesc_s, kk > 0);
-          }
-          tc::commit(&bars->s_full[b]);
-        }
-        if (j >= 1) {
-          const int jj = j - 1, st = jj % NS;
-          if (!mbar_wait(&bars->p_full, jj & 1)) { fail(kDevTimeoutSoftmax); break; }
-          tc::fence_after_sync();
-          const uint32_t v_addr = st_addr + st * Sm::kStage + Sm::kK;
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint32_t pa = p_addr + (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t va = v_addr + (kk >> 2) * (D * 128) + (kk & 3) * 32;
-            tc::mma_bf16_ss(t_o, tc::smem_desc_sw128(pa), tc::smem_desc_sw128(va), idesc_o, (jj > 0 || kk > 0));
-          }
-          tc::commit(&bars->o_done);
-          tc::commit(&kv_free[st]);
-        }
+      if (ok && n > 0) {
+        tc::fence_after_sync();
+        issue_s(0, 0);
+        if (two) issue_s(1, 0);
       }
+      for (int j = 0; ok && j < n; ++j) {
+        if (*abort_flag) break;
+        const int st = j % NS;
+        const bool more = j + 1 < n;
+        const int st1 = (j + 1) % NS;
+        if (!mbar_wait(&bars->p_full[0], j & 1)) { fail(kDevTimeoutSoftmax); break; }
+        tc::fence_after_sync();
+        issue_pv(0, st, j > 0);
+        if (more) {
+          if (!mbar_wait(&kv_full[st1], ((j + 1) / NS) & 1)) { fail(kDevTimeoutFull); break; }
+          tc::fence_after_sync();
+          issue_s(0, st1);
+        }
+        if (two) {
+          if (!mbar_wait(&bars->p_full[1], j & 1)) { fail(kDevTimeoutSoftmax); break; }
+          tc::fence_after_sync();
+          issue_pv(1, st, j > 0);
+        }
+        tc::commit(&kv_free[st]);
+        if (two && more) issue_s(1, st1);
+      }
+      tc::commit(&bars->o_done);
       // all MMAs issued by this thread complete before TMEM is released
       tc::commit(&bars->done);
       mbar_wait(&bars->done, 0);
@@ -205,128 +247,140 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     __syncwarp();
   } else {
     // ------------------------------ softmax ------------------------------
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    const int p = it.p0 + r;
-    const int p_last = it.p0 + it.n_rows - 1;
-    const float sl2 = a.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int b = j & 1;
-      const int t = j < n1 ? it.t0 + j : it.t2 + (j - n1);
-      const bool have1 = 2 * t + 1 < hd.n_vpages;
-      const PageDesc pg0 = a.pages[hd.vpage_begin + 2 * t];
-      const PageDesc pg1 = have1 ? a.pages[hd.vpage_begin + 2 * t + 1] : PageDesc{0, 0, 0, 0};
-      const bool full = page_fully_visible(pg0, true, hd, it.p0, p_last) &&
-                        page_fully_visible(pg1, have1, hd, it.p0, p_last);
-      // tcgen05.ld / st are warp-collective (.sync.aligned): every branch that
-      // guards one must be taken by the whole warp, so wait outcomes are voted.
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[b], (j >> 1) & 1))) {
-        fail(kDevTimeoutMma);
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-      float s[kTile];
-#pragma unroll
-      for (int c = 0; c < kTile / 32; ++c)
-        tc::tmem_ld32(t_s0 + b * 128 + lane_off + c * 32, *reinterpret_cast<float(*)[32]>(s + c * 32));
-      tc::tmem_wait_ld();
-      tc::fence_before_sync();
-      mbar_arrive(&bars->s_free[b]);
-      if (!full) {
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) {
-          const PageDesc& pg = c < 64 ? pg0 : pg1;
-          const int slot = c & 63;
-          const bool vis = slot < pg.nvalid && sees(hd.kind, hd.sink, hd.window, p, pg.abs_start + slot);
-          if (!vis) s[c] = -INFINITY;
+    const int x = (warp - 2) >> 2;  // query tile of this warpgroup
+    if (x == 0 || two) {
+      const int quarter = warp & 3;
+      const int r = quarter * 32 + lane;
+      const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+      const int p = it.p0[x] + r;
+      const int p_first = it.p0[x], p_last = it.p0[x] + it.n_rows[x] - 1;
+      const float sl2 = a.scale_log2;
+      float m_run = -INFINITY, l_run = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n; ++j) {
+        const int t = tile_of(j);
+        const bool have1 = 2 * t + 1 < hd.n_vpages;
+        const PageDesc pg0 = a.pages[hd.vpage_begin + 2 * t];
+        const PageDesc pg1 = have1 ? a.pages[hd.vpage_begin + 2 * t + 1] : PageDesc{0, 0, 0, 0};
+        const bool full = page_fully_visible(pg0, true, hd, p_first, p_last) &&
+                          page_fully_visible(pg1, have1, hd, p_first, p_last);
+        // tcgen05.ld / st are warp-collective (.sync.aligned): every branch that
+        // guards one is taken by the whole warp, so wait outcomes are voted.
+        if (!__all_sync(kFull, mbar_wait(&bars->s_full[x], j & 1))) {
+          fail(kDevTimeoutMma);
+          ok = false;
+          break;
         }
-      }
-      float mt = s[0];
+        tc::fence_after_sync();
+        // Visible slots of this row in the tile's two pages (boundary tiles only).
+        int h1a = 64, l2a = 0, h2a = 0, h1b = 64, l2b = 0, h2b = 0;
+        if (!full) {
+          visible_slots(pg0, true, hd, p, h1a, l2a, h2a);
+          visible_slots(pg1, have1, hd, p, h1b, l2b, h2b);
+        }
+        auto mask32 = [&](float (&v)[32], int chunk) {  // chunk c covers columns [32 c, 32 c + 32)
+          const int h1 = chunk < 2 ? h1a : h1b, l2 = chunk < 2 ? l2a : l2b, h2 = chunk < 2 ? h2a : h2b;
+          const int c0 = (chunk & 1) * 32;
 #pragma unroll
-      for (int c = 1; c < kTile; ++c) mt = fmaxf(mt, s[c]);
-      const float mts = mt * sl2;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (mts > m_run + kRescaleLog2) {
-        alpha = fast_exp2(m_run - mts);
-        rescale = m_run != -INFINITY;
-        m_run = mts;
-      }
-      const float base = m_run == -INFINITY ? 0.f : m_run;
-      uint32_t pk[kTile / 2];
-      float sum = 0.f;
+          for (int e = 0; e < 32; ++e) {
+            const int c = c0 + e;
+            if (!(c < h1 || (c >= l2 && c < h2))) v[e] = -INFINITY;
+          }
+        };
+        // pass 1: the row maximum (S stays in TMEM; 64 columns in registers at a time)
+        float mx[8];
 #pragma unroll
-      for (int c = 0; c < kTile / 2; ++c) {
-        const float e0 = fast_exp2(fmaf(s[2 * c], sl2, -base));
-        const float e1 = fast_exp2(fmaf(s[2 * c + 1], sl2, -base));
-        sum += e0 + e1;
-        pk[c] = pack_bf16x2(e0, e1);
+        for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+          float va[32], vb[32];
+          tc::tmem_ld32(t_s(x) + lane_off + hc * 64, va);
+          tc::tmem_ld32(t_s(x) + lane_off + hc * 64 + 32, vb);
+          tc::tmem_wait_ld();
+          if (!full) {
+            mask32(va, 2 * hc);
+            mask32(vb, 2 * hc + 1);
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], fmaxf(va[e], vb[e]));
+        }
+        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mts = mt * sl2;
+        float alpha = 1.f;
+        bool need = false;
+        if (mts > m_run + kRescaleLog2) {
+          alpha = fast_exp2(m_run - mts);
+          need = m_run != -INFINITY;
+          m_run = mts;
+        }
+        // O_x is stable here: the commit behind s_full also covered P_x(j-1) V.
+        // The decision is per row; the TMEM round trip runs for the whole warp.
+        if (__any_sync(kFull, need)) {
+          const float f = need ? alpha : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tc::tmem_ld32(t_o(x) + lane_off + c * 32, o);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= f;
+            tc::tmem_st32(t_o(x) + lane_off + c * 32, o);
+          }
+        }
+        // pass 2: P = 2^(s - m) in bf16, written over S columns already consumed:
+        // chunk c of S (columns [32 c, 32 c + 32)) becomes P columns [16 c, 16 c + 16).
+        const float base = m_run == -INFINITY ? 0.f : m_run;
+        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < kTile / 32; ++c) {
+          float v[32];
+          tc::tmem_ld32(t_s(x) + lane_off + c * 32, v);
+          tc::tmem_wait_ld();
+          if (!full) mask32(v, c);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float e0 = fast_exp2(fmaf(v[2 * e], sl2, -base));
+            const float e1 = fast_exp2(fmaf(v[2 * e + 1], sl2, -base));
+            sum[e & 3] += e0 + e1;
+            pk[e] = pack_bf16x2(e0, e1);
+          }
+          tc::tmem_st16(t_s(x) + lane_off + c * 16, pk);
+        }
+        l_run = l_run * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+        tc::tmem_wait_st();
+        tc::fence_before_sync();
+        mbar_arrive(&bars->p_full[x]);
       }
-      l_run = l_run * alpha + sum;
-      // P V of the previous tile must be done before P and O are touched
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->o_done, (j - 1) & 1))) {
-        fail(kDevTimeoutMma);
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-      // The rescale decision is per row; the TMEM round trip runs for the whole
-      // warp whenever one of its rows needs it (factor 1 for the others).
-      const bool need = rescale && j > 0;
-      if (__any_sync(0xffffffffu, need)) {
-        const float f = need ? alpha : 1.f;
+      // ------------------------------ epilogue ------------------------------
+      bool go = ok && n > 0 && mbar_wait(&bars->o_done, 0);
+      go = __all_sync(kFull, go && !*abort_flag);
+      if (go) {
+        tc::fence_after_sync();
+        const bool row_ok = r < it.n_rows[x];
+        const float inv_l = 1.f / l_run;
+        __nv_bfloat16* orow =
+            static_cast<__nv_bfloat16*>(a.out) + (int64_t(it.q_row[x] + r) * a.num_q_heads + it.qh[x]) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
-          tc::tmem_ld32(t_o + lane_off + c * 32, o);
+          tc::tmem_ld32(t_o(x) + lane_off + c * 32, o);
           tc::tmem_wait_ld();
+          if (row_ok) {
+            uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= f;
-          tc::tmem_st32(t_o + lane_off + c * 32, o);
+            for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
         }
-        tc::tmem_wait_st();
+        if (row_ok && a.lse)
+          a.lse[int64_t(it.q_row[x] + r) * a.num_q_heads + it.qh[x]] = (m_run + log2f(l_run)) * kLn2;
+      } else if (ok && n > 0) {
+        fail(kDevTimeoutMma);
       }
-      // P row r -> [2 atoms][128 rows][128 B], 16-byte chunk c at c ^ (r & 7)
-#pragma unroll
-      for (int cc = 0; cc < kTile / 8; ++cc) {
-        const int atom = cc >> 3, c = cc & 7;
-        uint8_t* dst = p_s + atom * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-      }
-      tc::fence_proxy_async_smem();
-      tc::fence_before_sync();
-      mbar_arrive(&bars->p_full);
-    }
-    // ------------------------------ epilogue ------------------------------
-    bool go = ok && n > 0 && mbar_wait(&bars->o_done, (n - 1) & 1);
-    go = __all_sync(0xffffffffu, go && !*abort_flag);
-    if (go) {
-      tc::fence_after_sync();
-      const bool row_ok = r < it.n_rows;
-      const float inv_l = 1.f / l_run;
-      __nv_bfloat16* orow =
-          static_cast<__nv_bfloat16*>(a.out) + (int64_t(it.q_row + r) * a.num_q_heads + it.qh) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float o[32];
-        tc::tmem_ld32(t_o + lane_off + c * 32, o);
-        tc::tmem_wait_ld();
-        if (row_ok) {
-          uint32_t w[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-        }
-      }
-      if (row_ok && a.lse) a.lse[int64_t(it.q_row + r) * a.num_q_heads + it.qh] = (m_run + log2f(l_run)) * kLn2;
-    } else if (ok && n > 0) {
-      fail(kDevTimeoutMma);
     }
   }
 

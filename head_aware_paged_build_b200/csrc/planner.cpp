@@ -142,7 +142,9 @@ sp_status plan_build(sp_plan& pl) {
       hd = HeadDesc{};
       hd.kind = local ? 1 : 0;
       hd.sink = int32_t(s);
-      hd.window = int32_t(std::min<int64_t>(w, std::numeric_limits<int32_t>::max()));
+      // windows beyond the 2^30 context cap change nothing; the clamp keeps
+      // position arithmetic such as p - window + 1 - a inside int32
+      hd.window = int32_t(std::min<int64_t>(w, int64_t(1) << 30));
       hd.ctx_len = int32_t(L);
       hd.q_start = int32_t(q0);
       hd.vpage_begin = int32_t(n_pages);
@@ -222,7 +224,13 @@ sp_status plan_build(sp_plan& pl) {
     }
   } else {
     // --- prefill: query tiles x visited KV tile ranges -----------------------
-    const int T = p.dtype == SP_BF16 ? kPrefillTileTokensBf16 : kPrefillTileTokensF32;
+    // bf16 items pair two query tiles of the same (sequence, kv-head) so that
+    // one K/V tile in shared memory feeds two 128-row tiles: two q-heads of the
+    // GQA group at the same positions, or (odd group sizes, MHA) neighbouring
+    // query tiles, whose visible KV ranges share the sink run and overlap in
+    // the window.  fp32 items hold a single 64-row tile.
+    const bool pair = p.dtype == SP_BF16;
+    const int T = pair ? kPrefillTileTokensBf16 : kPrefillTileTokensF32;
     const int ppt = T / P;
     pl.prefill_tile = T;
     std::vector<std::vector<PrefillItem>> per_head(nh);
@@ -230,20 +238,31 @@ sp_status plan_build(sp_plan& pl) {
     for (int h = 0; h < nh; ++h) {
       const HeadDesc& hd = pl.heads[h];
       const int64_t C = hd.ctx_len - hd.q_start;
-      for (int64_t qt = 0; qt * T < C; ++qt) {
+      std::vector<std::pair<int64_t, int>> units;  // (query tile, q-head)
+      for (int64_t qt = 0; qt * T < C; ++qt)
+        for (int g = 0; g < pl.group; ++g) units.emplace_back(qt, hd.kv * pl.group + g);
+      const size_t step = pair ? 2 : 1;
+      for (size_t u = 0; u < units.size(); u += step) {
         PrefillItem it{};
         it.head = h;
-        it.n_rows = int32_t(std::min<int64_t>(T, C - qt * T));
-        it.q_row = int32_t(hd.q_row0 + qt * T);
-        it.p0 = int32_t(hd.q_start + qt * T);
-        const int64_t p1 = it.p0 + it.n_rows - 1;
+        it.qh[1] = -1;
+        int64_t p_first = std::numeric_limits<int64_t>::max(), p_last = -1;
+        for (size_t x = 0; x < step && u + x < units.size(); ++x) {
+          const int64_t qt = units[u + x].first;
+          it.qh[x] = units[u + x].second;
+          it.n_rows[x] = int32_t(std::min<int64_t>(T, C - qt * T));
+          it.q_row[x] = int32_t(hd.q_row0 + qt * T);
+          it.p0[x] = int32_t(hd.q_start + qt * T);
+          p_first = std::min<int64_t>(p_first, it.p0[x]);
+          p_last = std::max<int64_t>(p_last, it.p0[x] + it.n_rows[x] - 1);
+        }
         int64_t v0, v1, v2, v3;
         if (hd.kind == 0 || dense_masked) {
-          pages_touching(pl, h, 0, p1, &v0, &v1);
+          pages_touching(pl, h, 0, p_last, &v0, &v1);
           v2 = v3 = 0;
         } else {
-          pages_touching(pl, h, 0, std::min<int64_t>(hd.sink, p1 + 1) - 1, &v0, &v1);
-          pages_touching(pl, h, std::max<int64_t>(hd.sink, int64_t(it.p0) - hd.window + 1), p1, &v2, &v3);
+          pages_touching(pl, h, 0, std::min<int64_t>(hd.sink, p_last + 1) - 1, &v0, &v1);
+          pages_touching(pl, h, std::max<int64_t>(hd.sink, p_first - hd.window + 1), p_last, &v2, &v3);
         }
         int64_t t0 = v0 / ppt, t1 = ceil_div(v1, ppt), t2 = v2 / ppt, t3 = ceil_div(v3, ppt);
         if (v0 == v1) t0 = t1 = 0;
@@ -256,21 +275,15 @@ sp_status plan_build(sp_plan& pl) {
         per_head[h].push_back(it);
       }
     }
-    // Heaviest heads first; within a head the heaviest query tiles first, the
-    // group's q-heads back to back so that they share KV tiles through L2.
+    // Heaviest heads first; within a head the heaviest items first.  Items of
+    // one head run back to back so that its KV tiles are reused through L2.
     std::vector<int> order(nh);
     std::iota(order.begin(), order.end(), 0);
     std::stable_sort(order.begin(), order.end(), [&](int a, int c) { return head_max[a] > head_max[c]; });
     for (int h : order) {
       auto& v = per_head[h];
       std::stable_sort(v.begin(), v.end(), [](const PrefillItem& a, const PrefillItem& c) { return a.work > c.work; });
-      const int kv = pl.heads[h].kv;
-      for (const PrefillItem& it : v)
-        for (int g = 0; g < pl.group; ++g) {
-          PrefillItem x = it;
-          x.qh = kv * pl.group + g;
-          pl.prefill.push_back(x);
-        }
+      pl.prefill.insert(pl.prefill.end(), v.begin(), v.end());
     }
   }
   pl.n_partial_slots = n_slots;

@@ -69,20 +69,22 @@ struct alignas(16) CombineItem {
   int32_t pad;
 };
 
-// One prefill work unit: a tile of query rows of one q-head.  KV tiles (of the
-// kernel's tile size, counted in the head's page list) are visited in
-// [t0, t1) then [t2, t3).
+// One prefill work unit: one or two query tiles of the same (sequence,
+// kv-head).  Tile x holds rows [q_row[x], q_row[x] + n_rows[x]) of q-head
+// qh[x] at positions p0[x] ...; qh[1] < 0 when there is a single tile.  The
+// KV tiles (of the kernel's tile size, counted in the head's page list) that
+// any row of either tile can see are visited in [t0, t1) then [t2, t3).
 struct alignas(16) PrefillItem {
   int32_t head;
-  int32_t qh;      // absolute q-head index
-  int32_t q_row;   // first varlen row of the tile
-  int32_t n_rows;  // rows in the tile (<= tile size)
-  int32_t p0;      // absolute position of the first row
+  int32_t qh[2];
+  int32_t q_row[2];
+  int32_t n_rows[2];
+  int32_t p0[2];
   int32_t t0, t1, t2, t3;
-  int32_t work;    // visited KV tiles
-  int32_t pad0, pad1;
+  int32_t work;  // visited KV tiles
+  int32_t pad[2];
 };
-static_assert(sizeof(PrefillItem) == 48, "PrefillItem layout");
+static_assert(sizeof(PrefillItem) == 64, "PrefillItem layout");
 
 struct alignas(16) TableHeader {
   int32_t magic;
