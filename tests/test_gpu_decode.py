@@ -115,3 +115,17 @@ def test_decode_custom_scale():
                                                  kind, s, w, scale=0.05)
             assert np.max(np.abs(out[b, h].float().cpu().numpy() - o_ref[0])) <= 2e-2
             assert abs(float(lse[b, h]) - l_ref[0]) <= 2e-3
+
+
+def test_decode_mha_128k_full_size():
+    """MHA 128K layer (64 heads, 8 global, window 128): every output row against the oracle."""
+    wl = W.mha()
+    prob = wl.decode_problem()
+    k, v = W.dense_kv(prob, device="cuda")
+    q = W.queries(prob, device="cuda")
+    layer = layer_for(prob)
+    layer.build(k, v)
+    out, lse = layer.attention(q)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    assert_close(compare(prob, q, k, v, out, lse), "bf16")

@@ -90,3 +90,27 @@ def test_prefill_bf16_page_permutation_and_determinism():
     perm = list(np.random.default_rng(2).permutation(n))
     _, _, out2, lse2 = run_prefill(prob, k=k, v=v, q=q, page_ids=perm, first_page=1)
     assert torch.equal(out0, out2) and torch.equal(lse0, lse2)
+
+
+@pytest.mark.parametrize("name,seqs,heads", [
+    ("llama", (0, 7), None),
+    ("mha", (0, 3), (0, 1, 7, 8, 9, 31, 32, 56, 63)),
+])
+def test_prefill_bf16_matches_oracle_sampled_at_full_size(name, seqs, heads):
+    """The bench's layer (and the MHA 128K layer) at full size, in the bench's launch configuration.
+
+    Inputs are generated on the GPU; the oracle checks sampled rows (chunk edges, tile edges at
+    multiples of 512 +- 1, seeded random rows) of the listed sequences and q-heads.
+    """
+    wl = W.ALL[name]()
+    prob = wl.prefill_problem()
+    k, v = W.dense_kv(prob, device="cuda")
+    q = W.queries(prob, device="cuda")
+    layer = layer_for(prob)
+    layer.build(k, v)
+    out, lse = layer.attention(q)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    rows = [sample_rows(c, stride=512, n_random=12, seed=b) if b in seqs else [] for b, c in enumerate(prob.q_counts)]
+    res = compare(prob, q, k, v, out, lse, rows_per_seq=rows, heads=heads, seqs=seqs)
+    assert_close(res, "bf16")
