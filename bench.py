@@ -283,7 +283,7 @@ def run_ours(args) -> None:
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(per_launch_pre / pk["bf16_tflops"], 4),
                      "peak_source": f"{pk['source']} bf16 burst",
                      "traffic": kernel_traffic("prefill_tc_kernel", csrc / "kernels_prefill_tc.cu")},
-        "roofline_decode": {"kernel": "decode_bf16_kernel + combine_kernel", "bound": "hbm",
+        "roofline_decode": {"kernel": "decode_bf16_kernel", "bound": "hbm",
                             "achieved": round(vis_dec / (ms["decode"] * 1e-3) / 1e9, 1), "peak": pk["hbm_gbs"],
                             "unit": "GB/s", "frac": round(vis_dec / (ms["decode"] * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                             "peak_source": f"{pk['source']} HBM copy",

@@ -133,7 +133,8 @@ sp_status segpaged_attention(const sp_plan* plan, const void* d_table, const voi
     L.page_bytes = plan->sizes.page_bytes;
     L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
     L.scale_log2 = scale_log2;
-    L.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
+    L.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + plan->partial_offset);
+    L.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
     L.status = status;
     e = launch_decode(L, s);
   } else {

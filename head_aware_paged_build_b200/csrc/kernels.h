@@ -43,6 +43,7 @@ struct DecodeLaunch {
   float* lse;     // [B, Hq] or null
   float scale_log2;  // softmax scale * log2(e)
   float* partial;    // workspace partial slots
+  int32_t* counters; // workspace arrival counters of split heads (zero between calls)
   int32_t* status;
 };
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t s);

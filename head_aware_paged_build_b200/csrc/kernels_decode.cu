@@ -10,9 +10,12 @@
 // run on mma.sync m16n8k16 with the GQA group's q-heads as the 16 rows, and
 // the online softmax runs on the accumulator fragments with quad shuffles.
 // At the end of a head's range the 4 warps' states merge through shared
-// memory in a fixed order, so results are bitwise reproducible.
+// memory in a fixed order, so results are bitwise reproducible.  A head split
+// across CTAs is finished by whichever of its CTAs publishes its partial last
+// (an arrival counter in the workspace): it merges the partials in slot order.
 //
-// fp32: a plain SIMT kernel over the same work list (FP32 FMA only).
+// fp32: a plain SIMT kernel over the same work list (FP32 FMA only), with a
+// separate combine pass for split heads.
 #include <cmath>
 
 #include "device_common.cuh"
@@ -44,6 +47,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
   constexpr int KSTEPS = D / 16;
   constexpr int NT = D / 8;  // n-tiles of the output
   extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ int s_last;
   uint8_t* stage = smem + S::kStageOff;
   float* mbuf = reinterpret_cast<float*>(smem + S::kMergeOff);
   float* mlbuf = reinterpret_cast<float*>(smem + S::kMlOff);
@@ -230,9 +234,65 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
         static_cast<__nv_bfloat16*>(a.out)[o_idx] = __float2bfloat16_rn(acc / L);
         if (col == 0 && a.lse) a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + row] = (M + log2f(L)) * kLn2;
       } else {
-        float* slot = a.partial + int64_t(item.slot) * G * (D + 2);
+        float* slot = a.partial + int64_t(item.slot) * partial_slot_floats(G, D);
         slot[row * D + col] = acc;
         if (col == 0) slot[G * D + row * 2] = M, slot[G * D + row * 2 + 1] = L;
+      }
+    }
+    if (item.slot >= 0) {
+      // Split head: publish this partial, take a ticket; the last of the head's
+      // n_slots CTAs merges all partials in slot order (fixed order: bitwise
+      // reproducible) and returns the counter to zero for the next call.
+      __threadfence();
+      asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+      if (threadIdx.x == 0) s_last = atomicAdd(&a.counters[item.comb], 1) == item.n_slots - 1;
+      asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+      if (s_last) {
+        __threadfence();
+        const int ns = item.n_slots;
+        const int64_t stride = partial_slot_floats(G, D);
+        const float* p0 = a.partial + int64_t(item.slot0) * stride;
+        float* row_m = mlbuf;              // [G] merged max
+        float* row_l = mlbuf + kMaxGroup;  // [G] merged sum
+        // per row: max and weighted sum over the slots, one warp per row
+        for (int row = warp; row < G; row += kConsumerWarps) {
+          float m = -INFINITY;
+          for (int i = lane; i < ns; i += 32) m = fmaxf(m, __ldcg(p0 + i * stride + G * D + row * 2));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          const float base = m == -INFINITY ? 0.f : m;
+          float l = 0.f;
+          for (int i = lane; i < ns; i += 32) {
+            const float* ml = p0 + i * stride + G * D + row * 2;
+            l += fast_exp2(__ldcg(ml) - base) * __ldcg(ml + 1);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+          if (lane == 0) row_m[row] = m, row_l[row] = l;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+        // weighted sum of the slots' accumulators, four columns per thread, slots in order
+        for (int e4 = threadIdx.x; e4 < G * D / 4; e4 += kConsumerWarps * 32) {
+          const int row = e4 / (D / 4), col = (e4 % (D / 4)) * 4;
+          const float M = row_m[row], base = M == -INFINITY ? 0.f : M;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+          for (int i = 0; i < ns; ++i) {
+            const float* sl = p0 + i * stride;
+            const float f = fast_exp2(__ldcg(sl + G * D + row * 2) - base);
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(sl + row * D + col));
+            acc.x += f * v.x, acc.y += f * v.y, acc.z += f * v.z, acc.w += f * v.w;
+          }
+          const float inv = 1.f / row_l[row];
+          __nv_bfloat16* o =
+              static_cast<__nv_bfloat16*>(a.out) + (int64_t(hd.q_row0) * a.num_q_heads + qh0 + row) * D + col;
+          reinterpret_cast<uint2*>(o)[0] = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv),
+                                                      pack_bf16x2(acc.z * inv, acc.w * inv));
+        }
+        if (threadIdx.x < G && a.lse)
+          a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + threadIdx.x] =
+              (row_m[threadIdx.x] + log2f(row_l[threadIdx.x])) * kLn2;
+        if (threadIdx.x == 0) a.counters[item.comb] = 0;
       }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
@@ -330,7 +390,7 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(DecodeLaunch a)
         static_cast<float*>(a.out)[o_idx] = acc[j] / L;
         if (col == 0 && a.lse) a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + row] = (M + log2f(L)) * kLn2;
       } else {
-        float* slot = a.partial + int64_t(item.slot) * G * (D + 2);
+        float* slot = a.partial + int64_t(item.slot) * partial_slot_floats(G, D);
         slot[row * D + col] = acc[j];
         if (col == 0) slot[G * D + row * 2] = M, slot[G * D + row * 2 + 1] = L;
       }
@@ -351,14 +411,14 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeLaunch a) {
   const HeadDesc hd = a.heads[ci.head];
   float M = -INFINITY;
   for (int i = 0; i < ci.n_slots; ++i)
-    M = fmaxf(M, a.partial[int64_t(ci.slot_begin + i) * G * (D + 2) + G * D + row * 2]);
+    M = fmaxf(M, a.partial[int64_t(ci.slot_begin + i) * partial_slot_floats(G, D) + G * D + row * 2]);
   const float base = M == -INFINITY ? 0.f : M;
   float acc[D / 32];
 #pragma unroll
   for (int j = 0; j < D / 32; ++j) acc[j] = 0.f;
   float L = 0.f;
   for (int i = 0; i < ci.n_slots; ++i) {
-    const float* slot = a.partial + int64_t(ci.slot_begin + i) * G * (D + 2);
+    const float* slot = a.partial + int64_t(ci.slot_begin + i) * partial_slot_floats(G, D);
     const float mi = slot[G * D + row * 2];
     const float f = FAST ? fast_exp2(mi - base) : exp2f(mi - base);
     L += f * slot[G * D + row * 2 + 1];
@@ -386,10 +446,7 @@ cudaError_t launch_bf16(const DecodeLaunch& a, cudaStream_t s) {
   auto kern = decode_bf16_kernel<D, kStagesBf16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kBytes);
   if (e != cudaSuccess) return e;
-  kern<<<a.n_ctas, kDecodeThreads, Sm::kBytes, s>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || a.n_combine == 0) return e;
-  combine_kernel<__nv_bfloat16, D, true><<<(a.n_combine * a.group + 3) / 4, 128, 0, s>>>(a);
+  kern<<<a.n_ctas, kDecodeThreads, Sm::kBytes, s>>>(a);  // split heads are merged in-kernel
   return cudaGetLastError();
 }
 

@@ -12,8 +12,8 @@
 //
 // The array lives for as long as the library is loaded, once on every GPU that
 // loads it, and is shared by every call on that GPU.  It keeps the last call's
-// contents; the only part that must start at zero (the status word) is
-// cleared by each call.  Calls whose kernels overlap on the GPU (different
+// contents; the parts that must start at zero (the status word and the split
+// heads' arrival counters) are cleared by each call.  Calls whose kernels overlap on the GPU (different
 // streams, or different host threads, same device) race on the array and
 // corrupt each other's partial results: serialise them.
 #include <cmath>
@@ -85,11 +85,10 @@ extern "C" sp_status segpaged_attention_decode_noalloc(const sp_plan* plan, cons
 
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* status = d_status ? d_status : static_cast<int32_t*>(scratch);
-  if (!d_status) {
-    // the status word is the only scratch that must start at zero
-    e = cudaMemsetAsync(scratch, 0, kStatusBytes, s);
-    if (e != cudaSuccess) return fail(SP_ERR_CUDA, std::string("clearing the status word: ") + cudaGetErrorString(e));
-  }
+  // The status word and the split heads' arrival counters must start at zero
+  // (the counters return to zero by themselves unless a call was cut short).
+  e = cudaMemsetAsync(scratch, 0, size_t(plan->partial_offset), s);
+  if (e != cudaSuccess) return fail(SP_ERR_CUDA, std::string("clearing the control block: ") + cudaGetErrorString(e));
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(plan->prob.head_dim));
   const uint8_t* tbl = static_cast<const uint8_t*>(d_table);
   DecodeLaunch L{};
@@ -108,7 +107,8 @@ extern "C" sp_status segpaged_attention_decode_noalloc(const sp_plan* plan, cons
   L.page_bytes = plan->sizes.page_bytes;
   L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
   L.scale_log2 = scale * 1.4426950408889634f;
-  L.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + kStatusBytes);
+  L.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + plan->partial_offset);
+  L.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + kStatusBytes);
   L.status = status;
   e = launch_decode(L, s);
   return e == cudaSuccess ? SP_OK : fail(SP_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));

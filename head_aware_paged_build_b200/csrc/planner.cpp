@@ -206,7 +206,7 @@ sp_status plan_build(sp_plan& pl) {
       while (lo < hi) {
         const int h = pl.pages[lo].head;
         const int64_t end = std::min<int64_t>(hi, pl.heads[h].vpage_begin + pl.heads[h].n_vpages);
-        pl.decode_items.push_back(DecodeItem{h, int32_t(lo), int32_t(end), -1});
+        pl.decode_items.push_back(DecodeItem{h, int32_t(lo), int32_t(end), -1, -1, 0, 0, 0});
         lo = end;
       }
       pl.decode_cta_begin.push_back(int32_t(pl.decode_items.size()));
@@ -217,8 +217,16 @@ sp_status plan_build(sp_plan& pl) {
       size_t j = i;
       while (j < pl.decode_items.size() && pl.decode_items[j].head == pl.decode_items[i].head) ++j;
       if (j - i > 1) {
+        const int32_t comb = int32_t(pl.combine.size());
         pl.combine.push_back(CombineItem{pl.decode_items[i].head, n_slots, int32_t(j - i), 0});
-        for (size_t k = i; k < j; ++k) pl.decode_items[k].slot = n_slots++;
+        const int32_t slot0 = n_slots;
+        for (size_t k = i; k < j; ++k) {
+          DecodeItem& d = pl.decode_items[k];
+          d.slot = n_slots++;
+          d.comb = comb;
+          d.n_slots = int32_t(j - i);
+          d.slot0 = slot0;
+        }
       }
       i = j;
     }
@@ -315,8 +323,10 @@ sp_status plan_build(sp_plan& pl) {
   z.pool_pages = p.first_page + max_id + 1;
   z.page_bytes = int64_t(P) * D * pl.elem_bytes;
   z.table_bytes = int64_t(pl.blob.size());
-  const int64_t partial = int64_t(n_slots) * pl.group * (D + 2) * 4;
-  z.workspace_bytes = kStatusBytes + ceil_div(partial, 256) * 256;
+  // workspace: status word block | one arrival counter per split head | partial slots
+  const int64_t partial = int64_t(n_slots) * partial_slot_floats(pl.group, D) * 4;
+  pl.partial_offset = kStatusBytes + ceil_div(int64_t(pl.combine.size()) * 4, 256) * 256;
+  z.workspace_bytes = pl.partial_offset + ceil_div(partial, 256) * 256;
   z.stored_token_heads = stored;
   z.dense_token_heads = dense_rows;
   z.visible_pairs = visible;
@@ -325,6 +335,9 @@ sp_status plan_build(sp_plan& pl) {
   z.num_decode_ctas = H.n_decode_ctas;
   z.num_prefill_items = H.n_prefill_items;
   z.num_combine = H.n_combine;
+  // bf16 decode merges split heads inside its kernel; fp32 decode adds a combine pass
+  z.launches_per_call = decode ? (H.n_decode_ctas > 0) + (p.dtype == SP_F32 && H.n_combine > 0)
+                               : (H.n_prefill_items > 0);
   return SP_OK;
 }
 

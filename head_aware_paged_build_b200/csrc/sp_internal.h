@@ -8,6 +8,12 @@
 
 #include "segpaged.h"
 
+#if defined(__CUDACC__)
+#define SP_HD __host__ __device__
+#else
+#define SP_HD
+#endif
+
 namespace sp {
 
 constexpr int32_t kTableMagic = 0x53504731;  // "SPG1"
@@ -15,6 +21,10 @@ constexpr int kStatusBytes = 256;            // workspace prefix holding the sta
 constexpr int kPrefillTileTokensBf16 = 128;  // KV / query tile of the tcgen05 prefill kernel
 constexpr int kPrefillTileTokensF32 = 64;    // KV / query tile of the fp32 prefill kernel
 constexpr int kMaxGroup = 16;                // q-heads per kv-head handled by one decode CTA
+
+// Floats of one decode partial-result slot: acc [G][D], then (m, l) per row in
+// a 4G-float block, so that every slot starts 16-byte aligned.
+SP_HD constexpr int64_t partial_slot_floats(int G, int D) { return int64_t(G) * (D + 4); }
 
 // Device status codes (workspace word 0); the first error sticks.
 enum DeviceCode : int32_t {
@@ -59,7 +69,12 @@ struct alignas(16) DecodeItem {
   int32_t vp_begin;  // global page-array indices [vp_begin, vp_end)
   int32_t vp_end;
   int32_t slot;      // partial-result slot in the workspace, or -1: the item covers the head
+  int32_t comb;      // split head index (arrival counter), -1 if not split
+  int32_t n_slots;   // items the split head has
+  int32_t slot0;     // first slot of the split head
+  int32_t pad;
 };
+static_assert(sizeof(DecodeItem) == 32, "DecodeItem layout");
 
 // A head whose decode result is split across several items.
 struct alignas(16) CombineItem {
@@ -120,6 +135,7 @@ struct sp_plan {
   int32_t elem_bytes = 4;
   int32_t prefill_tile = 0;
   int32_t n_partial_slots = 0;
+  int64_t partial_offset = 0;  // workspace byte offset of the partial slots (status word, then counters)
 };
 
 namespace sp {

@@ -58,16 +58,14 @@ class sp_sizes(ctypes.Structure):
                 ("stored_token_heads", ctypes.c_int64), ("dense_token_heads", ctypes.c_int64),
                 ("visible_pairs", ctypes.c_int64), ("num_queries", ctypes.c_int64), ("is_decode", ctypes.c_int32),
                 ("num_decode_ctas", ctypes.c_int32), ("num_prefill_items", ctypes.c_int32),
-                ("num_combine", ctypes.c_int32)]
+                ("num_combine", ctypes.c_int32), ("launches_per_call", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
 
     def kernel_launches(self) -> int:
         """Kernels one segpaged_attention call launches."""
-        if self.is_decode:
-            return (1 if self.num_decode_ctas else 0) + (1 if self.num_combine else 0)
-        return 1 if self.num_prefill_items else 0
+        return int(self.launches_per_call)
 
 
 class sp_segment(ctypes.Structure):

@@ -125,7 +125,8 @@ typedef struct {
   int32_t is_decode;          /* 1 if every C_b == 1 */
   int32_t num_decode_ctas;    /* decode grid size (0 for prefill plans) */
   int32_t num_prefill_items;  /* prefill grid size (0 for decode plans) */
-  int32_t num_combine;        /* decode heads split across CTAs (> 0: a combine pass runs) */
+  int32_t num_combine;        /* decode heads split across CTAs */
+  int32_t launches_per_call;  /* kernels one segpaged_attention call launches */
 } sp_sizes;
 
 /* One contiguous run of stored positions of a head; it starts on a fresh page. */
@@ -195,8 +196,12 @@ SP_API sp_status segpaged_gather(const sp_plan* plan, const void* d_table, const
  *   out  device, same shape and dtype as q
  *   lse  device [sum_b C_b, num_q_heads] fp32 natural-log sum-exp, or NULL
  *   softmax_scale  <= 0 selects 1/sqrt(head_dim)
- *   workspace      device, >= workspace_bytes, 256-byte aligned; its first
- *                  256 bytes hold the device status word
+ *   workspace      device, >= workspace_bytes, 256-byte aligned, zero-filled
+ *                  before its first use; it holds the device status word (first
+ *                  256 bytes), one arrival counter per split decode head (the
+ *                  kernels return them to zero) and the split partial results.
+ *                  After a non-zero device status, zero it again before reuse.
+ *                  Calls that overlap on the GPU need separate workspaces.
  * Decode plans run a split-KV kernel over each head's own pages plus a
  * combine pass; prefill plans run one tile kernel (tcgen05 for bf16). */
 SP_API sp_status segpaged_attention(const sp_plan* plan, const void* d_table, const void* k_pool,
@@ -221,8 +226,8 @@ SP_API sp_status segpaged_attention(const sp_plan* plan, const void* d_table, co
  *     up the array's device address (cudaGetSymbolAddress) with that device
  *     current; make that first call before any stream capture.
  *   - All calls on one GPU share the array and leave their contents in it.
- *     Each call clears the status word; the partial results need no
- *     clearing.  Calls whose kernels overlap on the GPU race on the array:
+ *     Each call clears the status word and the split heads' arrival
+ *     counters; the partial results need no clearing.  Calls whose kernels overlap on the GPU race on the array:
  *     serialise them.
  *   - d_status: NULL, or a device int32 the caller owns (and clears) that
  *     receives the device status code instead of the built-in word.
