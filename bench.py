@@ -57,9 +57,9 @@ def config_of(wl, n_gpus: int) -> dict:
         kinds[k] = kinds.get(k, 0) + 1
     loc = next(((s, w) for k, s, w in wl.policy if k == "local"), None)
     return {
-        "workload": {"llama": "Llama-70B-shaped layer, 32K context", "mistral": "Mistral-7B-shaped layer, 8K context",
-                     "mha": "MHA-style layer, 128K context", "ragged": "ragged decode batch"}.get(
-                         wl.name.split("_")[0], wl.name),
+        "workload": ("Llama-70B-shaped layer, 32K context" if wl.name.startswith("llama")
+                     else {"mistral": "Mistral-7B-shaped layer, 8K context", "mha": "MHA-style layer, 128K context",
+                           "ragged": "ragged decode batch"}.get(wl.name, wl.name)),
         "batch": wl.batch, "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
         "context": max(wl.ctx_lens), "page_size": wl.page_size, "prefill_chunk": wl.prefill_chunk,
         "heads": {"global": kinds.get("global", 0), "local": kinds.get("local", 0)},
@@ -414,7 +414,7 @@ def main() -> None:
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="llama", choices=("llama", "mistral", "mha"))
+    ap.add_argument("--workload", default="llama", choices=("llama", "mistral", "mha", "llama_b1"))
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="time budget of the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -139,6 +139,59 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic) and 3-input max ----------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair, on the FMA and integer pipes instead of the SFU.
+// x = n + f with n = round(x) (adding 1.5 * 2^23 rounds to an integer held in
+// the low mantissa bits) and f in [-1/2, 1/2]; 2^f is a cubic fitted by
+// weighted least squares on 64 Chebyshev nodes of [-1/2, 1/2] (maximum
+// relative error 7.7e-5, below bf16's 2^-8 rounding of P); n is added to the
+// exponent field.  x is clamped at -126 so the exponent never wraps: lanes
+// below that (masked, -inf) give ~1e-38, which vanishes next to the row's
+// largest weight (>= 1) in every fp32 sum.
+__device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& e0, float& e1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x0 = fmaxf(x0, -126.f), x1 = fmaxf(x1, -126.f);
+  const uint64_t xc = f2_pack(x0, x1);
+  const uint64_t t = f2_add(xc, f2_pack(kRound, kRound));
+  const uint64_t j = f2_add(t, f2_pack(-kRound, -kRound));
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), xc);
+  uint64_t p = f2_fma(f2_pack(0.05508868396282196f, 0.05508868396282196f), f,
+                      f2_pack(0.24260404706001282f, 0.24260404706001282f));
+  p = f2_fma(p, f, f2_pack(0.6932762265205383f, 0.6932762265205383f));
+  p = f2_fma(p, f, f2_pack(0.9999289512634277f, 0.9999289512634277f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 // Visibility of key position `a` for query position `p` of a head:
 // causal, and for a local head inside the sink or the recent window.
 __device__ __forceinline__ bool sees(int local, int sink, int window, int p, int a) {

@@ -287,25 +287,33 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if (!(c < h1 || (c >= l2 && c < h2))) v[e] = -INFINITY;
           }
         };
-        // pass 1: the row maximum (S stays in TMEM; 64 columns in registers at a time)
-        float mx[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-#pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-          float va[32], vb[32];
-          tc::tmem_ld32(t_s(x) + lane_off + hc * 64, va);
-          tc::tmem_ld32(t_s(x) + lane_off + hc * 64 + 32, vb);
+        // pass 1: the row maximum (S stays in TMEM).  The second pair of loads is
+        // in flight while the first pair is reduced.
+        float mx[4];
+        {
+          float va[32], vb[32], vc[32], vd[32];
+          tc::tmem_ld32(t_s(x) + lane_off, va);
+          tc::tmem_ld32(t_s(x) + lane_off + 32, vb);
           tc::tmem_wait_ld();
+          tc::tmem_ld32(t_s(x) + lane_off + 64, vc);
+          tc::tmem_ld32(t_s(x) + lane_off + 96, vd);
           if (!full) {
-            mask32(va, 2 * hc);
-            mask32(vb, 2 * hc + 1);
+            mask32(va, 0);
+            mask32(vb, 1);
           }
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], fmaxf(va[e], vb[e]));
+          for (int i = 0; i < 4; ++i) mx[i] = fmax3(va[i], vb[i], -INFINITY);
+#pragma unroll
+          for (int e = 4; e < 32; ++e) mx[e & 3] = fmax3(mx[e & 3], va[e], vb[e]);
+          tc::tmem_wait_ld();
+          if (!full) {
+            mask32(vc, 2);
+            mask32(vd, 3);
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx[e & 3] = fmax3(mx[e & 3], vc[e], vd[e]);
         }
-        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), mx[3], -INFINITY);
         const float mts = mt * sl2;
         float alpha = 1.f;
         bool need = false;
@@ -330,25 +338,41 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         // pass 2: P = 2^(s - m) in bf16, written over S columns already consumed:
         // chunk c of S (columns [32 c, 32 c + 32)) becomes P columns [16 c, 16 c + 16).
+        // Chunk c + 1 is loading while chunk c is exponentiated; one pair in four
+        // takes its 2^x on the FMA pipe so that the SFU is not the bottleneck.
         const float base = m_run == -INFINITY ? 0.f : m_run;
-        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint64_t scale2 = f2_pack(sl2, sl2), nbase2 = f2_pack(-base, -base);
+        uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        float vbuf[2][32];
+        tc::tmem_ld32(t_s(x) + lane_off, vbuf[0]);
+        tc::tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < kTile / 32; ++c) {
-          float v[32];
-          tc::tmem_ld32(t_s(x) + lane_off + c * 32, v);
-          tc::tmem_wait_ld();
+          float (&v)[32] = vbuf[c & 1];
+          if (c + 1 < kTile / 32) tc::tmem_ld32(t_s(x) + lane_off + (c + 1) * 32, vbuf[(c + 1) & 1]);
           if (!full) mask32(v, c);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float e0 = fast_exp2(fmaf(v[2 * e], sl2, -base));
-            const float e1 = fast_exp2(fmaf(v[2 * e + 1], sl2, -base));
-            sum[e & 3] += e0 + e1;
+            const uint64_t x2 = f2_fma(f2_pack(v[2 * e], v[2 * e + 1]), scale2, nbase2);
+            float e0, e1;
+            if ((e & 3) == 3) {
+              exp2_poly_pair(x2, e0, e1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+            }
+            sum2[e & 1] = f2_add(sum2[e & 1], f2_pack(e0, e1));
             pk[e] = pack_bf16x2(e0, e1);
           }
           tc::tmem_st16(t_s(x) + lane_off + c * 16, pk);
+          if (c + 1 < kTile / 32) tc::tmem_wait_ld();
         }
-        l_run = l_run * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+        float s0, s1, s2, s3;
+        f2_unpack(sum2[0], s0, s1);
+        f2_unpack(sum2[1], s2, s3);
+        l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
         tc::tmem_wait_st();
         tc::fence_before_sync();
         mbar_arrive(&bars->p_full[x]);

@@ -206,12 +206,17 @@ def llama_layer_globals(n_layers: int = 80) -> list[int]:
     return [rnd.randrange(8) for _ in range(n_layers)]
 
 
-def llama(layer: int = 0) -> Workload:
-    """Llama-70B-shaped layer: B8, 64/8 heads, d128, bf16, 32K context, page 64; 1 of 8 kv-heads global."""
+def llama(layer: int = 0, batch: int = 8) -> Workload:
+    """Llama-70B-shaped layer: B8, 64/8 heads, d128, bf16, 32K context, page 64; 1 of 8 kv-heads global.
+
+    ``batch=1`` keeps sequence 0 only: the same per-sequence work at one eighth
+    of the memory (used for detailed profiles).
+    """
     g = llama_layer_globals()[layer]
     row = tuple(GLOBAL if h == g else _local(4, 8192) for h in range(8))
-    return Workload(f"llama_l{layer}", 2 + 1000 * layer, 8, 64, 8, 128, "bf16", 64, (32768,) * 8,
-                    row * 8, prefill_chunk=4096)
+    name = f"llama_l{layer}" if batch == 8 else f"llama_l{layer}_b{batch}"
+    return Workload(name, 2 + 1000 * layer, batch, 64, 8, 128, "bf16", 64, (32768,) * batch,
+                    row * batch, prefill_chunk=4096)
 
 
 def ragged() -> Workload:
@@ -235,7 +240,8 @@ def mha() -> Workload:
                     prefill_chunk=4096)
 
 
-ALL = {"tiny": tiny, "mistral": mistral, "llama": llama, "ragged": ragged, "mha": mha}
+ALL = {"tiny": tiny, "mistral": mistral, "llama": llama, "ragged": ragged, "mha": mha,
+       "llama_b1": lambda: llama(batch=1)}
 
 
 def custom(name: str, seed: int, batch: int, hq: int, hkv: int, d: int, dtype: str, page: int,
