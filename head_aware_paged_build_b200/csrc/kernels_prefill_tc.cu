@@ -49,6 +49,11 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by more than 2^8
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kFull = 0xffffffffu;
+// One exponent pair in every kPolyPeriod is computed on the FMA pipe (0: none).
+#ifndef SP_EXP2_POLY_PERIOD
+#define SP_EXP2_POLY_PERIOD 4
+#endif
+constexpr int kPolyPeriod = SP_EXP2_POLY_PERIOD;
 
 template <int D, int NS>
 struct TcSmem {
@@ -257,11 +262,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const float sl2 = a.scale_log2;
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
+      // The page descriptors of tile j + 1 are fetched while tile j is processed.
+      auto fetch_descs = [&](int j, PageDesc& d0, PageDesc& d1) {
+        const int t = tile_of(j);
+        d0 = a.pages[hd.vpage_begin + 2 * t];
+        d1 = a.pages[hd.vpage_begin + min(2 * t + 1, hd.n_vpages - 1)];
+      };
+      PageDesc nx0{}, nx1{};
+      if (n > 0) fetch_descs(0, nx0, nx1);
       for (int j = 0; j < n; ++j) {
         const int t = tile_of(j);
         const bool have1 = 2 * t + 1 < hd.n_vpages;
-        const PageDesc pg0 = a.pages[hd.vpage_begin + 2 * t];
-        const PageDesc pg1 = have1 ? a.pages[hd.vpage_begin + 2 * t + 1] : PageDesc{0, 0, 0, 0};
+        const PageDesc pg0 = nx0;
+        const PageDesc pg1 = have1 ? nx1 : PageDesc{0, 0, 0, 0};
+        if (j + 1 < n) fetch_descs(j + 1, nx0, nx1);
         const bool full = page_fully_visible(pg0, true, hd, p_first, p_last) &&
                           page_fully_visible(pg1, have1, hd, p_first, p_last);
         // tcgen05.ld / st are warp-collective (.sync.aligned): every branch that
@@ -313,6 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
           for (int e = 0; e < 32; ++e) mx[e & 3] = fmax3(mx[e & 3], vc[e], vd[e]);
         }
+        // pass 2's first chunk loads while the maximum is finished
+        float vbuf[2][32];
+        tc::tmem_ld32(t_s(x) + lane_off, vbuf[0]);
         const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), mx[3], -INFINITY);
         const float mts = mt * sl2;
         float alpha = 1.f;
@@ -343,8 +360,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const float base = m_run == -INFINITY ? 0.f : m_run;
         const uint64_t scale2 = f2_pack(sl2, sl2), nbase2 = f2_pack(-base, -base);
         uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-        float vbuf[2][32];
-        tc::tmem_ld32(t_s(x) + lane_off, vbuf[0]);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < kTile / 32; ++c) {
@@ -356,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           for (int e = 0; e < 16; ++e) {
             const uint64_t x2 = f2_fma(f2_pack(v[2 * e], v[2 * e + 1]), scale2, nbase2);
             float e0, e1;
-            if ((e & 3) == 3) {
+            if (kPolyPeriod > 0 && (e % (kPolyPeriod > 0 ? kPolyPeriod : 1)) == kPolyPeriod - 1) {
               exp2_poly_pair(x2, e0, e1);
             } else {
               float x0, x1;
