@@ -159,6 +159,37 @@ sp_status segpaged_attention(const sp_plan* plan, const void* d_table, const voi
   return e == cudaSuccess ? SP_OK : cuda_fail(e, "segpaged_attention launch");
 }
 
+sp_status segpaged_decode_append(const sp_plan* plan, void* d_table, const void* k_new, const void* v_new,
+                                 int64_t stride_seq, int64_t stride_head, void* k_pool, void* v_pool, void* workspace,
+                                 void* stream) {
+  using namespace sp;
+  sp_status st = check_table(plan, d_table);
+  if (st != SP_OK) return st;
+  if (!(plan->prob.flags & SP_FLAG_RING)) return fail(SP_ERR_INVALID_ARG, "segpaged_decode_append needs a ring plan");
+  if (!k_new || !v_new || !k_pool || !v_pool || !workspace)
+    return fail(SP_ERR_INVALID_ARG, "k_new, v_new, pools and workspace must be non-NULL");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
+      !aligned(workspace, 256))
+    return fail(SP_ERR_INVALID_ARG, "new rows and pools must be 16-byte aligned, workspace 256-byte aligned");
+  const int64_t eb = plan->elem_bytes;
+  if (stride_seq < 0 || stride_head < 0 || (stride_seq * eb) % 16 || (stride_head * eb) % 16)
+    return fail(SP_ERR_INVALID_ARG, "strides must be >= 0 and give 16-byte aligned rows");
+  AppendLaunch L{};
+  L.heads = const_cast<HeadDesc*>(section<HeadDesc>(d_table, plan->hdr.off_heads));
+  L.pages = const_cast<PageDesc*>(section<PageDesc>(d_table, plan->hdr.off_pages));
+  L.n_heads = plan->hdr.n_heads;
+  L.D = plan->prob.head_dim;
+  L.P = plan->prob.page_size;
+  L.bf16 = plan->prob.dtype == SP_BF16;
+  L.stride_seq = stride_seq;
+  L.stride_head = stride_head;
+  L.page_bytes = plan->sizes.page_bytes;
+  L.k_new = k_new, L.v_new = v_new, L.kpool = k_pool, L.vpool = v_pool;
+  L.status = static_cast<int32_t*>(workspace);
+  const cudaError_t e = launch_append(L, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SP_OK : cuda_fail(e, "segpaged_decode_append launch");
+}
+
 sp_status segpaged_read_device_status(const void* workspace, int32_t* code, void* stream) {
   if (!workspace || !code) return sp::fail(SP_ERR_INVALID_ARG, "workspace and code must be non-NULL");
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

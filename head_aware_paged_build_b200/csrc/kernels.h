@@ -66,4 +66,19 @@ struct PrefillLaunch {
 };
 cudaError_t launch_prefill(const PrefillLaunch& L, cudaStream_t s);
 
+struct AppendLaunch {
+  HeadDesc* heads;  // device table, updated in place
+  PageDesc* pages;
+  int32_t n_heads;
+  int32_t D, P;
+  bool bf16;
+  int64_t stride_seq, stride_head, page_bytes;
+  const void* k_new;  // [B, Hkv, D] with the given strides (elements)
+  const void* v_new;
+  void* kpool;
+  void* vpool;
+  int32_t* status;
+};
+cudaError_t launch_append(const AppendLaunch& a, cudaStream_t s);
+
 }  // namespace sp

@@ -80,11 +80,16 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
           record_error(a.status, kDevTimeoutEmpty);
           break;
         }
-        const int64_t phys = a.pages[g].phys;
+        const PageDesc pgd = a.pages[g];
+        const int64_t phys = pgd.phys;
         uint8_t* kd = stage + s * 2 * PB;
-        mbar_arrive_expect_tx(&full[s], 2 * PB);
-        bulk_g2s(kd, kpool + phys * a.page_bytes, PB, &full[s]);
-        bulk_g2s(kd + PB, vpool + phys * a.page_bytes, PB, &full[s]);
+        if (slot_hi(pgd) > slot_lo(pgd)) {
+          mbar_arrive_expect_tx(&full[s], 2 * PB);
+          bulk_g2s(kd, kpool + phys * a.page_bytes, PB, &full[s]);
+          bulk_g2s(kd + PB, vpool + phys * a.page_bytes, PB, &full[s]);
+        } else {
+          mbar_arrive(&full[s]);  // empty page (ring or reserved): nothing to copy
+        }
       }
       // Do not leave while copies into this CTA's shared memory are in flight.
       const int n = ge - gb;
@@ -131,7 +136,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
       }
       const PageDesc pg = a.pages[g];
       const int tok0 = warp * 16;
-      if (ok && tok0 < pg.nvalid) {
+      const int lo = slot_lo(pg), hi = slot_hi(pg);
+      if (ok && tok0 < hi && tok0 + 16 > lo) {
         const uint32_t kst = smem_u32(stage + s * 2 * PB);
         const uint32_t vst = kst + PB;
         // S = Q K^T over this warp's 16 tokens (two n8 tiles)
@@ -151,7 +157,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int tok = tok0 + n * 8 + tq * 2 + (e & 1);
-            bool vis = tok < pg.nvalid;
+            bool vis = tok >= lo && tok < hi;
             if (hd.mask_local) vis = vis && sees(1, hd.sink, hd.window, qpos, pg.abs_start + tok);
             sc[n][e] = vis ? sc[n][e] * a.scale_log2 : -INFINITY;
           }
@@ -343,7 +349,7 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(DecodeLaunch a)
       __syncthreads();
       for (int e = threadIdx.x; e < G * P; e += kF32Threads) {
         const int h = e / P, t = e % P;
-        bool vis = t < pg.nvalid;
+        bool vis = t >= slot_lo(pg) && t < slot_hi(pg);
         if (hd.mask_local) vis = vis && sees(1, hd.sink, hd.window, qpos, pg.abs_start + t);
         float s = 0.f;
         for (int i = 0; i < D; ++i) s = fmaf(qs[h * D + i], kp[t * D + i], s);

@@ -3,8 +3,8 @@
 // One CTA per page: it copies the page's stored rows of dense K/V (16-byte
 // vector loads, consecutive threads on consecutive chunks of a row) into the
 // pool's page layout.  K chunks move straight to their swizzled slot; V is
-// transposed through shared memory.  Slots past the last stored position of a
-// segment are written as zeros so that every pool byte the attention kernels
+// transposed through shared memory.  Slots outside the page's valid range
+// [lo, hi) are written as zeros so that every pool byte the attention kernels
 // read is a finite number ("SegPagedAttention runtime design", §3:
 // build_segpaged_cache packs dense KV and keeps only what a head can see).
 #include "device_common.cuh"
@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(PackArgs a, const T*
   for (int idx = threadIdx.x; idx < P * CR; idx += kPackThreads) {
     const int t = idx / CR, c = idx % CR;
     uint4 kv4 = make_uint4(0, 0, 0, 0), vv4 = make_uint4(0, 0, 0, 0);
-    if (t < pg.nvalid) {
+    if (t >= slot_lo(pg) && t < slot_hi(pg)) {
       const int64_t row = base + int64_t(pg.abs_start + t) * a.stride_tok;
       kv4 = __ldg(reinterpret_cast<const uint4*>(kd + row) + c);
       vv4 = __ldg(reinterpret_cast<const uint4*>(vd + row) + c);
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kPackThreads) gather_kernel(PackArgs a, const 
   __syncthreads();
   for (int idx = threadIdx.x; idx < P * CR; idx += kPackThreads) {
     const int t = idx / CR, c = idx % CR;
-    if (t >= pg.nvalid) continue;
+    if (t < slot_lo(pg) || t >= slot_hi(pg)) continue;
     const int64_t row = base + int64_t(pg.abs_start + t) * a.stride_tok;
     reinterpret_cast<uint4*>(kd + row)[c] = *reinterpret_cast<const uint4*>(ksrc + kpage_chunk<T>(t, c, P, D));
     const uint32_t* s = stage + t * PW + c * 4;

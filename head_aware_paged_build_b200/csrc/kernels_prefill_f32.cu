@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kRows) prefill_f32_kernel(PrefillLaunch a) {
           const int ii = e / P, t2 = e % P;
           vs[ii * kRows + j * P + t2] = have ? vpp[e] : 0.f;
         }
-        for (int tt = threadIdx.x; tt < P; tt += kRows) pos[j * P + tt] = (have && tt < pg.nvalid) ? pg.abs_start + tt : -1;
+        for (int tt = threadIdx.x; tt < P; tt += kRows) pos[j * P + tt] = (have && tt >= slot_lo(pg) && tt < slot_hi(pg)) ? pg.abs_start + tt : -1;
       }
       __syncthreads();
       if (!active) continue;

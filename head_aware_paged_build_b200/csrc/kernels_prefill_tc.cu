@@ -79,26 +79,28 @@ struct Bars {
 // Does every row p in [p_first, p_last] see every slot of this page?
 __device__ __forceinline__ bool page_fully_visible(const PageDesc& pg, bool exists, const HeadDesc& hd, int p_first,
                                                    int p_last) {
-  if (!exists || pg.nvalid != 64) return false;
+  if (!exists || pg.span != make_span(0, 64)) return false;
   const int a0 = pg.abs_start, a1 = pg.abs_start + 63;
   if (a1 > p_first) return false;
   if (hd.kind == 0) return true;
   return a1 < hd.sink || a0 > p_last - hd.window;
 }
 
-// Slots of a page visible to row p: [0, h1) and [l2, h2) (possibly empty).
+// Slots of a page visible to row p: [0, h1) (sink run) and [l2, h2) (causal
+// part / recent window), inside the page's valid range [lo, hi).  A page with
+// lo > 0 never holds sink positions (sink pages always start at slot 0; only
+// ring pages of decode plans start later), so its sink run is empty.
 __device__ __forceinline__ void visible_slots(const PageDesc& pg, bool exists, const HeadDesc& hd, int p, int& h1,
                                               int& l2, int& h2) {
-  if (!exists) {
-    h1 = 0, l2 = 0, h2 = 0;
-    return;
-  }
-  const int causal = min(pg.nvalid, p - pg.abs_start + 1);  // positions <= p
+  h1 = l2 = h2 = 0;
+  if (!exists) return;
+  const int lo = slot_lo(pg);
+  const int causal = min(slot_hi(pg), p - pg.abs_start + 1);  // valid slots with position <= p
   if (hd.kind == 0) {
-    h1 = causal, l2 = 0, h2 = 0;
+    l2 = lo, h2 = causal;
   } else {
-    h1 = min(causal, hd.sink - pg.abs_start);           // sink run
-    l2 = max(0, p - hd.window + 1 - pg.abs_start);      // recent window
+    h1 = lo > 0 ? 0 : min(causal, hd.sink - pg.abs_start);     // sink run
+    l2 = max(lo, p - hd.window + 1 - pg.abs_start);            // recent window
     h2 = causal;
   }
 }

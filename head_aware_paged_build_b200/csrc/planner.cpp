@@ -36,7 +36,12 @@ sp_status validate(const sp_problem& p) {
     return fail(SP_ERR_INVALID_ARG, "batch, head counts, head_dim and page_size must be >= 1");
   if (!p.ctx_len || !p.q_start || !p.policy)
     return fail(SP_ERR_INVALID_ARG, "ctx_len, q_start and policy must be non-NULL host arrays");
-  if (p.flags & ~uint32_t(SP_FLAG_DENSE_MASKED)) return fail(SP_ERR_INVALID_ARG, "unknown flag bits");
+  if (p.flags & ~uint32_t(SP_FLAG_DENSE_MASKED | SP_FLAG_RING)) return fail(SP_ERR_INVALID_ARG, "unknown flag bits");
+  if (p.append_capacity < 0) return fail(SP_ERR_INVALID_ARG, "append_capacity must be >= 0");
+  if (p.append_capacity > 0 && !(p.flags & SP_FLAG_RING))
+    return fail(SP_ERR_INVALID_ARG, "append_capacity needs SP_FLAG_RING");
+  if ((p.flags & SP_FLAG_RING) && (p.flags & SP_FLAG_DENSE_MASKED))
+    return fail(SP_ERR_UNSUPPORTED, "ring plans are SegPaged plans (no dense-masked variant)");
   if (p.first_page < 0) return fail(SP_ERR_INVALID_ARG, "first_page must be >= 0");
   if (p.target_ctas < 0) return fail(SP_ERR_INVALID_ARG, "target_ctas must be >= 0");
   if (p.dtype != SP_F32 && p.dtype != SP_BF16) return fail(SP_ERR_UNSUPPORTED, "dtype must be SP_F32 or SP_BF16");
@@ -64,8 +69,8 @@ sp_status validate(const sp_problem& p) {
       return fail(SP_ERR_UNSUPPORTED, "RETRIEVAL heads are not implemented (no scoring rule is defined)");
     if (h.kind != SP_GLOBAL && h.kind != SP_LOCAL && h.kind != SP_DENSE)
       return fail(SP_ERR_INVALID_ARG, "policy[" + std::to_string(i) + "].kind is not a head kind");
-    if (h.kind == SP_LOCAL && (h.sink < 0 || h.window < 1))
-      return fail(SP_ERR_INVALID_ARG, "policy[" + std::to_string(i) + "]: local heads need sink >= 0, window >= 1");
+    if (h.kind == SP_LOCAL && (h.sink < 0 || h.window == 0))
+      return fail(SP_ERR_INVALID_ARG, "policy[" + std::to_string(i) + "]: local heads need sink >= 0, window != 0");
   }
   return SP_OK;
 }
@@ -113,6 +118,13 @@ sp_status plan_build(sp_plan& pl) {
   for (int b = 0; b < B; ++b) qrow[b + 1] = qrow[b] + (pl.ctx_len[b] - pl.q_start[b]);
   bool decode = true;
   for (int b = 0; b < B; ++b) decode = decode && (pl.ctx_len[b] - pl.q_start[b] == 1);
+  const bool ring = (p.flags & SP_FLAG_RING) != 0;
+  if (ring && !decode) return fail(SP_ERR_UNSUPPORTED, "ring plans are decode plans (one query per sequence)");
+  const int64_t cap = p.append_capacity;
+  if (ring) {
+    for (int b = 0; b < B; ++b)
+      if (int64_t(pl.ctx_len[b]) + cap > (int64_t(1) << 30)) return fail(SP_ERR_UNSUPPORTED, "ctx_len + capacity above 2^30");
+  }
 
   int64_t ctx_row = 0;
   for (int b = 0; b < B; ++b, ctx_row += pl.ctx_len[b - 1]) {
@@ -123,7 +135,9 @@ sp_status plan_build(sp_plan& pl) {
       const int h = b * Hkv + kv;
       const sp_head_policy& pol = pl.policy[h];
       const bool local = pol.kind == SP_LOCAL;
-      const int64_t s = local ? pol.sink : 0, w = local ? pol.window : 0;
+      const int64_t s = local ? pol.sink : 0;
+      // adaptive window (window <= -1): max(1, L / -window) for this sequence
+      const int64_t w = !local ? 0 : pol.window > 0 ? pol.window : std::max<int64_t>(1, L / (-int64_t(pol.window)));
       int64_t firsts[2], lens[2];
       int ns = 0;
       if (!local || dense_masked) {
@@ -136,6 +150,20 @@ sp_status plan_build(sp_plan& pl) {
         } else {
           if (sink_len > 0) firsts[ns] = 0, lens[ns++] = sink_len;
           if (rec < L) firsts[ns] = rec, lens[ns++] = L - rec;
+        }
+      }
+      if (ring) {
+        // Ring plan: pages aligned to absolute multiples of P.  GLOBAL: [0, L)
+        // plus pages for `cap` more tokens.  LOCAL: the sink's pages (for all
+        // s positions) and a ring of R pages; position a >= s sits in ring slot
+        // a mod (R P), so appends never move a token.
+        firsts[0] = 0, lens[0] = L, ns = 1;
+        if (local) {
+          const int64_t sink_len = std::min<int64_t>(s, L);
+          const int64_t wlo = std::max<int64_t>(s, L - w), whi = L;
+          ns = 0;
+          if (sink_len > 0) firsts[ns] = 0, lens[ns++] = sink_len;
+          if (whi > wlo) firsts[ns] = wlo, lens[ns++] = whi - wlo;
         }
       }
       HeadDesc& hd = pl.heads[h];
@@ -153,14 +181,47 @@ sp_status plan_build(sp_plan& pl) {
       hd.kv = kv;
       hd.q_row0 = qrow[b];
       int32_t vp = 0;
-      for (int i = 0; i < ns; ++i) {
+      if (ring) {
+        auto add_page = [&](int64_t abs0, int64_t lo, int64_t hi) {
+          PageDesc pd{};
+          pd.abs_start = int32_t(abs0);
+          pd.span = hi > lo ? make_span(int32_t(lo), int32_t(hi)) : 0;
+          pd.head = h;
+          pl.pages.push_back(pd);
+          ++vp;
+        };
+        if (!local) {
+          const int64_t np = ceil_div(L + cap, P);
+          for (int64_t k = 0; k < np; ++k) add_page(k * P, 0, std::clamp<int64_t>(L - k * P, 0, P));
+          pl.segments.push_back(sp_segment{0, int32_t(L), 0, int32_t(np)});
+        } else {
+          const int64_t nsink = ceil_div(s, P);
+          const int64_t sink_len = std::min<int64_t>(s, L);
+          for (int64_t k = 0; k < nsink; ++k) add_page(k * P, 0, std::clamp<int64_t>(sink_len - k * P, 0, P));
+          if (sink_len > 0) pl.segments.push_back(sp_segment{0, int32_t(sink_len), 0, int32_t(nsink)});
+          const int64_t R = ceil_div(w, P) + 1, RP = R * P;
+          const int64_t wlo = std::max<int64_t>(s, L - w), whi = L;
+          for (int64_t i = 0; i < R; ++i) {
+            // latest run of ring page i (positions q RP + i P ...) that starts before whi
+            const int64_t x = whi - 1 - i * P;
+            const int64_t q = x >= 0 ? x / RP : -((-x + RP - 1) / RP);
+            const int64_t run = q * RP + i * P;
+            const int64_t lo = std::max<int64_t>(wlo, run) - run, hi = std::min<int64_t>(whi, run + P) - run;
+            add_page(run, std::max<int64_t>(lo, 0), std::max<int64_t>(hi, 0));
+          }
+          if (whi > wlo)
+            pl.segments.push_back(sp_segment{int32_t(wlo), int32_t(whi - wlo), int32_t(nsink), int32_t(R)});
+        }
+        for (int i = 0; i < ns; ++i) stored += lens[i];
+      }
+      for (int i = 0; i < ns && !ring; ++i) {
         sp_segment g{int32_t(firsts[i]), int32_t(lens[i]), vp, int32_t(ceil_div(lens[i], P))};
         pl.segments.push_back(g);
         for (int k = 0; k < g.num_pages; ++k) {
           PageDesc pd{};
           pd.phys = 0;  // assigned below
           pd.abs_start = g.abs_start + k * P;
-          pd.nvalid = int32_t(std::min<int64_t>(P, int64_t(g.abs_start) + g.length - pd.abs_start));
+          pd.span = make_span(0, int32_t(std::min<int64_t>(P, int64_t(g.abs_start) + g.length - pd.abs_start)));
           pd.head = h;
           pl.pages.push_back(pd);
         }

@@ -34,6 +34,7 @@ enum DeviceCode : int32_t {
   kDevTimeoutMma = 3,      // a wait on a tensor-core commit ran out
   kDevTimeoutSoftmax = 4,  // the MMA issuer gave up waiting for P
   kDevBadPage = 5,         // a page id outside the pool (debug builds)
+  kDevAppendFull = 6,      // an append found no reserved page left (ring plans)
 };
 
 // One (sequence, kv-head).  Kinds are resolved: 0 reads the whole causal
@@ -54,14 +55,20 @@ struct alignas(16) HeadDesc {
 };
 static_assert(sizeof(HeadDesc) == 48, "HeadDesc layout");
 
-// One page of a head, in the head's position order.
+// One page of a head.  Slot t holds position abs_start + t; only slots
+// [lo, hi) hold tokens (lo = span & 0xffff, hi = span >> 16).  Pages of a
+// head are in position order except in ring plans, where the recent window
+// is a ring of pages (see the planner).
 struct alignas(16) PageDesc {
   int32_t phys;       // physical page id in the pools
-  int32_t abs_start;  // absolute position held by slot 0
-  int32_t nvalid;     // slots [0, nvalid) hold positions abs_start .. abs_start + nvalid - 1
+  int32_t abs_start;  // absolute position of slot 0
+  int32_t span;       // lo | hi << 16
   int32_t head;       // owning HeadDesc index
 };
 static_assert(sizeof(PageDesc) == 16, "PageDesc layout");
+SP_HD inline int32_t slot_lo(const PageDesc& p) { return p.span & 0xffff; }
+SP_HD inline int32_t slot_hi(const PageDesc& p) { return p.span >> 16; }
+SP_HD inline int32_t make_span(int32_t lo, int32_t hi) { return lo | (hi << 16); }
 
 // A run of consecutive pages of one head processed by one decode CTA.
 struct alignas(16) DecodeItem {

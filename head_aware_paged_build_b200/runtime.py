@@ -32,13 +32,13 @@ class SegPagedLayer:
                  dtype: str, ctx_len: Sequence[int], q_start: Sequence[int],
                  policy: Sequence[tuple[str, int, int]], device="cuda", flags: int = 0,
                  page_ids: Sequence[int] | None = None, first_page: int = 0, target_ctas: int = 0,
-                 pools: tuple[torch.Tensor, torch.Tensor] | None = None):
+                 append_capacity: int = 0, pools: tuple[torch.Tensor, torch.Tensor] | None = None):
         self.dtype = dtype
         self.torch_dtype = {"f32": torch.float32, "bf16": torch.bfloat16}[dtype]
         self.num_q_heads, self.num_kv_heads, self.head_dim = num_q_heads, num_kv_heads, head_dim
         self.device = torch.device(device)
         self.problem = S.make_problem(batch, num_q_heads, num_kv_heads, head_dim, page_size, dtype, ctx_len,
-                                      q_start, policy, first_page, page_ids, target_ctas, flags)
+                                      q_start, policy, first_page, page_ids, target_ctas, flags, append_capacity)
         self.plan = S.segpaged_plan_create(self.problem)
         self.sizes = S.segpaged_plan_sizes(self.plan)
         z = self.sizes
@@ -83,6 +83,13 @@ class SegPagedLayer:
                              q.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None, scale,
                              self.workspace.data_ptr(), self.workspace.numel(), _stream(stream))
         return out, lse
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
+        """Ring plans: add one token per sequence (k_new, v_new: [B, Hkv, d])."""
+        assert k_new.stride() == v_new.stride() and k_new.stride(-1) == 1
+        S.segpaged_decode_append(self.plan, self.table.data_ptr(), k_new.data_ptr(), v_new.data_ptr(),
+                                 k_new.stride(0), k_new.stride(1), self.k_pool.data_ptr(), self.v_pool.data_ptr(),
+                                 self.workspace.data_ptr(), _stream(stream))
 
     def device_status(self, stream=None) -> int:
         return S.segpaged_read_device_status(self.workspace.data_ptr(), _stream(stream))

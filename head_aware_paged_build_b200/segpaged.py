@@ -21,6 +21,7 @@ SP_OK, SP_ERR_INVALID_ARG, SP_ERR_UNSUPPORTED, SP_ERR_WORKSPACE, SP_ERR_CUDA, SP
 SP_GLOBAL, SP_LOCAL, SP_DENSE, SP_RETRIEVAL = range(4)
 SP_F32, SP_BF16 = 0, 1
 SP_FLAG_DENSE_MASKED = 1
+SP_FLAG_RING = 2
 SP_VARLEN = -1
 KIND_CODES = {"global": SP_GLOBAL, "local": SP_LOCAL, "dense": SP_DENSE, "retrieval": SP_RETRIEVAL}
 DTYPE_CODES = {"f32": SP_F32, "bf16": SP_BF16}
@@ -29,7 +30,7 @@ DTYPE_CODES = {"f32": SP_F32, "bf16": SP_BF16}
 EXPORTED = ("segpaged_plan_create", "segpaged_plan_destroy", "segpaged_plan_sizes",
             "segpaged_plan_head_segments", "segpaged_plan_head_pages", "segpaged_table_write",
             "build_segpaged_cache", "segpaged_gather", "segpaged_attention",
-            "segpaged_attention_decode_noalloc", "segpaged_read_device_status", "segpaged_clear_device_status", "segpaged_status_string",
+            "segpaged_attention_decode_noalloc", "segpaged_decode_append", "segpaged_read_device_status", "segpaged_clear_device_status", "segpaged_status_string",
             "segpaged_last_error", "segpaged_abi_version")
 
 
@@ -49,7 +50,7 @@ class sp_problem(ctypes.Structure):
                 ("ctx_len", ctypes.POINTER(ctypes.c_int32)), ("q_start", ctypes.POINTER(ctypes.c_int32)),
                 ("policy", ctypes.POINTER(sp_head_policy)), ("first_page", ctypes.c_int64),
                 ("page_ids", ctypes.POINTER(ctypes.c_int32)), ("target_ctas", ctypes.c_int32),
-                ("flags", ctypes.c_uint32)]
+                ("flags", ctypes.c_uint32), ("append_capacity", ctypes.c_int32)]
 
 
 class sp_sizes(ctypes.Structure):
@@ -98,6 +99,7 @@ def load(path: Path | str | None = None) -> ctypes.CDLL:
         "segpaged_gather": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
         "segpaged_attention": ([vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp], i32),
         "segpaged_attention_decode_noalloc": ([vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp], i32),
+        "segpaged_decode_append": ([vp, vp, vp, vp, i64, i64, vp, vp, vp, vp], i32),
         "segpaged_read_device_status": ([vp, ctypes.POINTER(i32), vp], i32),
         "segpaged_clear_device_status": ([vp, vp], i32),
         "segpaged_status_string": ([i32], ctypes.c_char_p),
@@ -133,7 +135,7 @@ def _check(st: int, where: str) -> None:
 def make_problem(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, page_size: int, dtype: str,
                  ctx_len: Sequence[int], q_start: Sequence[int], policy: Sequence[tuple[str, int, int]],
                  first_page: int = 0, page_ids: Sequence[int] | None = None, target_ctas: int = 0,
-                 flags: int = 0):
+                 flags: int = 0, append_capacity: int = 0):
     """Build an ``sp_problem`` plus the host arrays it points to (kept alive in the result)."""
     B = batch
     ctx = (ctypes.c_int32 * B)(*ctx_len)
@@ -145,7 +147,7 @@ def make_problem(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
                       DTYPE_CODES[dtype] if isinstance(dtype, str) else dtype,
                       ctx, q0, pol, first_page,
                       ctypes.cast(ids, ctypes.POINTER(ctypes.c_int32)) if ids is not None else None,
-                      target_ctas, flags)
+                      target_ctas, flags, append_capacity)
     prob._keep = (ctx, q0, pol, ids)
     return prob
 
@@ -216,6 +218,13 @@ def segpaged_attention_decode_noalloc(plan: int, d_table: int, k_pool: int, v_po
     """Decode attention with the library's built-in scratch (no workspace argument, no allocation)."""
     _check(load().segpaged_attention_decode_noalloc(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale,
                                                     d_status, stream), "segpaged_attention_decode_noalloc")
+
+
+def segpaged_decode_append(plan: int, d_table: int, k_new: int, v_new: int, stride_seq: int, stride_head: int,
+                           k_pool: int, v_pool: int, workspace: int, stream: int = 0) -> None:
+    """Append one token per sequence to a ring plan's cache, in place (device table updated)."""
+    _check(load().segpaged_decode_append(plan, d_table, k_new, v_new, stride_seq, stride_head, k_pool, v_pool,
+                                         workspace, stream), "segpaged_decode_append")
 
 
 def segpaged_attention_status(*args) -> int:

@@ -71,11 +71,24 @@ enum {
    * the kernels visit every causal tile, masking LOCAL heads per element
    * ("SegPagedAttention runtime design", §4 verify_against_dense and §5: the
    * dense baseline the speedups are quoted against). */
-  SP_FLAG_DENSE_MASKED = 1u
+  SP_FLAG_DENSE_MASKED = 1u,
+  /* Ring plan (decode plans only): every page holds positions aligned to
+   * multiples of page_size; a LOCAL head's recent window lives in a ring of
+   * ceil(window / page_size) + 1 pages (position a in ring slot
+   * a mod (ring pages * page_size)), and GLOBAL heads reserve pages for
+   * append_capacity more tokens.  segpaged_decode_append then adds one token
+   * per sequence and evicts the token that leaves each LOCAL window, in
+   * place, with no new plan ("SegPagedAttention runtime design", §3: local
+   * occupancy independent of context length; "RedKnot overview (aipuzi)",
+   * §3.2: per-head pools that reclaim free pages). */
+  SP_FLAG_RING = 2u
 };
 
-/* Policy of one (sequence, kv-head).  `sink` >= 0 and `window` >= 1 are read
- * for SP_LOCAL only. */
+/* Policy of one (sequence, kv-head).  `sink` >= 0 and `window` are read for
+ * SP_LOCAL only.  window >= 1 is a fixed window; window <= -1 is an adaptive
+ * window of max(1, ctx_len / -window) tokens for that sequence ("RedKnot head
+ * classification", adaptive window: e.g. -2 gives ctx_len // 2).  window == 0
+ * is invalid. */
 typedef struct {
   int32_t kind;
   int32_t sink;
@@ -95,6 +108,9 @@ typedef struct {
  *               reported by segpaged_plan_sizes of a plan made with NULL
  *   target_ctas decode work is split into this many equal page ranges; 0 picks
  *               2 x 148 (two CTAs on each B200 SM)
+ *   append_capacity  SP_FLAG_RING plans: extra tokens per sequence that
+ *               segpaged_decode_append may add (GLOBAL heads reserve pages for
+ *               them); must be 0 otherwise
  */
 typedef struct {
   int32_t batch;
@@ -110,6 +126,7 @@ typedef struct {
   const int32_t* page_ids;
   int32_t target_ctas;
   uint32_t flags;
+  int32_t append_capacity; /* ring plans: tokens every sequence may still gain */
 } sp_problem;
 
 typedef struct {
@@ -235,6 +252,24 @@ SP_API sp_status segpaged_attention(const sp_plan* plan, const void* d_table, co
 SP_API sp_status segpaged_attention_decode_noalloc(const sp_plan* plan, const void* d_table, const void* k_pool,
                                                    const void* v_pool, const void* q, void* out, float* lse,
                                                    float softmax_scale, int32_t* d_status, void* stream);
+
+/* segpaged_decode_append: the next decode step of a ring plan (SP_FLAG_RING),
+ * in place.  For every sequence b, the token at position L_b (its current
+ * context length, as held by the device table) is written into the cache:
+ *   k_new, v_new  device [batch, num_kv_heads, head_dim]: element (b, kv, i) at
+ *                 base + b*stride_seq + kv*stride_head + i (16-byte aligned rows)
+ * and the device table d_table is updated: L_b grows by one, the new token
+ * joins its page, and the token at L_b - window leaves each LOCAL head's
+ * window (its page slot is released; a ring page whose tokens have all left
+ * is reused when the ring wraps onto it).  GLOBAL heads use the pages
+ * reserved by append_capacity; when none is left the append of that head is
+ * skipped and the device status word records the error.  Subsequent
+ * segpaged_attention calls on the same table see the longer context; the
+ * host plan (and segpaged_plan_sizes) keep describing the state at plan
+ * creation, and segpaged_table_write restores that state. */
+SP_API sp_status segpaged_decode_append(const sp_plan* plan, void* d_table, const void* k_new, const void* v_new,
+                                        int64_t stride_seq, int64_t stride_head, void* k_pool, void* v_pool,
+                                        void* workspace, void* stream);
 
 /* Device status word: kernels never trap; a failed device-side check or a
  * bounded wait that ran out records a non-zero code.  read synchronises

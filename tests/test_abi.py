@@ -158,6 +158,7 @@ BASE = dict(batch=1, num_q_heads=4, num_kv_heads=2, head_dim=64, page_size=16, d
     (dict(q_start=[100]), S.SP_ERR_INVALID_ARG),
     (dict(q_start=[-1]), S.SP_ERR_INVALID_ARG),
     (dict(policy=[("global", 0, 0), ("local", 4, 0)]), S.SP_ERR_INVALID_ARG),
+    (dict(policy=[("global", 0, 0), ("local", -1, -2)]), S.SP_ERR_INVALID_ARG),
     (dict(policy=[("global", 0, 0), ("local", -1, 8)]), S.SP_ERR_INVALID_ARG),
     (dict(policy=[("global", 0, 0), (7, 0, 8)]), S.SP_ERR_INVALID_ARG),
     (dict(policy=[("global", 0, 0), ("retrieval", 0, 0)]), S.SP_ERR_UNSUPPORTED),
@@ -212,4 +213,62 @@ def test_device_calls_reject_bad_arguments_before_launch():
     assert lib.build_segpaged_cache(plan, 256, 16, 16, -5, 0, 64, 16, 16, None) == S.SP_ERR_INVALID_ARG
     assert lib.build_segpaged_cache(plan, 256, 16, 16, 0, 0, 3, 16, 16, None) == S.SP_ERR_INVALID_ARG
     assert lib.segpaged_table_write(plan, 256, 8, None) == S.SP_ERR_WORKSPACE
+    S.segpaged_plan_destroy(plan)
+
+
+@pytest.mark.parametrize("div", [1, 2, 3, 7])
+def test_adaptive_window_resolves_per_sequence(div):
+    """window = -div selects max(1, L // div) per sequence (adaptive window of the head-classification page)."""
+    lens = [1, 5, 64, 100, 1000, 4097]
+    pol = []
+    for _ in lens:
+        pol += [("local", 4, -div), ("global", 0, 0)]
+    for mode in ("decode", "prefill"):
+        q0 = [L - 1 if mode == "decode" else max(0, L - 37) for L in lens]
+        p = S.make_problem(len(lens), 2, 2, 64, 16, "f32", lens, q0, pol)
+        plan = S.segpaged_plan_create(p)
+        for b, L in enumerate(lens):
+            segs = S.segpaged_plan_head_segments(plan, b, 0)
+            held = np.zeros(L, bool)
+            for start, length, _, _ in segs:
+                held[start:start + length] = True
+            want = oracle.stored_mask("local", 4, max(1, L // div), L, q0[b])
+            assert np.array_equal(held, want), (b, L, div)
+        S.segpaged_plan_destroy(plan)
+
+
+@pytest.mark.parametrize("page", [16, 64])
+def test_ring_plan_layout(page):
+    """Ring plans hold the same stored set; GLOBAL heads reserve pages, LOCAL heads a ring of ceil(w/P)+1 pages."""
+    rng = np.random.default_rng(page)
+    for _ in range(40):
+        L = int(rng.integers(1, 400))
+        s = int(rng.integers(0, 70))
+        w = int(rng.integers(1, 150))
+        cap = int(rng.integers(0, 200))
+        p = S.make_problem(1, 2, 2, 64, page, "f32", [L], [L - 1], [("local", s, w), ("global", 0, 0)],
+                           flags=S.SP_FLAG_RING, append_capacity=cap)
+        plan = S.segpaged_plan_create(p)
+        held = np.zeros(L, bool)
+        for start, length, _, _ in S.segpaged_plan_head_segments(plan, 0, 0):
+            held[start:start + length] = True
+        assert np.array_equal(held, oracle.stored_mask("local", s, w, L, L - 1))
+        assert len(S.segpaged_plan_head_pages(plan, 0, 0)) == -(-s // page) + (-(-w // page) + 1)
+        assert len(S.segpaged_plan_head_pages(plan, 0, 1)) == -(-(L + cap) // page)
+        assert S.segpaged_plan_sizes(plan).stored_token_heads == int(held.sum()) + L
+        S.segpaged_plan_destroy(plan)
+
+
+def test_ring_plan_validation():
+    base = dict(batch=1, num_q_heads=2, num_kv_heads=2, head_dim=64, page_size=16, dtype="f32", ctx_len=[100],
+                policy=[("local", 4, 8), ("global", 0, 0)])
+    for kw, code in ((dict(q_start=[90], flags=S.SP_FLAG_RING), S.SP_ERR_UNSUPPORTED),
+                     (dict(q_start=[99], flags=S.SP_FLAG_RING | S.SP_FLAG_DENSE_MASKED), S.SP_ERR_UNSUPPORTED),
+                     (dict(q_start=[99], append_capacity=5), S.SP_ERR_INVALID_ARG),
+                     (dict(q_start=[99], flags=S.SP_FLAG_RING, append_capacity=-1), S.SP_ERR_INVALID_ARG)):
+        st, _ = S.segpaged_plan_create_status(S.make_problem(**base, **kw))
+        assert st == code, (kw, S.last_error())
+    # appends need a ring plan (host-side check, no launch)
+    plan = S.segpaged_plan_create(S.make_problem(**base, q_start=[99]))
+    assert S.load().segpaged_decode_append(plan, 256, 16, 16, 0, 0, 16, 16, 256, None) == S.SP_ERR_INVALID_ARG
     S.segpaged_plan_destroy(plan)

@@ -129,3 +129,20 @@ def test_decode_mha_128k_full_size():
     torch.cuda.synchronize()
     assert layer.device_status() == 0
     assert_close(compare(prob, q, k, v, out, lse), "bf16")
+
+
+def test_decode_adaptive_window_matches_oracle():
+    """Adaptive windows (window = ctx_len // 2 and // 5) against the oracle with the resolved windows."""
+    lens = (300, 1000, 2500, 77)
+    pol = []
+    for _ in lens:
+        pol += [("local", 4, -2), ("global", 0, 0), ("local", 0, -5), ("local", 4, 100)]
+    wl = W.custom("adaptive", 51, len(lens), 16, 4, 128, "bf16", 64, lens, pol)
+    prob = wl.decode_problem()
+    _, (k, v, q), out, lse = run_decode(prob)
+    resolved = []
+    for b, L in enumerate(lens):
+        for kind, s, w in pol[4 * b: 4 * b + 4]:
+            resolved.append((kind, s, max(1, L // -w) if w < 0 else w))
+    ref = W.custom("adaptive", 51, len(lens), 16, 4, 128, "bf16", 64, lens, resolved)
+    assert_close(compare(ref.decode_problem(), q, k, v, out, lse), "bf16")

@@ -114,3 +114,19 @@ def test_prefill_bf16_matches_oracle_sampled_at_full_size(name, seqs, heads):
     rows = [sample_rows(c, stride=512, n_random=12, seed=b) if b in seqs else [] for b, c in enumerate(prob.q_counts)]
     res = compare(prob, q, k, v, out, lse, rows_per_seq=rows, heads=heads, seqs=seqs)
     assert_close(res, "bf16")
+
+
+def test_prefill_adaptive_window_matches_oracle():
+    lens = (300, 1000, 777)
+    pol = []
+    for _ in lens:
+        pol += [("local", 4, -2), ("global", 0, 0)]
+    wl = W.custom("adaptive_p", 52, len(lens), 4, 2, 128, "bf16", 64, lens, pol, chunk=200)
+    prob = wl.prefill_problem()
+    _, (k, v, q), out, lse = run_prefill(prob)
+    resolved = []
+    for b, L in enumerate(lens):
+        for kind, s, w in pol[2 * b: 2 * b + 2]:
+            resolved.append((kind, s, max(1, L // -w) if w < 0 else w))
+    ref = W.custom("adaptive_p", 52, len(lens), 4, 2, 128, "bf16", 64, lens, resolved, chunk=200)
+    assert_close(compare(ref.prefill_problem(), q, k, v, out, lse), "bf16")
