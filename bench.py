@@ -235,7 +235,9 @@ def run_ours(args) -> None:
     del Ldm, Lpm
 
     # ---- end to end through the public API with host buffers ----
-    e2e = run_e2e(args, dev, Ld, k, v, qd, od, lsed, world)
+    e2e_dense = run_e2e_dense(args, dev, Ld, k, v, qd, od, lsed, world)
+    e2e, append_us = run_e2e_serving(args, dev, wl, dec, k, v, world)
+    e2e["dense_upload_variant"] = e2e_dense
 
     zd, zp = Ld.sizes, Lp.sizes
     eb = 2
@@ -289,6 +291,7 @@ def run_ours(args) -> None:
                             "peak_source": f"{pk['source']} HBM copy",
                             "traffic": kernel_traffic("decode_bf16_kernel", csrc / "kernels_decode.cu")},
         "e2e": e2e,
+        "append": {"us": round(append_us, 2), "what": "segpaged_decode_append: one token per sequence, all heads"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "wall_s_timed": round(wall, 3),
@@ -300,8 +303,79 @@ def run_ours(args) -> None:
         dist.destroy_process_group()
 
 
-def run_e2e(args, dev, layer, k, v, qd, od, lsed, world) -> dict:
-    """Decode through the public API with the step's inputs copied from pinned host memory."""
+def run_e2e_serving(args, dev, wl, dec, k, v, world) -> tuple[dict, float]:
+    """Serving decode steps through the public API, cache resident on the GPU.
+
+    A ring plan of the decode layer is built once (untimed).  Every timed step
+    copies that step's inputs from pinned host memory (the new token's K and V
+    rows and its queries), appends the token (segpaged_decode_append),
+    runs decode attention and copies O and LSE back to the host.
+    """
+    import torch
+
+    from head_aware_paged_build_b200 import segpaged as S
+    from head_aware_paged_build_b200 import workloads as W
+    from head_aware_paged_build_b200.runtime import layer_for
+
+    n_steps = args.warmup + max(3, args.steps // 2)
+    start = W.Problem(wl, tuple(L - n_steps for L in dec.ctx_lens), tuple(L - n_steps - 1 for L in dec.ctx_lens))
+    layer = layer_for(start, device=dev, flags=S.SP_FLAG_RING, append_capacity=n_steps)
+    layer.build(k, v)
+    B, Hkv, Hq, d = wl.batch, wl.num_kv_heads, wl.num_q_heads, wl.head_dim
+    kin = torch.empty(n_steps, B, Hkv, d, dtype=k.dtype).pin_memory()
+    vin = torch.empty_like(kin).pin_memory()
+    qin = torch.empty(n_steps, B, Hq, d, dtype=k.dtype).pin_memory()
+    for i in range(n_steps):
+        pos = [L + i for L in start.ctx_lens]
+        kin[i] = torch.stack([k[b, :, p] for b, p in enumerate(pos)]).cpu()
+        vin[i] = torch.stack([v[b, :, p] for b, p in enumerate(pos)]).cpu()
+        qin[i] = W.queries(W.Problem(wl, tuple(p + 1 for p in pos), tuple(pos)), gen_device=dev).cpu()
+    kd, vd = torch.empty(B, Hkv, d, dtype=k.dtype, device=dev), torch.empty(B, Hkv, d, dtype=k.dtype, device=dev)
+    qdev = torch.empty(B, Hq, d, dtype=k.dtype, device=dev)
+    od = torch.empty_like(qdev)
+    lsed = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    lh = torch.empty(lsed.shape, dtype=torch.float32).pin_memory()
+    s = torch.cuda.current_stream()
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    times, app = [], []
+    for i in range(n_steps):
+        e0.record(s)
+        kd.copy_(kin[i], non_blocking=True)
+        vd.copy_(vin[i], non_blocking=True)
+        qdev.copy_(qin[i], non_blocking=True)
+        e2.record(s)
+        layer.append(kd, vd)
+        layer.attention(qdev, od, lsed)
+        oh.copy_(od, non_blocking=True)
+        lh.copy_(lsed, non_blocking=True)
+        e1.record(s)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    # the append alone, on a second ring plan with its own capacity
+    probe = layer_for(start, device=dev, flags=S.SP_FLAG_RING, append_capacity=64)
+    probe.build(k, v)
+    for i in range(8):
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ea.record(s)
+        probe.append(kd, vd)
+        eb.record(s)
+        torch.cuda.synchronize()
+        app.append(ea.elapsed_time(eb) * 1e3)
+    assert layer.device_status() == 0 and probe.device_status() == 0
+    ms = reduce_max([statistics.median(times)], world, dev)[0]
+    vis = layer.sizes.stored_token_heads * 2 * d * k.element_size()
+    h2d = (kin[0].numel() + vin[0].numel() + qin[0].numel()) * kin.element_size()
+    d2h = oh.numel() * oh.element_size() + lh.numel() * 4
+    return ({"value": round(weak_rate(vis, world, ms) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 4),
+             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+             "path": "pinned host q, k_new, v_new -> segpaged_decode_append -> segpaged_attention (decode, "
+                     "cache resident) -> host O, LSE"}, statistics.median(app))
+
+
+def run_e2e_dense(args, dev, layer, k, v, qd, od, lsed, world) -> dict:
+    """Decode with the whole dense K/V uploaded from pinned host memory and packed every step."""
     import torch
     kh, vh, qh = (t.cpu().pin_memory() for t in (k, v, qd))
     oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()

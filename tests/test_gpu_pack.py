@@ -108,3 +108,28 @@ def test_pack_varlen_layout_matches_padded():
             m = torch.from_numpy(oracle.stored_mask(kind, s, w, L, L - 1)).cuda()
             assert torch.equal(ko[off:off + L, kv][m], kvar[off:off + L, kv][m])
             assert torch.equal(vo[off:off + L, kv][m], vvar[off:off + L, kv][m])
+
+
+def test_two_layers_share_one_pool_through_first_page():
+    """Layers of a model keep their pages in one pool: layer 1 starts at layer 0's pool_pages."""
+    l0 = W.llama(layer=0, batch=1)
+    l1 = W.llama(layer=1, batch=1)
+    p0, p1 = l0.decode_problem(), l1.decode_problem()
+    a = layer_for(p0)
+    n0 = a.sizes.pool_pages
+    b = layer_for(p1, first_page=n0)
+    pool_bytes = b.sizes.pool_pages * b.sizes.page_bytes
+    kpool = torch.empty(pool_bytes, dtype=torch.uint8, device="cuda")
+    vpool = torch.empty(pool_bytes, dtype=torch.uint8, device="cuda")
+    a = layer_for(p0, pools=(kpool, vpool))
+    b = layer_for(p1, first_page=n0, pools=(kpool, vpool))
+    from _parity import assert_close, compare
+    inputs = []
+    for lay, prob in ((a, p0), (b, p1)):
+        k, v = W.dense_kv(prob, device="cuda")
+        lay.build(k, v)
+        inputs.append((k, v, W.queries(prob, device="cuda")))
+    for lay, prob, (k, v, q) in ((a, p0, inputs[0]), (b, p1, inputs[1])):
+        out, lse = lay.attention(q)
+        torch.cuda.synchronize()
+        assert_close(compare(prob, q, k, v, out, lse), "bf16")
