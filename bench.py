@@ -130,16 +130,32 @@ def weak_rate(units_per_rank: float, world: int, max_ms: float) -> float:
     return world * units_per_rank / (max_ms * 1e-3)
 
 
-def kernel_traffic(kernel: str, source: Path) -> int | None:
-    """DRAM bytes per launch from the last ncu capture, if the kernel source is unchanged since."""
+def kernel_traffic(kernel: str, source: Path, workload_name: str) -> int | None:
+    """DRAM bytes per launch from the last ncu capture of this workload, if the kernel source is unchanged since."""
     p = ROOT / "profiles" / "traffic.json"
     if not p.exists():
         return None
     rec = json.loads(p.read_text()).get(kernel)
-    if not rec:
+    if not rec or rec.get("workload_key") != workload_name:
         return None
     sha = hashlib.sha256(source.read_bytes()).hexdigest()[:16]
     return int(rec["bytes_per_launch"]) if rec.get("source_sha16") == sha else None
+
+
+def median_ms(fn, flush, n: int) -> float:
+    """Median CUDA-event time of fn() over n runs, L2 flushed before each (after one untimed run)."""
+    import torch
+    fn()
+    vals = []
+    for _ in range(n):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        vals.append(e0.elapsed_time(e1))
+    return statistics.median(vals)
 
 
 def run_ours(args) -> None:
@@ -218,21 +234,21 @@ def run_ours(args) -> None:
     Lpm = layer_for(pre, device=dev, flags=S.SP_FLAG_DENSE_MASKED)
     Ldm.build(k, v)
     Lpm.build(k, v)
-    dm = {}
-    for nm, fn in (("decode", lambda: Ldm.attention(qd, od, lsed)), ("prefill", lambda: Lpm.attention(qp, op, lsep))):
-        fn()
-        vals = []
-        for _ in range(3 if nm == "prefill" else 10):
-            flush()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            vals.append(e0.elapsed_time(e1))
-        dm[nm] = statistics.median(vals)
+    dm = {"decode": median_ms(lambda: Ldm.attention(qd, od, lsed), flush, 10),
+          "prefill": median_ms(lambda: Lpm.attention(qp, op, lsep), flush, 3)}
     dm = dict(zip(("decode", "prefill"), reduce_max([dm["decode"], dm["prefill"]], world, dev)))
     del Ldm, Lpm
+
+    # ---- E4M3 pages: the same decode on 1-byte pages (per-tensor scales amax / 448) ----
+    k_scale = float(k.abs().max()) / 448.0
+    v_scale = float(v.abs().max()) / 448.0
+    Ld8 = layer_for(dec, device=dev, kv_dtype="e4m3", k_scale=k_scale, v_scale=v_scale)
+    Ld8.build(k, v)
+    fp8_ms = median_ms(lambda: Ld8.attention(qd, od, lsed), flush, 10)
+    fp8_pack_ms = median_ms(lambda: Ld8.build(k, v), flush, 5)
+    assert Ld8.device_status() == 0, "device status word set by the E4M3 decode"
+    fp8_ms, fp8_pack_ms = reduce_max([fp8_ms, fp8_pack_ms], world, dev)
+    del Ld8
 
     # ---- end to end through the public API with host buffers ----
     e2e_dense = run_e2e_dense(args, dev, Ld, k, v, qd, od, lsed, world)
@@ -284,12 +300,17 @@ def run_ours(args) -> None:
         "roofline": {"kernel": "prefill_tc_kernel", "bound": "tensor", "achieved": round(per_launch_pre, 1),
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(per_launch_pre / pk["bf16_tflops"], 4),
                      "peak_source": f"{pk['source']} bf16 burst",
-                     "traffic": kernel_traffic("prefill_tc_kernel", csrc / "kernels_prefill_tc.cu")},
+                     "traffic": kernel_traffic("prefill_tc_kernel", csrc / "kernels_prefill_tc.cu", wl.name)},
         "roofline_decode": {"kernel": "decode_bf16_kernel", "bound": "hbm",
                             "achieved": round(vis_dec / (ms["decode"] * 1e-3) / 1e9, 1), "peak": pk["hbm_gbs"],
                             "unit": "GB/s", "frac": round(vis_dec / (ms["decode"] * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                             "peak_source": f"{pk['source']} HBM copy",
-                            "traffic": kernel_traffic("decode_bf16_kernel", csrc / "kernels_decode.cu")},
+                            "traffic": kernel_traffic("decode_bf16_kernel", csrc / "kernels_decode.cu", wl.name)},
+        "decode_e4m3": {"ms": round(fp8_ms, 5), "visible_kv_bytes": vis_dec // eb,
+                        "GB/s": round(weak_rate(vis_dec // eb, world, fp8_ms) / 1e9, 1),
+                        "frac_hbm": round(vis_dec // eb / (fp8_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                        "speedup_vs_bf16": round(ms["decode"] / fp8_ms, 3), "pack_ms": round(fp8_pack_ms, 5),
+                        "what": "decode on FP8 E4M3 pages (1 byte per element), bf16 queries and output"},
         "e2e": e2e,
         "append": {"us": round(append_us, 2), "what": "segpaged_decode_append: one token per sequence, all heads"},
         "gpu_launches": launches_per_step * args.steps,

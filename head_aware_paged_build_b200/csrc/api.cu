@@ -41,7 +41,8 @@ sp_status pack_common(const sp_plan* plan, const void* d_table, const void* k_in
   if (!k_in || !v_in || !k_out || !v_out) return fail(SP_ERR_INVALID_ARG, "K/V pointers must be non-NULL");
   if (!aligned(k_in, 16) || !aligned(v_in, 16) || !aligned(k_out, 16) || !aligned(v_out, 16))
     return fail(SP_ERR_INVALID_ARG, "K/V pointers must be 16-byte aligned");
-  const int64_t eb = plan->elem_bytes;
+  // dense element size: the problem dtype, except the 1-byte codes a gather of E4M3 pages writes
+  const int64_t eb = (inverse && plan->fp8) ? 1 : plan->elem_bytes;
   if (stride_head < 0 || stride_tok < 0 || (stride_seq < 0 && stride_seq != SP_VARLEN))
     return fail(SP_ERR_INVALID_ARG, "strides must be >= 0 (stride_seq may be SP_VARLEN)");
   if ((stride_head * eb) % 16 || (stride_tok * eb) % 16 || (stride_seq > 0 && (stride_seq * eb) % 16))
@@ -53,6 +54,9 @@ sp_status pack_common(const sp_plan* plan, const void* d_table, const void* k_in
   L.D = plan->prob.head_dim;
   L.P = plan->prob.page_size;
   L.bf16 = plan->prob.dtype == SP_BF16;
+  L.fp8 = plan->fp8;
+  L.k_inv = 1.0f / plan->k_scale;
+  L.v_inv = 1.0f / plan->v_scale;
   L.inverse = inverse;
   L.stride_seq = stride_seq;
   L.stride_head = stride_head;
@@ -132,7 +136,9 @@ sp_status segpaged_attention(const sp_plan* plan, const void* d_table, const voi
     L.bf16 = plan->prob.dtype == SP_BF16;
     L.page_bytes = plan->sizes.page_bytes;
     L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
-    L.scale_log2 = scale_log2;
+    L.scale_log2 = plan->fp8 ? scale_log2 * plan->k_scale : scale_log2;
+    L.fp8 = plan->fp8;
+    L.v_scale = plan->fp8 ? plan->v_scale : 1.f;
     L.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + plan->partial_offset);
     L.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
     L.status = status;
@@ -181,6 +187,9 @@ sp_status segpaged_decode_append(const sp_plan* plan, void* d_table, const void*
   L.D = plan->prob.head_dim;
   L.P = plan->prob.page_size;
   L.bf16 = plan->prob.dtype == SP_BF16;
+  L.fp8 = plan->fp8;
+  L.k_inv = 1.0f / plan->k_scale;
+  L.v_inv = 1.0f / plan->v_scale;
   L.stride_seq = stride_seq;
   L.stride_head = stride_head;
   L.page_bytes = plan->sizes.page_bytes;

@@ -30,6 +30,28 @@ __host__ __device__ __forceinline__ int64_t vpage_chunk_offset_bf16(int i, int c
   // row i (dimension), chunk c16 holds tokens 8*c16 .. 8*c16+7 (P = 64)
   return int64_t(i) * 128 + ((c16 ^ (i & 7)) << 4);
 }
+// E4M3 pages (P = 64): K page [64 tokens][D] codes, V page [D][64 positions]
+// codes; byte (row, col) of a page with `pitch`-byte rows lives at its linear
+// address with the 16-byte chunks of each 128-byte line XOR-swizzled by the
+// line index.  A warp reading 8 consecutive rows at one column then hits 8
+// distinct chunks (no bank conflicts) for pitch 64 and 128.
+__host__ __device__ __forceinline__ int fp8_page_offset(int row, int col, int pitch) {
+  const int a = row * pitch + col;
+  const int line = a >> 7;
+  return (line << 7) | ((((a >> 4) & 7) ^ (line & 7)) << 4) | (a & 15);
+}
+// Position of token u (0 .. 63) inside a V row of an E4M3 page.  Within each
+// group of 16 tokens, tokens 2i, 2i+1, 8+2i, 9+2i sit at positions 4i .. 4i+3:
+// exactly the four values one lane's mma.sync B fragment (two f16x2
+// registers) needs, so one 32-bit load feeds both registers.
+__host__ __device__ __forceinline__ int fp8_vtok_pos(int u) {
+  const int w = u & 15;
+  return (u & ~15) + ((w & 7) >> 1) * 4 + ((w >> 3) << 1) + (w & 1);
+}
+__host__ __device__ __forceinline__ int fp8_vpos_tok(int p) {  // inverse of fp8_vtok_pos
+  const int w = p & 15;
+  return (p & ~15) + ((w >> 1) & 1) * 8 + (w >> 2) * 2 + (w & 1);
+}
 
 // --------------------------------------------------------------------------
 // Status word (workspace word 0).  The first error sticks.
@@ -126,9 +148,41 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two fp32 values to two FP8 E4M3 codes (round to nearest even, saturating);
+// `lo` lands in the low byte.
+__device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Two E4M3 codes (low byte first) to two fp16 values (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(codes));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(x & 0xffff0000u)), "f"(__uint_as_float(x << 16)));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
 

@@ -13,6 +13,8 @@ struct PackLaunch {
   int32_t n_pages;
   int32_t D, P;
   bool bf16;
+  bool fp8;      // E4M3 pages (dense side bf16 for pack, 1-byte codes for gather)
+  float k_inv, v_inv;  // quantisation multipliers 1 / scale (fp8 pack)
   bool inverse;  // gather (pool -> dense) instead of pack
   int64_t stride_seq, stride_head, stride_tok, page_bytes;
   const void* kdense_in;
@@ -41,7 +43,9 @@ struct DecodeLaunch {
   const void* q;  // [B, Hq, D]
   void* out;      // [B, Hq, D]
   float* lse;     // [B, Hq] or null
-  float scale_log2;  // softmax scale * log2(e)
+  float scale_log2;  // softmax scale * log2(e) (* k_scale for E4M3 pages)
+  bool fp8;          // E4M3 pages
+  float v_scale;     // E4M3 pages: value scale, applied to the normalised output
   float* partial;    // workspace partial slots
   int32_t* counters; // workspace arrival counters of split heads (zero between calls)
   int32_t* status;
@@ -72,6 +76,8 @@ struct AppendLaunch {
   int32_t n_heads;
   int32_t D, P;
   bool bf16;
+  bool fp8;            // E4M3 pages: the new bf16 rows are quantised on the way in
+  float k_inv, v_inv;  // 1 / k_scale, 1 / v_scale
   int64_t stride_seq, stride_head, page_bytes;
   const void* k_new;  // [B, Hkv, D] with the given strides (elements)
   const void* v_new;

@@ -12,7 +12,8 @@
 // the token at L - window leaves a LOCAL head's window (its page's range
 // shrinks from below: eviction), and the head's context grows by one.  No
 // token ever moves ("SegPagedAttention runtime design", §3: a local head's
-// occupancy does not depend on the context length).
+// occupancy does not depend on the context length).  E4M3 pages receive the
+// codes of the new bf16 row, quantised as the pack does.
 #include "device_common.cuh"
 #include "kernels.h"
 
@@ -21,7 +22,7 @@ namespace {
 
 constexpr int kAppendThreads = 128;
 
-template <typename T, int D, int P>
+template <typename T, int D, int P, bool FP8 = false>
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendLaunch a) {
   HeadDesc* hd = a.heads + blockIdx.x;
   const int L = hd->ctx_len;
@@ -46,6 +47,25 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendLaunch a) 
   uint8_t* kdst = static_cast<uint8_t*>(a.kpool) + phys * a.page_bytes;
   uint8_t* vdst = static_cast<uint8_t*>(a.vpool) + phys * a.page_bytes;
   constexpr int CR = D * int(sizeof(T)) / 16;
+  if constexpr (FP8) {
+    for (int c = threadIdx.x; c < CR; c += kAppendThreads) {  // 8 values -> 8 codes
+      const uint4 v = reinterpret_cast<const uint4*>(kn)[c];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t q[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float x0 = __uint_as_float(w[2 * h] << 16) * a.k_inv, x1 = __uint_as_float(w[2 * h] & 0xffff0000u) * a.k_inv;
+        const float x2 = __uint_as_float(w[2 * h + 1] << 16) * a.k_inv,
+                    x3 = __uint_as_float(w[2 * h + 1] & 0xffff0000u) * a.k_inv;
+        q[h] = uint32_t(pack_e4m3x2(x0, x1)) | (uint32_t(pack_e4m3x2(x2, x3)) << 16);
+      }
+      *reinterpret_cast<uint2*>(kdst + fp8_page_offset(slot, c * 8, D)) = make_uint2(q[0], q[1]);
+    }
+    for (int i = threadIdx.x; i < D; i += kAppendThreads) {
+      const float x = __bfloat162float(vn[i]) * a.v_inv;
+      vdst[fp8_page_offset(i, fp8_vtok_pos(slot), P)] = uint8_t(pack_e4m3x2(x, 0.f));
+    }
+  } else {
   for (int c = threadIdx.x; c < CR; c += kAppendThreads) {
     const uint4 v = reinterpret_cast<const uint4*>(kn)[c];
     if constexpr (sizeof(T) == 2)
@@ -61,6 +81,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendLaunch a) 
     else
       off = (int64_t(i) * P + slot) * 4;
     *reinterpret_cast<T*>(vdst + off) = vn[i];
+  }
   }
   if (threadIdx.x != 0) return;
   // the target page: a new run starts when the page held other positions
@@ -91,7 +112,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendLaunch a) 
 
 cudaError_t launch_append(const AppendLaunch& a, cudaStream_t s) {
   if (a.n_heads == 0) return cudaSuccess;
-  if (a.bf16) {
+  if (a.fp8) {
+    if (a.D == 128) append_kernel<__nv_bfloat16, 128, 64, true><<<a.n_heads, kAppendThreads, 0, s>>>(a);
+    else append_kernel<__nv_bfloat16, 64, 64, true><<<a.n_heads, kAppendThreads, 0, s>>>(a);
+  } else if (a.bf16) {
     if (a.D == 128) append_kernel<__nv_bfloat16, 128, 64><<<a.n_heads, kAppendThreads, 0, s>>>(a);
     else append_kernel<__nv_bfloat16, 64, 64><<<a.n_heads, kAppendThreads, 0, s>>>(a);
   } else if (a.P == 16) {

@@ -14,6 +14,15 @@
 // across CTAs is finished by whichever of its CTAs publishes its partial last
 // (an arrival counter in the workspace): it merges the partials in slot order.
 //
+// E4M3 pages: the same kernel with 1-byte pages.  Each lane loads the codes
+// of its mma.sync B fragments straight from the staged page (one 64-bit load
+// per K fragment pair, one 32-bit load per V fragment: the page layout puts
+// them side by side) and widens them exactly to f16; Q and P enter the
+// tensor cores as f16, so the MMAs run kind f16 with f32 accumulation.  For
+// K the head dimension is visited in a permuted order (Q loaded to match),
+// which leaves the dot products unchanged.  k_scale is folded into the
+// softmax scale and v_scale into the output normalisation.
+//
 // fp32: a plain SIMT kernel over the same work list (FP32 FMA only), with a
 // separate combine pass for split heads.
 #include <cmath>
@@ -28,9 +37,9 @@ constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
 
-template <int D, int NST>
+template <int D, int NST, bool FP8>
 struct DecodeSmem {
-  static constexpr int kPageBytes = 64 * D * 2;
+  static constexpr int kPageBytes = 64 * D * (FP8 ? 1 : 2);
   static constexpr int kMergePitch = D + 8;  // floats per merge row (breaks bank aliasing)
   static constexpr int kStageOff = 0;
   static constexpr int kMergeOff = NST * 2 * kPageBytes;
@@ -39,9 +48,9 @@ struct DecodeSmem {
   static constexpr int kBytes = kBarOff + 2 * NST * 8;
 };
 
-template <int D, int NST>
+template <int D, int NST, bool FP8>
 __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunch a) {
-  using S = DecodeSmem<D, NST>;
+  using S = DecodeSmem<D, NST, FP8>;
   constexpr int P = 64;
   constexpr int PB = S::kPageBytes;
   constexpr int KSTEPS = D / 16;
@@ -112,13 +121,28 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
     const int qh0 = hd.kv * G;
     const __nv_bfloat16* qrow = qg + (int64_t(hd.q_row0) * a.num_q_heads + qh0) * D;
     uint32_t qa[KSTEPS][4];
+    if constexpr (FP8) {
+      // k-steps 2j, 2j+1 cover dims 32j .. 32j+31; lane tq owns dims 32j+8tq .. +7
+      // (pairs {0,1},{2,3} -> k-step 2j, {4,5},{6,7} -> k-step 2j+1), matching the K loads.
 #pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk) {
-      const int c0 = kk * 16 + tq * 2;
-      qa[kk][0] = r0 < G ? *reinterpret_cast<const uint32_t*>(qrow + r0 * D + c0) : 0u;
-      qa[kk][1] = r1 < G ? *reinterpret_cast<const uint32_t*>(qrow + r1 * D + c0) : 0u;
-      qa[kk][2] = r0 < G ? *reinterpret_cast<const uint32_t*>(qrow + r0 * D + c0 + 8) : 0u;
-      qa[kk][3] = r1 < G ? *reinterpret_cast<const uint32_t*>(qrow + r1 * D + c0 + 8) : 0u;
+      for (int j = 0; j < D / 32; ++j) {
+        const int c0 = j * 32 + tq * 8;
+        const uint4 x0 = r0 < G ? *reinterpret_cast<const uint4*>(qrow + r0 * D + c0) : make_uint4(0, 0, 0, 0);
+        const uint4 x1 = r1 < G ? *reinterpret_cast<const uint4*>(qrow + r1 * D + c0) : make_uint4(0, 0, 0, 0);
+        qa[2 * j][0] = bf16x2_to_f16x2(x0.x), qa[2 * j][2] = bf16x2_to_f16x2(x0.y);
+        qa[2 * j + 1][0] = bf16x2_to_f16x2(x0.z), qa[2 * j + 1][2] = bf16x2_to_f16x2(x0.w);
+        qa[2 * j][1] = bf16x2_to_f16x2(x1.x), qa[2 * j][3] = bf16x2_to_f16x2(x1.y);
+        qa[2 * j + 1][1] = bf16x2_to_f16x2(x1.z), qa[2 * j + 1][3] = bf16x2_to_f16x2(x1.w);
+      }
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        const int c0 = kk * 16 + tq * 2;
+        qa[kk][0] = r0 < G ? *reinterpret_cast<const uint32_t*>(qrow + r0 * D + c0) : 0u;
+        qa[kk][1] = r1 < G ? *reinterpret_cast<const uint32_t*>(qrow + r1 * D + c0) : 0u;
+        qa[kk][2] = r0 < G ? *reinterpret_cast<const uint32_t*>(qrow + r0 * D + c0 + 8) : 0u;
+        qa[kk][3] = r1 < G ? *reinterpret_cast<const uint32_t*>(qrow + r1 * D + c0 + 8) : 0u;
+      }
     }
     float o[NT][4];
 #pragma unroll
@@ -143,13 +167,27 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
         // S = Q K^T over this warp's 16 tokens (two n8 tiles)
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         const int mi = lane >> 3, rr = lane & 7;
-        const int ktok = tok0 + (mi >> 1) * 8 + rr;
+        if constexpr (FP8) {
+          const uint8_t* kp8 = stage + s * 2 * PB;
 #pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4(b0, b1, b2, b3, kst + uint32_t(kpage_chunk_offset_bf16(ktok, 2 * kk + (mi & 1), P)));
-          mma_bf16_16816(sc[0], qa[kk], b0, b1);
-          mma_bf16_16816(sc[1], qa[kk], b2, b3);
+          for (int j = 0; j < D / 32; ++j)
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+              const uint2 u =
+                  *reinterpret_cast<const uint2*>(kp8 + fp8_page_offset(tok0 + n * 8 + grp, j * 32 + tq * 8, D));
+              mma_f16_16816(sc[n], qa[2 * j], e4m3x2_to_f16x2(uint16_t(u.x)), e4m3x2_to_f16x2(uint16_t(u.x >> 16)));
+              mma_f16_16816(sc[n], qa[2 * j + 1], e4m3x2_to_f16x2(uint16_t(u.y)),
+                            e4m3x2_to_f16x2(uint16_t(u.y >> 16)));
+            }
+        } else {
+          const int ktok = tok0 + (mi >> 1) * 8 + rr;
+#pragma unroll
+          for (int kk = 0; kk < KSTEPS; ++kk) {
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(b0, b1, b2, b3, kst + uint32_t(kpage_chunk_offset_bf16(ktok, 2 * kk + (mi & 1), P)));
+            mma_bf16_16816(sc[0], qa[kk], b0, b1);
+            mma_bf16_16816(sc[1], qa[kk], b2, b3);
+          }
         }
         // mask and scale (log2 domain)
 #pragma unroll
@@ -182,6 +220,21 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
         l0 = l0 * al0 + ((p[0][0] + p[0][1]) + (p[1][0] + p[1][1]));
         l1 = l1 * al1 + ((p[0][2] + p[0][3]) + (p[1][2] + p[1][3]));
         uint32_t pa[4];
+        if constexpr (FP8) {
+          pa[0] = pack_f16x2(p[0][0], p[0][1]);
+          pa[1] = pack_f16x2(p[0][2], p[0][3]);
+          pa[2] = pack_f16x2(p[1][0], p[1][1]);
+          pa[3] = pack_f16x2(p[1][2], p[1][3]);
+          // O = alpha O + P V: lane (grp, tq) needs V rows d = 8 j + grp at this
+          // warp's tokens 2tq, 2tq+1, 8+2tq, 9+2tq: positions 4tq .. 4tq+3
+          const uint8_t* vp8 = stage + s * 2 * PB + PB;
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            const uint32_t u = *reinterpret_cast<const uint32_t*>(vp8 + fp8_page_offset(j * 8 + grp, tok0 + tq * 4, P));
+            o[j][0] *= al0, o[j][1] *= al0, o[j][2] *= al1, o[j][3] *= al1;
+            mma_f16_16816(o[j], pa, e4m3x2_to_f16x2(uint16_t(u)), e4m3x2_to_f16x2(uint16_t(u >> 16)));
+          }
+        } else {
         pa[0] = pack_bf16x2(p[0][0], p[0][1]);
         pa[1] = pack_bf16x2(p[0][2], p[0][3]);
         pa[2] = pack_bf16x2(p[1][0], p[1][1]);
@@ -197,6 +250,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
           o[2 * j + 1][0] *= al0, o[2 * j + 1][1] *= al0, o[2 * j + 1][2] *= al1, o[2 * j + 1][3] *= al1;
           mma_bf16_16816(o[2 * j], pa, b0, b1);
           mma_bf16_16816(o[2 * j + 1], pa, b2, b3);
+        }
         }
       }
       __syncwarp();
@@ -237,7 +291,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
       }
       if (item.slot < 0) {
         const int64_t o_idx = (int64_t(hd.q_row0) * a.num_q_heads + qh0 + row) * D + col;
-        static_cast<__nv_bfloat16*>(a.out)[o_idx] = __float2bfloat16_rn(acc / L);
+        if constexpr (FP8)
+          static_cast<__nv_bfloat16*>(a.out)[o_idx] = __float2bfloat16_rn(acc * a.v_scale / L);
+        else
+          static_cast<__nv_bfloat16*>(a.out)[o_idx] = __float2bfloat16_rn(acc / L);
         if (col == 0 && a.lse) a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + row] = (M + log2f(L)) * kLn2;
       } else {
         float* slot = a.partial + int64_t(item.slot) * partial_slot_floats(G, D);
@@ -289,7 +346,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
             const float4 v = __ldcg(reinterpret_cast<const float4*>(sl + row * D + col));
             acc.x += f * v.x, acc.y += f * v.y, acc.z += f * v.z, acc.w += f * v.w;
           }
-          const float inv = 1.f / row_l[row];
+          const float inv = (FP8 ? a.v_scale : 1.f) / row_l[row];
           __nv_bfloat16* o =
               static_cast<__nv_bfloat16*>(a.out) + (int64_t(hd.q_row0) * a.num_q_heads + qh0 + row) * D + col;
           reinterpret_cast<uint2*>(o)[0] = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv),
@@ -445,11 +502,13 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeLaunch a) {
 }
 
 constexpr int kStagesBf16 = 2;
+constexpr int kStagesFp8 = 4;  // half-size pages: twice the stages for the same bytes in flight
 
-template <int D>
+template <int D, bool FP8>
 cudaError_t launch_bf16(const DecodeLaunch& a, cudaStream_t s) {
-  using Sm = DecodeSmem<D, kStagesBf16>;
-  auto kern = decode_bf16_kernel<D, kStagesBf16>;
+  constexpr int NST = FP8 ? kStagesFp8 : kStagesBf16;
+  using Sm = DecodeSmem<D, NST, FP8>;
+  auto kern = decode_bf16_kernel<D, NST, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kBytes);
   if (e != cudaSuccess) return e;
   kern<<<a.n_ctas, kDecodeThreads, Sm::kBytes, s>>>(a);  // split heads are merged in-kernel
@@ -473,7 +532,8 @@ cudaError_t launch_f32(const DecodeLaunch& a, cudaStream_t s) {
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s) {
   if (a.n_ctas == 0) return cudaSuccess;
-  if (a.bf16) return a.D == 128 ? launch_bf16<128>(a, s) : launch_bf16<64>(a, s);
+  if (a.fp8) return a.D == 128 ? launch_bf16<128, true>(a, s) : launch_bf16<64, true>(a, s);
+  if (a.bf16) return a.D == 128 ? launch_bf16<128, false>(a, s) : launch_bf16<64, false>(a, s);
   if (a.P == 16) return a.D == 128 ? launch_f32<128, 16>(a, s) : launch_f32<64, 16>(a, s);
   return a.D == 128 ? launch_f32<128, 64>(a, s) : launch_f32<64, 64>(a, s);
 }

@@ -124,6 +124,115 @@ __global__ void __launch_bounds__(kPackThreads) gather_kernel(PackArgs a, const 
   }
 }
 
+// ---------------------------------------------------------------------------
+// E4M3 pages (page size 64): K page [64 tokens][D] codes, V page [D][64
+// positions] codes, both at fp8_page_offset(); V positions order the tokens
+// as fp8_vtok_pos() says.  Dense side: bf16 for pack, 1-byte codes for gather.
+// Codes are E4M3(fp32(x) * (1 / scale)), nearest-even, saturating.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+
+__device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float inv) {
+  // four bf16 values (two words, low half first) -> four codes, first value in the low byte
+  const uint16_t c0 = pack_e4m3x2(bf16_bits_to_float(w0 & 0xffff) * inv, bf16_bits_to_float(w0 >> 16) * inv);
+  const uint16_t c1 = pack_e4m3x2(bf16_bits_to_float(w1 & 0xffff) * inv, bf16_bits_to_float(w1 >> 16) * inv);
+  return uint32_t(c0) | (uint32_t(c1) << 16);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPackThreads) pack_fp8_kernel(PackArgs a, float k_inv, float v_inv,
+                                                                const __nv_bfloat16* __restrict__ kd,
+                                                                const __nv_bfloat16* __restrict__ vd,
+                                                                uint8_t* __restrict__ kpool,
+                                                                uint8_t* __restrict__ vpool) {
+  constexpr int P = 64;
+  constexpr int CR = D * 2 / 16;                            // 16-byte bf16 chunks per dense row
+  constexpr int PW = vstage_pitch_words<__nv_bfloat16>(D);  // staging pitch (32-bit words)
+  __shared__ uint32_t stage[P * PW];
+  const PageDesc pg = a.pages[blockIdx.x];
+  const HeadDesc hd = a.heads[pg.head];
+  const int64_t base = (a.stride_seq >= 0 ? int64_t(hd.b) * a.stride_seq : int64_t(hd.ctx_row0) * a.stride_tok) +
+                       int64_t(hd.kv) * a.stride_head;
+  uint8_t* kdst = kpool + int64_t(pg.phys) * a.page_bytes;
+  uint8_t* vdst = vpool + int64_t(pg.phys) * a.page_bytes;
+  for (int idx = threadIdx.x; idx < P * CR; idx += kPackThreads) {
+    const int t = idx / CR, c = idx % CR;
+    uint4 kv4 = make_uint4(0, 0, 0, 0), vv4 = make_uint4(0, 0, 0, 0);
+    if (t >= slot_lo(pg) && t < slot_hi(pg)) {
+      const int64_t row = base + int64_t(pg.abs_start + t) * a.stride_tok;
+      kv4 = __ldg(reinterpret_cast<const uint4*>(kd + row) + c);
+      vv4 = __ldg(reinterpret_cast<const uint4*>(vd + row) + c);
+    }
+    *reinterpret_cast<uint2*>(kdst + fp8_page_offset(t, c * 8, D)) =
+        make_uint2(quant4(kv4.x, kv4.y, k_inv), quant4(kv4.z, kv4.w, k_inv));
+    uint32_t* st = stage + t * PW + c * 4;
+    st[0] = vv4.x, st[1] = vv4.y, st[2] = vv4.z, st[3] = vv4.w;
+  }
+  __syncthreads();
+  const uint16_t* sv = reinterpret_cast<const uint16_t*>(stage);  // [token][dim] bf16, pitch 2 PW
+  for (int idx = threadIdx.x; idx < D * 4; idx += kPackThreads) {
+    const int i = idx / 4, c = idx % 4;  // row i (dimension), positions 16 c .. 16 c + 15
+    uint32_t q[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = bf16_bits_to_float(sv[fp8_vpos_tok(c * 16 + e * 4 + u) * PW * 2 + i]) * v_inv;
+      q[e] = uint32_t(pack_e4m3x2(x[0], x[1])) | (uint32_t(pack_e4m3x2(x[2], x[3])) << 16);
+    }
+    *reinterpret_cast<uint4*>(vdst + fp8_page_offset(i, c * 16, P)) = make_uint4(q[0], q[1], q[2], q[3]);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPackThreads) gather_fp8_kernel(PackArgs a, const uint8_t* __restrict__ kpool,
+                                                                  const uint8_t* __restrict__ vpool,
+                                                                  uint8_t* __restrict__ kd, uint8_t* __restrict__ vd) {
+  constexpr int P = 64;
+  constexpr int SP = P + 4;  // staging pitch (bytes) of the V codes [D][tokens]
+  __shared__ uint8_t stage[D * SP];
+  const PageDesc pg = a.pages[blockIdx.x];
+  const HeadDesc hd = a.heads[pg.head];
+  const int64_t base = (a.stride_seq >= 0 ? int64_t(hd.b) * a.stride_seq : int64_t(hd.ctx_row0) * a.stride_tok) +
+                       int64_t(hd.kv) * a.stride_head;
+  const uint8_t* ksrc = kpool + int64_t(pg.phys) * a.page_bytes;
+  const uint8_t* vsrc = vpool + int64_t(pg.phys) * a.page_bytes;
+  for (int idx = threadIdx.x; idx < D * P / 16; idx += kPackThreads) {
+    const int i = idx / (P / 16), c = idx % (P / 16);
+    alignas(16) uint8_t b[16];
+    *reinterpret_cast<uint4*>(b) = *reinterpret_cast<const uint4*>(vsrc + fp8_page_offset(i, c * 16, P));
+#pragma unroll
+    for (int e = 0; e < 16; ++e) stage[i * SP + fp8_vpos_tok(c * 16 + e)] = b[e];
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < P * D / 16; idx += kPackThreads) {
+    const int t = idx / (D / 16), c = idx % (D / 16);
+    if (t < slot_lo(pg) || t >= slot_hi(pg)) continue;
+    const int64_t row = base + int64_t(pg.abs_start + t) * a.stride_tok;
+    reinterpret_cast<uint4*>(kd + row)[c] = *reinterpret_cast<const uint4*>(ksrc + fp8_page_offset(t, c * 16, D));
+    alignas(16) uint8_t b[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) b[e] = stage[(c * 16 + e) * SP + t];
+    reinterpret_cast<uint4*>(vd + row)[c] = *reinterpret_cast<const uint4*>(b);
+  }
+}
+
+template <int D>
+void launch_pack_fp8(const PackLaunch& L, cudaStream_t s) {
+  PackArgs a{L.heads, L.pages, L.stride_seq, L.stride_head, L.stride_tok, L.page_bytes};
+  if (L.inverse)
+    gather_fp8_kernel<D><<<L.n_pages, kPackThreads, 0, s>>>(a, static_cast<const uint8_t*>(L.kpool_in),
+                                                            static_cast<const uint8_t*>(L.vpool_in),
+                                                            static_cast<uint8_t*>(L.kdense_out),
+                                                            static_cast<uint8_t*>(L.vdense_out));
+  else
+    pack_fp8_kernel<D><<<L.n_pages, kPackThreads, 0, s>>>(a, L.k_inv, L.v_inv,
+                                                          static_cast<const __nv_bfloat16*>(L.kdense_in),
+                                                          static_cast<const __nv_bfloat16*>(L.vdense_in),
+                                                          static_cast<uint8_t*>(L.kpool_out),
+                                                          static_cast<uint8_t*>(L.vpool_out));
+}
+
 template <typename T, int D, int P>
 void launch_pack_t(const PackLaunch& L, cudaStream_t s) {
   PackArgs a{L.heads, L.pages, L.stride_seq, L.stride_head, L.stride_tok, L.page_bytes};
@@ -143,7 +252,10 @@ void launch_pack_t(const PackLaunch& L, cudaStream_t s) {
 
 void launch_pack(const PackLaunch& L, cudaStream_t s) {
   if (L.n_pages == 0) return;
-  if (L.bf16) {
+  if (L.fp8) {
+    if (L.D == 128) launch_pack_fp8<128>(L, s);
+    else launch_pack_fp8<64>(L, s);
+  } else if (L.bf16) {
     if (L.D == 128) launch_pack_t<__nv_bfloat16, 128, 64>(L, s);
     else launch_pack_t<__nv_bfloat16, 64, 64>(L, s);
   } else if (L.P == 16) {

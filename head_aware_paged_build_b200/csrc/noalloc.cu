@@ -106,7 +106,9 @@ extern "C" sp_status segpaged_attention_decode_noalloc(const sp_plan* plan, cons
   L.bf16 = plan->prob.dtype == SP_BF16;
   L.page_bytes = plan->sizes.page_bytes;
   L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
-  L.scale_log2 = scale * 1.4426950408889634f;
+  L.scale_log2 = scale * 1.4426950408889634f * (plan->fp8 ? plan->k_scale : 1.f);
+  L.fp8 = plan->fp8;
+  L.v_scale = plan->fp8 ? plan->v_scale : 1.f;
   L.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + plan->partial_offset);
   L.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + kStatusBytes);
   L.status = status;

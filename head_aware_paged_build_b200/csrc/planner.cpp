@@ -53,6 +53,13 @@ sp_status validate(const sp_problem& p) {
     return fail(SP_ERR_UNSUPPORTED, "num_q_heads must be a multiple of num_kv_heads");
   if (p.num_q_heads / p.num_kv_heads > kMaxGroup)
     return fail(SP_ERR_UNSUPPORTED, "at most 16 q-heads per kv-head");
+  if (p.kv_dtype != 0 && p.kv_dtype != p.dtype && p.kv_dtype != SP_E4M3)
+    return fail(SP_ERR_UNSUPPORTED, "kv_dtype must be 0, the problem dtype or SP_E4M3");
+  if (p.kv_dtype == SP_E4M3) {
+    if (p.dtype != SP_BF16) return fail(SP_ERR_UNSUPPORTED, "E4M3 pages need bf16 queries");
+    if (!(p.k_scale > 0.f) || !(p.v_scale > 0.f) || p.k_scale > 3.0e38f || p.v_scale > 3.0e38f)
+      return fail(SP_ERR_INVALID_ARG, "E4M3 pages need finite k_scale, v_scale > 0");
+  }
   int64_t rows = 0;
   for (int b = 0; b < p.batch; ++b) {
     const int64_t L = p.ctx_len[b], q0 = p.q_start[b];
@@ -120,6 +127,10 @@ sp_status plan_build(sp_plan& pl) {
   for (int b = 0; b < B; ++b) decode = decode && (pl.ctx_len[b] - pl.q_start[b] == 1);
   const bool ring = (p.flags & SP_FLAG_RING) != 0;
   if (ring && !decode) return fail(SP_ERR_UNSUPPORTED, "ring plans are decode plans (one query per sequence)");
+  pl.fp8 = p.kv_dtype == SP_E4M3;
+  if (pl.fp8 && !decode) return fail(SP_ERR_UNSUPPORTED, "E4M3 pages are supported for decode plans");
+  pl.k_scale = pl.fp8 ? p.k_scale : 1.f;
+  pl.v_scale = pl.fp8 ? p.v_scale : 1.f;
   const int64_t cap = p.append_capacity;
   if (ring) {
     for (int b = 0; b < B; ++b)
@@ -382,7 +393,7 @@ sp_status plan_build(sp_plan& pl) {
   z = sp_sizes{};
   z.num_pages = n_pages;
   z.pool_pages = p.first_page + max_id + 1;
-  z.page_bytes = int64_t(P) * D * pl.elem_bytes;
+  z.page_bytes = int64_t(P) * D * (pl.fp8 ? 1 : pl.elem_bytes);
   z.table_bytes = int64_t(pl.blob.size());
   // workspace: status word block | one arrival counter per split head | partial slots
   const int64_t partial = int64_t(n_slots) * partial_slot_floats(pl.group, D) * 4;

@@ -139,7 +139,9 @@ struct sp_plan {
   sp::TableHeader hdr{};
   sp_sizes sizes{};
   int32_t group = 1;
-  int32_t elem_bytes = 4;
+  int32_t elem_bytes = 4;                 // bytes of a Q / K / V / O element (dense inputs)
+  bool fp8 = false;                       // pages hold E4M3 codes
+  float k_scale = 1.f, v_scale = 1.f;     // E4M3 page scales
   int32_t prefill_tile = 0;
   int32_t n_partial_slots = 0;
   int64_t partial_offset = 0;  // workspace byte offset of the partial slots (status word, then counters)

@@ -32,13 +32,16 @@ class SegPagedLayer:
                  dtype: str, ctx_len: Sequence[int], q_start: Sequence[int],
                  policy: Sequence[tuple[str, int, int]], device="cuda", flags: int = 0,
                  page_ids: Sequence[int] | None = None, first_page: int = 0, target_ctas: int = 0,
-                 append_capacity: int = 0, pools: tuple[torch.Tensor, torch.Tensor] | None = None):
+                 append_capacity: int = 0, pools: tuple[torch.Tensor, torch.Tensor] | None = None,
+                 kv_dtype: str | None = None, k_scale: float = 1.0, v_scale: float = 1.0):
         self.dtype = dtype
         self.torch_dtype = {"f32": torch.float32, "bf16": torch.bfloat16}[dtype]
         self.num_q_heads, self.num_kv_heads, self.head_dim = num_q_heads, num_kv_heads, head_dim
         self.device = torch.device(device)
         self.problem = S.make_problem(batch, num_q_heads, num_kv_heads, head_dim, page_size, dtype, ctx_len,
-                                      q_start, policy, first_page, page_ids, target_ctas, flags, append_capacity)
+                                      q_start, policy, first_page, page_ids, target_ctas, flags, append_capacity,
+                                      kv_dtype, k_scale, v_scale)
+        self.kv_dtype = kv_dtype or dtype
         self.plan = S.segpaged_plan_create(self.problem)
         self.sizes = S.segpaged_plan_sizes(self.plan)
         z = self.sizes

@@ -19,12 +19,12 @@ LIB_PATH = _PKG / "libsegpaged.so"
 
 SP_OK, SP_ERR_INVALID_ARG, SP_ERR_UNSUPPORTED, SP_ERR_WORKSPACE, SP_ERR_CUDA, SP_ERR_DEVICE_CHECK = range(6)
 SP_GLOBAL, SP_LOCAL, SP_DENSE, SP_RETRIEVAL = range(4)
-SP_F32, SP_BF16 = 0, 1
+SP_F32, SP_BF16, SP_E4M3 = 0, 1, 2
 SP_FLAG_DENSE_MASKED = 1
 SP_FLAG_RING = 2
 SP_VARLEN = -1
 KIND_CODES = {"global": SP_GLOBAL, "local": SP_LOCAL, "dense": SP_DENSE, "retrieval": SP_RETRIEVAL}
-DTYPE_CODES = {"f32": SP_F32, "bf16": SP_BF16}
+DTYPE_CODES = {"f32": SP_F32, "bf16": SP_BF16, "e4m3": SP_E4M3}
 
 # every symbol include/segpaged.h declares
 EXPORTED = ("segpaged_plan_create", "segpaged_plan_destroy", "segpaged_plan_sizes",
@@ -50,7 +50,8 @@ class sp_problem(ctypes.Structure):
                 ("ctx_len", ctypes.POINTER(ctypes.c_int32)), ("q_start", ctypes.POINTER(ctypes.c_int32)),
                 ("policy", ctypes.POINTER(sp_head_policy)), ("first_page", ctypes.c_int64),
                 ("page_ids", ctypes.POINTER(ctypes.c_int32)), ("target_ctas", ctypes.c_int32),
-                ("flags", ctypes.c_uint32), ("append_capacity", ctypes.c_int32)]
+                ("flags", ctypes.c_uint32), ("append_capacity", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
 
 class sp_sizes(ctypes.Structure):
@@ -135,7 +136,8 @@ def _check(st: int, where: str) -> None:
 def make_problem(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, page_size: int, dtype: str,
                  ctx_len: Sequence[int], q_start: Sequence[int], policy: Sequence[tuple[str, int, int]],
                  first_page: int = 0, page_ids: Sequence[int] | None = None, target_ctas: int = 0,
-                 flags: int = 0, append_capacity: int = 0):
+                 flags: int = 0, append_capacity: int = 0, kv_dtype: str | int | None = None,
+                 k_scale: float = 1.0, v_scale: float = 1.0):
     """Build an ``sp_problem`` plus the host arrays it points to (kept alive in the result)."""
     B = batch
     ctx = (ctypes.c_int32 * B)(*ctx_len)
@@ -147,7 +149,9 @@ def make_problem(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
                       DTYPE_CODES[dtype] if isinstance(dtype, str) else dtype,
                       ctx, q0, pol, first_page,
                       ctypes.cast(ids, ctypes.POINTER(ctypes.c_int32)) if ids is not None else None,
-                      target_ctas, flags, append_capacity)
+                      target_ctas, flags, append_capacity,
+                      0 if kv_dtype is None else (DTYPE_CODES[kv_dtype] if isinstance(kv_dtype, str) else kv_dtype),
+                      k_scale, v_scale)
     prob._keep = (ctx, q0, pol, ids)
     return prob
 

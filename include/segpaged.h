@@ -24,8 +24,9 @@
  *  - Positions are 0-based absolute positions in a sequence.  Query q-head h
  *    uses kv-head h / (num_q_heads / num_kv_heads).
  *  - Supported: head_dim 64 or 128; dtype fp32 with page size 16 or 64; dtype
- *    bf16 with page size 64; num_q_heads / num_kv_heads <= 16.  Anything else
- *    returns SP_ERR_UNSUPPORTED.
+ *    bf16 with page size 64 (pages bf16, or FP8 E4M3 for decode plans);
+ *    num_q_heads / num_kv_heads <= 16.  Anything else returns
+ *    SP_ERR_UNSUPPORTED.
  */
 #ifndef SEGPAGED_H_
 #define SEGPAGED_H_
@@ -63,7 +64,8 @@ typedef enum {
  * implemented: the pages give no scoring rule; it returns SP_ERR_UNSUPPORTED. */
 typedef enum { SP_GLOBAL = 0, SP_LOCAL = 1, SP_DENSE = 2, SP_RETRIEVAL = 3 } sp_kind;
 
-typedef enum { SP_F32 = 0, SP_BF16 = 1 } sp_dtype;
+/* SP_E4M3 is a page type only (sp_problem.kv_dtype): FP8 E4M3 codes, 1 byte. */
+typedef enum { SP_F32 = 0, SP_BF16 = 1, SP_E4M3 = 2 } sp_dtype;
 
 /* Problem flags. */
 enum {
@@ -111,6 +113,13 @@ typedef struct {
  *   append_capacity  SP_FLAG_RING plans: extra tokens per sequence that
  *               segpaged_decode_append may add (GLOBAL heads reserve pages for
  *               them); must be 0 otherwise
+ *   kv_dtype, k_scale, v_scale  SP_E4M3: pages hold FP8 E4M3 codes of
+ *               fp32(x * (1 / scale)) (round to nearest even, saturating at
+ *               +-448), one scale per layer for K and one for V; attention uses
+ *               code * scale.  Supported for bf16 decode plans (page size 64);
+ *               halves the bytes decode reads.  The pages say the system works
+ *               with FP8 quantisation ("RedKnot overview (aipuzi)", FAQ Q5); the
+ *               per-layer scale is this library's reading.
  */
 typedef struct {
   int32_t batch;
@@ -127,6 +136,8 @@ typedef struct {
   int32_t target_ctas;
   uint32_t flags;
   int32_t append_capacity; /* ring plans: tokens every sequence may still gain */
+  int32_t kv_dtype;        /* page type: 0 = dtype, or SP_E4M3 (bf16 decode plans) */
+  float k_scale, v_scale;  /* SP_E4M3 pages: stored code = E4M3(x * (1 / scale)) */
 } sp_problem;
 
 typedef struct {
@@ -192,14 +203,16 @@ SP_API sp_status segpaged_table_write(const sp_plan* plan, void* d_table, size_t
  *                     Covers [B,Hkv,Lmax,d] (stride_tok = d) and varlen
  *                     [sum L, Hkv, d] (stride_tok = Hkv*d, SP_VARLEN) layouts.
  *   k_pool, v_pool    device, pool_pages * page_bytes each, 16-byte aligned.
- * Base pointers and strides must give 16-byte aligned rows. */
+ * Base pointers and strides must give 16-byte aligned rows.  With SP_E4M3
+ * pages the dense input is bf16 and is quantised here. */
 SP_API sp_status build_segpaged_cache(const sp_plan* plan, const void* d_table, const void* k_dense,
                                const void* v_dense, int64_t stride_seq, int64_t stride_head,
                                int64_t stride_tok, void* k_pool, void* v_pool, void* stream);
 
 /* Inverse of build_segpaged_cache, for checking: writes each stored row back
  * into dense-shaped k_out / v_out (same addressing rules); rows that are not
- * stored are left untouched. */
+ * stored are left untouched.  With SP_E4M3 pages it writes the 1-byte codes
+ * (strides then count bytes). */
 SP_API sp_status segpaged_gather(const sp_plan* plan, const void* d_table, const void* k_pool,
                           const void* v_pool, void* k_out, void* v_out, int64_t stride_seq,
                           int64_t stride_head, int64_t stride_tok, void* stream);

@@ -49,6 +49,10 @@ def _bind(lib):
     lib.oracle_visible_pairs.argtypes = [ctypes.c_int, i64, i64, i64, i64]
     lib.oracle_visible_pairs.restype = i64
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_e4m3_encode.argtypes = [i64, p, ctypes.c_float, p]
+    lib.oracle_e4m3_encode.restype = None
+    lib.oracle_e4m3_decode.argtypes = [i64, p, dbl, p]
+    lib.oracle_e4m3_decode.restype = None
     return lib
 
 
@@ -119,3 +123,21 @@ def problem_rows(q_rows, q_positions, k_dense, v_dense, kind, sink, window, scal
         return np.asarray(t, np.float64)
     return attention_rows(np64(q_rows), np.asarray(q_positions, np.int64), np64(k_dense),
                           np64(v_dense), kind, sink, window, scale, lib)
+
+
+def e4m3_encode(x, inv_scale: float, lib=None) -> np.ndarray:
+    """E4M3 codes (uint8) of fp32(x * inv_scale): nearest, ties to even, saturating at +-448."""
+    lib = lib or load()
+    xf = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    codes = np.empty(xf.shape, np.uint8)
+    lib.oracle_e4m3_encode(xf.size, _ptr(xf), float(np.float32(inv_scale)), _ptr(codes))
+    return codes
+
+
+def e4m3_decode(codes, scale: float, lib=None) -> np.ndarray:
+    """fp64 values of E4M3 codes times scale."""
+    lib = lib or load()
+    c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    out = np.empty(c.shape, np.float64)
+    lib.oracle_e4m3_decode(c.size, _ptr(c), float(scale), _ptr(out))
+    return out

@@ -150,3 +150,55 @@ int64_t oracle_visible_pairs(int kind, int64_t sink, int64_t window, int64_t L, 
     for (int64_t j = 0; j <= p; ++j) n += oracle_sees(kind, sink, window, p, j);
   return n;
 }
+
+/*
+ * FP8 E4M3 codes for KV pages quantised with a per-layer scale (the pages
+ * say only that the system works with FP8 quantisation; the plainest
+ * reading is a per-layer scale, code = round(x * inv_scale), value =
+ * code * scale).  E4M3 as defined by the OCP 8-bit floating point format:
+ * 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
+ * S.1111.111 is NaN, largest finite magnitude 448 = 1.75 * 2^8, subnormals
+ * m * 2^-9.  Encoding rounds to nearest, ties to even, and saturates finite
+ * values to +-448.  The product x * inv_scale is formed in fp32 (the
+ * precision in which the GPU takes the same decision).
+ */
+static double oracle_e4m3_value(uint8_t c) {
+  const int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double mag = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+  return sgn ? -mag : mag;
+}
+
+static uint8_t oracle_e4m3_encode_f32(float xf) {
+  const double x = (double)xf;
+  if (x != x) return 0x7F;
+  const uint8_t sgn = (x < 0.0 || (x == 0.0 && signbit(x))) ? 0x80 : 0;
+  const double a = fabs(x);
+  if (a >= 448.0) return sgn | 0x7E;
+  /* The values of codes 0 .. 0x7E increase with the code: find the first
+   * code whose value is >= a, then take the nearer of it and the code below
+   * (a tie goes to the even code). */
+  int lo = 0, hi = 0x7E;
+  while (lo < hi) {
+    const int mid = (lo + hi) / 2;
+    if (oracle_e4m3_value((uint8_t)mid) >= a) hi = mid;
+    else lo = mid + 1;
+  }
+  uint8_t best = (uint8_t)lo;
+  if (lo > 0) {
+    const double up = oracle_e4m3_value((uint8_t)lo) - a, down = a - oracle_e4m3_value((uint8_t)(lo - 1));
+    if (down < up || (down == up && ((lo - 1) & 1) == 0)) best = (uint8_t)(lo - 1);
+  }
+  return sgn | best;
+}
+
+/* codes[i] = E4M3 code of fp32(x[i] * inv_scale) (x[i] given as float). */
+void oracle_e4m3_encode(int64_t n, const float* x, float inv_scale, uint8_t* codes) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) codes[i] = oracle_e4m3_encode_f32(x[i] * inv_scale);
+}
+
+/* values[i] = value of codes[i] times scale, in fp64. */
+void oracle_e4m3_decode(int64_t n, const uint8_t* codes, double scale, double* values) {
+  for (int64_t i = 0; i < n; ++i) values[i] = oracle_e4m3_value(codes[i]) * scale;
+}

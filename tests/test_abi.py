@@ -272,3 +272,31 @@ def test_ring_plan_validation():
     plan = S.segpaged_plan_create(S.make_problem(**base, q_start=[99]))
     assert S.load().segpaged_decode_append(plan, 256, 16, 16, 0, 0, 16, 16, 256, None) == S.SP_ERR_INVALID_ARG
     S.segpaged_plan_destroy(plan)
+
+
+def test_e4m3_pages_plan_and_validation():
+    """E4M3 pages: 1-byte pages for bf16 decode plans; everything else is rejected before any launch."""
+    base = dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=128, page_size=64, dtype="bf16",
+                ctx_len=[300, 77], q_start=[299, 76], policy=[("global", 0, 0), ("local", 4, 64)] * 2)
+    plan = S.segpaged_plan_create(S.make_problem(**base, kv_dtype="e4m3", k_scale=0.5, v_scale=2.0))
+    ref = S.segpaged_plan_create(S.make_problem(**base))
+    z, zr = S.segpaged_plan_sizes(plan), S.segpaged_plan_sizes(ref)
+    assert z.page_bytes == 64 * 128 and zr.page_bytes == 2 * 64 * 128
+    assert (z.num_pages, z.stored_token_heads, z.visible_pairs) == (zr.num_pages, zr.stored_token_heads,
+                                                                   zr.visible_pairs)
+    S.segpaged_plan_destroy(plan)
+    S.segpaged_plan_destroy(ref)
+    # the problem dtype as kv_dtype is the default layout
+    plan = S.segpaged_plan_create(S.make_problem(**base, kv_dtype="bf16"))
+    assert S.segpaged_plan_sizes(plan).page_bytes == 2 * 64 * 128
+    S.segpaged_plan_destroy(plan)
+    prefill = dict(base, q_start=[0, 0])
+    for kw, code in ((dict(base, kv_dtype="e4m3", k_scale=0.0), S.SP_ERR_INVALID_ARG),
+                     (dict(base, kv_dtype="e4m3", v_scale=-1.0), S.SP_ERR_INVALID_ARG),
+                     (dict(base, kv_dtype="e4m3", k_scale=float("inf")), S.SP_ERR_INVALID_ARG),
+                     (dict(base, kv_dtype="e4m3", v_scale=float("nan")), S.SP_ERR_INVALID_ARG),
+                     (dict(base, kv_dtype=9), S.SP_ERR_UNSUPPORTED),
+                     (dict(prefill, kv_dtype="e4m3"), S.SP_ERR_UNSUPPORTED),
+                     (dict(BASE, kv_dtype="e4m3"), S.SP_ERR_UNSUPPORTED)):  # fp32 queries
+        st, pl = S.segpaged_plan_create_status(S.make_problem(**kw))
+        assert st == code and not pl, (kw, S.last_error())

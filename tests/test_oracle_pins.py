@@ -236,3 +236,54 @@ def test_golden_deepseek_policy_savings():
         assert saving == pytest.approx(frac_local * (1 - (s + w) / L), abs=1e-12)
         assert float(g["kv_saving_low"]) <= saving <= float(g["kv_saving_high"])
     assert int(g["default_window"]) == 512 and int(g["default_sink"]) == 4
+
+
+def test_e4m3_codes_fixed_by_the_format():
+    """Values fixed by the E4M3 definition (bias 7, 3 mantissa bits, max 448, subnormal step 2^-9)."""
+    vals = np.array([0.0, 1.0, -1.0, 448.0, 500.0, -1e6, 2.0 ** -9, 2.0 ** -6, 1.125, 0.875 * 2 ** -6,
+                     240.0, 256.0], np.float32)
+    want = [0x00, 0x38, 0xB8, 0x7E, 0x7E, 0xFE, 0x01, 0x08, 0x39, 0x07, 0x77, 0x78]
+    assert oracle.e4m3_encode(vals, 1.0).tolist() == want
+    back = oracle.e4m3_decode(np.array(want, np.uint8), 1.0)
+    np.testing.assert_array_equal(back, [0, 1, -1, 448, 448, -448, 2 ** -9, 2 ** -6, 1.125, 0.875 * 2 ** -6, 240, 256])
+
+
+def test_e4m3_rounds_to_nearest_even_and_saturates():
+    # 1.0625 lies halfway between 1.0 (code 0x38, even) and 1.125 (0x39): ties to even -> 1.0
+    # 1.1875 lies halfway between 1.125 (0x39) and 1.25 (0x3A, even) -> 1.25
+    assert oracle.e4m3_encode(np.array([1.0625, 1.1875, 1.07], np.float32), 1.0).tolist() == [0x38, 0x3A, 0x39]
+    # every code's value encodes back to itself; scaling divides by the scale before rounding
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    vals = oracle.e4m3_decode(codes, 1.0).astype(np.float32)
+    assert np.array_equal(oracle.e4m3_encode(vals, 1.0)[codes != 0x80], codes[codes != 0x80])
+    assert oracle.e4m3_encode(np.array([3.0], np.float32), 0.5).tolist() == [0x3C]  # 1.5 -> 0.0111.100
+    # brute force: the chosen code is a nearest finite value of every random input
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal(2000) * 50).astype(np.float32)
+    c = oracle.e4m3_encode(x, 1.0)
+    finite = oracle.e4m3_decode(codes, 1.0)
+    best = np.abs(x[:, None].astype(np.float64) - finite[None, :]).min(1)
+    got = np.abs(x.astype(np.float64) - oracle.e4m3_decode(c, 1.0))
+    clipped = np.abs(x) > 448
+    assert np.all(got[~clipped] == best[~clipped])
+
+
+def test_e4m3_every_midpoint_goes_to_the_even_neighbour():
+    """Halfway between any two adjacent finite values (exact in fp32) the even code wins, both signs."""
+    codes = np.arange(0x7F, dtype=np.uint8)  # 0 .. 0x7E: increasing values
+    vals = oracle.e4m3_decode(codes, 1.0)
+    mid = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    assert np.array_equal(mid.astype(np.float64), (vals[:-1] + vals[1:]) / 2)  # exact in fp32
+    even = np.where(codes[:-1] % 2 == 0, codes[:-1], codes[1:])
+    assert np.array_equal(oracle.e4m3_encode(mid, 1.0), even)
+    assert np.array_equal(oracle.e4m3_encode(-mid, 1.0), even | 0x80)
+    # just above / below each midpoint: the nearer neighbour
+    up = np.nextafter(mid, np.float32(np.inf))
+    down = np.nextafter(mid, np.float32(0))
+    assert np.array_equal(oracle.e4m3_encode(up, 1.0), codes[1:])
+    assert np.array_equal(oracle.e4m3_encode(down, 1.0), codes[:-1])
+    # the subnormal range against brute force
+    x = np.random.default_rng(5).uniform(-2.0 ** -5, 2.0 ** -5, 4000).astype(np.float32)
+    c = oracle.e4m3_encode(x, 1.0)
+    best = np.abs(x[:, None].astype(np.float64) - np.concatenate([vals, -vals])[None, :]).min(1)
+    assert np.all(np.abs(x.astype(np.float64) - oracle.e4m3_decode(c, 1.0)) == best)

@@ -27,14 +27,18 @@ def _close(a: torch.Tensor, b: torch.Tensor, tol_abs: float, cos_min: float) -> 
     assert float(a @ b / (a.norm() * b.norm())) >= cos_min
 
 
-@pytest.mark.parametrize("name", ["mistral", "ragged"])
+@pytest.mark.parametrize("name", ["mistral", "ragged", "mistral-e4m3"])
 def test_noalloc_decode_matches_workspace_decode_twice(name):
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
-    wl = W.ALL[name]()
+    wl = W.ALL[name.split("-")[0]]()
     prob = wl.decode_problem()
     k, v = W.dense_kv(prob, device="cuda")
     q = W.queries(prob, device="cuda")
-    layer = layer_for(prob)
+    if name.endswith("e4m3"):  # E4M3 pages, per-tensor scales amax / 448
+        layer = layer_for(prob, kv_dtype="e4m3", k_scale=float(k.float().abs().max()) / 448,
+                          v_scale=float(v.float().abs().max()) / 448)
+    else:
+        layer = layer_for(prob)
     layer.build(k, v)
     ref_o, ref_l = layer.attention(q)
     torch.cuda.synchronize()
