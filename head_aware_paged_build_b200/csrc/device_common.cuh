@@ -31,12 +31,21 @@ __host__ __device__ __forceinline__ int64_t vpage_chunk_offset_bf16(int i, int c
   return int64_t(i) * 128 + ((c16 ^ (i & 7)) << 4);
 }
 // E4M3 pages (P = 64): K page [64 tokens][D] codes, V page [D][64 positions]
-// codes; byte (row, col) of a page with `pitch`-byte rows lives at its linear
-// address with the 16-byte chunks of each 128-byte line XOR-swizzled by the
-// line index.  A warp reading 8 consecutive rows at one column then hits 8
-// distinct chunks (no bank conflicts) for pitch 64 and 128.
-__host__ __device__ __forceinline__ int fp8_page_offset(int row, int col, int pitch) {
-  const int a = row * pitch + col;
+// codes.  A byte lives at its linear address with the 16-byte chunks of each
+// 128-byte line XOR-swizzled by the line index, in the pattern that keeps the
+// decode's shared-memory reads free of bank conflicts:
+//  K: each half-warp reads 32 contiguous bytes of 4 consecutive token rows
+//     (64-bit loads): chunks XOR 2 * (line mod 4) give the 4 rows distinct
+//     32-byte bank groups for D = 64 and 128;
+//  V: a warp reads 16 bytes of 8 consecutive dimension rows (32-bit loads):
+//     chunks XOR (line mod 8) give the 8 rows distinct 16-byte bank groups.
+__host__ __device__ __forceinline__ int fp8_kpage_offset(int t, int col, int D) {
+  const int a = t * D + col;
+  const int line = a >> 7;
+  return (line << 7) | ((((a >> 4) & 7) ^ ((line & 3) << 1)) << 4) | (a & 15);
+}
+__host__ __device__ __forceinline__ int fp8_vpage_offset(int i, int pos) {
+  const int a = i * 64 + pos;
   const int line = a >> 7;
   return (line << 7) | ((((a >> 4) & 7) ^ (line & 7)) << 4) | (a & 15);
 }

@@ -59,11 +59,11 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendLaunch a) 
                     x3 = __uint_as_float(w[2 * h + 1] & 0xffff0000u) * a.k_inv;
         q[h] = uint32_t(pack_e4m3x2(x0, x1)) | (uint32_t(pack_e4m3x2(x2, x3)) << 16);
       }
-      *reinterpret_cast<uint2*>(kdst + fp8_page_offset(slot, c * 8, D)) = make_uint2(q[0], q[1]);
+      *reinterpret_cast<uint2*>(kdst + fp8_kpage_offset(slot, c * 8, D)) = make_uint2(q[0], q[1]);
     }
     for (int i = threadIdx.x; i < D; i += kAppendThreads) {
       const float x = __bfloat162float(vn[i]) * a.v_inv;
-      vdst[fp8_page_offset(i, fp8_vtok_pos(slot), P)] = uint8_t(pack_e4m3x2(x, 0.f));
+      vdst[fp8_vpage_offset(i, fp8_vtok_pos(slot))] = uint8_t(pack_e4m3x2(x, 0.f));
     }
   } else {
   for (int c = threadIdx.x; c < CR; c += kAppendThreads) {

@@ -36,6 +36,7 @@ namespace {
 constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLazyLog2 = 8.f;  // decode softmax: rescale O only when the max grows by more than 2^8
 
 template <int D, int NST, bool FP8>
 struct DecodeSmem {
@@ -45,7 +46,8 @@ struct DecodeSmem {
   static constexpr int kMergeOff = NST * 2 * kPageBytes;
   static constexpr int kMlOff = kMergeOff + kConsumerWarps * kMaxGroup * kMergePitch * 4;
   static constexpr int kBarOff = kMlOff + kConsumerWarps * kMaxGroup * 2 * 4;
-  static constexpr int kBytes = kBarOff + 2 * NST * 8;
+  static constexpr int kDescOff = kBarOff + 2 * NST * 8;  // PageDesc of each stage (16-byte aligned)
+  static constexpr int kBytes = kDescOff + NST * 16;
 };
 
 template <int D, int NST, bool FP8>
@@ -62,6 +64,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
   float* mlbuf = reinterpret_cast<float*>(smem + S::kMlOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
   uint64_t* empty = full + NST;
+  PageDesc* sdesc = reinterpret_cast<PageDesc*>(smem + S::kDescOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ib = a.cta_begin[blockIdx.x], ie = a.cta_begin[blockIdx.x + 1];
@@ -82,29 +85,50 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
 
   if (warp == kConsumerWarps) {
     // ---------------- producer ----------------
-    if (lane == 0) {
-      for (int g = gb, k = 0; g < ge; ++g, ++k) {
+    // The warp's lanes fetch the next 32 page descriptors together, so no global
+    // load sits between two stage refills; lane 0 walks them: wait for the stage,
+    // publish the descriptor in shared memory (the consumers read it there after
+    // the stage's full barrier), start the copies.
+    int k = 0;
+    bool ok = true;
+    for (int base = gb; base < ge && ok; base += 32) {
+      const int4 mine = base + lane < ge ? __ldg(reinterpret_cast<const int4*>(a.pages + base + lane))
+                                         : make_int4(0, 0, 0, 0);
+      const int n = min(32, ge - base);
+      for (int i = 0; i < n; ++i, ++k) {
+        PageDesc pgd;
+        pgd.phys = __shfl_sync(0xffffffffu, mine.x, i);
+        pgd.abs_start = __shfl_sync(0xffffffffu, mine.y, i);
+        pgd.span = __shfl_sync(0xffffffffu, mine.z, i);
+        pgd.head = __shfl_sync(0xffffffffu, mine.w, i);
         const int s = k % NST;
-        if (k >= NST && !mbar_wait(&empty[s], ((k / NST) & 1) ^ 1)) {
-          record_error(a.status, kDevTimeoutEmpty);
+        int good = 1;
+        if (lane == 0) {
+          if (k >= NST && !mbar_wait(&empty[s], ((k / NST) & 1) ^ 1)) {
+            record_error(a.status, kDevTimeoutEmpty);
+            good = 0;
+          } else {
+            sdesc[s] = pgd;
+            uint8_t* kd = stage + s * 2 * PB;
+            if (slot_hi(pgd) > slot_lo(pgd)) {
+              mbar_arrive_expect_tx(&full[s], 2 * PB);
+              bulk_g2s(kd, kpool + int64_t(pgd.phys) * a.page_bytes, PB, &full[s]);
+              bulk_g2s(kd + PB, vpool + int64_t(pgd.phys) * a.page_bytes, PB, &full[s]);
+            } else {
+              mbar_arrive(&full[s]);  // empty page (ring or reserved): nothing to copy
+            }
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, good, 0)) {
+          ok = false;
           break;
         }
-        const PageDesc pgd = a.pages[g];
-        const int64_t phys = pgd.phys;
-        uint8_t* kd = stage + s * 2 * PB;
-        if (slot_hi(pgd) > slot_lo(pgd)) {
-          mbar_arrive_expect_tx(&full[s], 2 * PB);
-          bulk_g2s(kd, kpool + phys * a.page_bytes, PB, &full[s]);
-          bulk_g2s(kd + PB, vpool + phys * a.page_bytes, PB, &full[s]);
-        } else {
-          mbar_arrive(&full[s]);  // empty page (ring or reserved): nothing to copy
-        }
       }
-      // Do not leave while copies into this CTA's shared memory are in flight.
-      const int n = ge - gb;
-      for (int k = (n > NST ? n - NST : 0); k < n; ++k)
-        if (!mbar_wait(&full[k % NST], (k / NST) & 1)) break;
     }
+    // Do not leave while copies into this CTA's shared memory are in flight.
+    if (lane == 0)
+      for (int j = (k > NST ? k - NST : 0); j < k; ++j)
+        if (!mbar_wait(&full[j % NST], (j / NST) & 1)) break;
     return;
   }
 
@@ -113,6 +137,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
   const int r0 = grp, r1 = grp + 8;
   const int G = a.group;
   const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q);
+  const float scale_log2 = a.scale_log2;
   bool ok = true;
   int k = 0;
   for (int it = ib; it < ie; ++it) {
@@ -158,7 +183,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
         record_error(a.status, kDevTimeoutFull);
         ok = false;
       }
-      const PageDesc pg = a.pages[g];
+      const PageDesc pg = sdesc[s];
       const int tok0 = warp * 16;
       const int lo = slot_lo(pg), hi = slot_hi(pg);
       if (ok && tok0 < hi && tok0 + 16 > lo) {
@@ -174,7 +199,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
 #pragma unroll
             for (int n = 0; n < 2; ++n) {
               const uint2 u =
-                  *reinterpret_cast<const uint2*>(kp8 + fp8_page_offset(tok0 + n * 8 + grp, j * 32 + tq * 8, D));
+                  *reinterpret_cast<const uint2*>(kp8 + fp8_kpage_offset(tok0 + n * 8 + grp, j * 32 + tq * 8, D));
               mma_f16_16816(sc[n], qa[2 * j], e4m3x2_to_f16x2(uint16_t(u.x)), e4m3x2_to_f16x2(uint16_t(u.x >> 16)));
               mma_f16_16816(sc[n], qa[2 * j + 1], e4m3x2_to_f16x2(uint16_t(u.y)),
                             e4m3x2_to_f16x2(uint16_t(u.y >> 16)));
@@ -189,26 +214,41 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
             mma_bf16_16816(sc[1], qa[kk], b2, b3);
           }
         }
-        // mask and scale (log2 domain)
+        // mask and scale (log2 domain); the warp's 16 slots are usually all valid
+        if (lo <= tok0 && hi >= tok0 + 16 && !hd.mask_local) {
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+          for (int n = 0; n < 2; ++n)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int tok = tok0 + n * 8 + tq * 2 + (e & 1);
-            bool vis = tok >= lo && tok < hi;
-            if (hd.mask_local) vis = vis && sees(1, hd.sink, hd.window, qpos, pg.abs_start + tok);
-            sc[n][e] = vis ? sc[n][e] * a.scale_log2 : -INFINITY;
-          }
+            for (int e = 0; e < 4; ++e) sc[n][e] *= scale_log2;
+        } else {
+#pragma unroll
+          for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int tok = tok0 + n * 8 + tq * 2 + (e & 1);
+              bool vis = tok >= lo && tok < hi;
+              if (hd.mask_local) vis = vis && sees(1, hd.sink, hd.window, qpos, pg.abs_start + tok);
+              sc[n][e] = vis ? sc[n][e] * scale_log2 : -INFINITY;
+            }
+        }
         float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
         float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
-        const float al0 = fast_exp2(m0 - base0), al1 = fast_exp2(m1 - base1);
-        m0 = mn0, m1 = mn1;
+        // Lazy rescaling: a row's reference m moves only when a score exceeds it
+        // by more than kLazyLog2; until then the weights 2^(s - m) stay below
+        // 2^kLazyLog2 and O and l keep their scale (no multiply of O per page).
+        if (__any_sync(0xffffffffu, mx0 > m0 + kLazyLog2 || mx1 > m1 + kLazyLog2)) {
+          const float mn0 = mx0 > m0 + kLazyLog2 ? mx0 : m0, mn1 = mx1 > m1 + kLazyLog2 ? mx1 : m1;
+          const float al0 = mn0 == m0 ? 1.f : fast_exp2(m0 - mn0), al1 = mn1 == m1 ? 1.f : fast_exp2(m1 - mn1);
+          l0 *= al0, l1 *= al1;
+#pragma unroll
+          for (int j = 0; j < NT; ++j) o[j][0] *= al0, o[j][1] *= al0, o[j][2] *= al1, o[j][3] *= al1;
+          m0 = mn0, m1 = mn1;
+        }
+        const float base0 = m0 == -INFINITY ? 0.f : m0, base1 = m1 == -INFINITY ? 0.f : m1;
         float p[2][4];
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
@@ -217,8 +257,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
           p[n][2] = fast_exp2(sc[n][2] - base1);
           p[n][3] = fast_exp2(sc[n][3] - base1);
         }
-        l0 = l0 * al0 + ((p[0][0] + p[0][1]) + (p[1][0] + p[1][1]));
-        l1 = l1 * al1 + ((p[0][2] + p[0][3]) + (p[1][2] + p[1][3]));
+        l0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+        l1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
         uint32_t pa[4];
         if constexpr (FP8) {
           pa[0] = pack_f16x2(p[0][0], p[0][1]);
@@ -230,8 +270,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
           const uint8_t* vp8 = stage + s * 2 * PB + PB;
 #pragma unroll
           for (int j = 0; j < NT; ++j) {
-            const uint32_t u = *reinterpret_cast<const uint32_t*>(vp8 + fp8_page_offset(j * 8 + grp, tok0 + tq * 4, P));
-            o[j][0] *= al0, o[j][1] *= al0, o[j][2] *= al1, o[j][3] *= al1;
+            const uint32_t u = *reinterpret_cast<const uint32_t*>(vp8 + fp8_vpage_offset(j * 8 + grp, tok0 + tq * 4));
             mma_f16_16816(o[j], pa, e4m3x2_to_f16x2(uint16_t(u)), e4m3x2_to_f16x2(uint16_t(u >> 16)));
           }
         } else {
@@ -246,8 +285,6 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunc
           const int dd = (2 * j + (mi >> 1)) * 8 + rr;
           uint32_t b0, b1, b2, b3;
           ldmatrix_x4(b0, b1, b2, b3, vst + uint32_t(vpage_chunk_offset_bf16(dd, vc)));
-          o[2 * j][0] *= al0, o[2 * j][1] *= al0, o[2 * j][2] *= al1, o[2 * j][3] *= al1;
-          o[2 * j + 1][0] *= al0, o[2 * j + 1][1] *= al0, o[2 * j + 1][2] *= al1, o[2 * j + 1][3] *= al1;
           mma_bf16_16816(o[2 * j], pa, b0, b1);
           mma_bf16_16816(o[2 * j + 1], pa, b2, b3);
         }

@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(kPackThreads) gather_kernel(PackArgs a, const 
 
 // ---------------------------------------------------------------------------
 // E4M3 pages (page size 64): K page [64 tokens][D] codes, V page [D][64
-// positions] codes, both at fp8_page_offset(); V positions order the tokens
+// positions] codes at fp8_kpage_offset() / fp8_vpage_offset(); V positions order the tokens
 // as fp8_vtok_pos() says.  Dense side: bf16 for pack, 1-byte codes for gather.
 // Codes are E4M3(fp32(x) * (1 / scale)), nearest-even, saturating.
 // ---------------------------------------------------------------------------
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_fp8_kernel(PackArgs a, floa
       kv4 = __ldg(reinterpret_cast<const uint4*>(kd + row) + c);
       vv4 = __ldg(reinterpret_cast<const uint4*>(vd + row) + c);
     }
-    *reinterpret_cast<uint2*>(kdst + fp8_page_offset(t, c * 8, D)) =
+    *reinterpret_cast<uint2*>(kdst + fp8_kpage_offset(t, c * 8, D)) =
         make_uint2(quant4(kv4.x, kv4.y, k_inv), quant4(kv4.z, kv4.w, k_inv));
     uint32_t* st = stage + t * PW + c * 4;
     st[0] = vv4.x, st[1] = vv4.y, st[2] = vv4.z, st[3] = vv4.w;
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_fp8_kernel(PackArgs a, floa
       for (int u = 0; u < 4; ++u) x[u] = bf16_bits_to_float(sv[fp8_vpos_tok(c * 16 + e * 4 + u) * PW * 2 + i]) * v_inv;
       q[e] = uint32_t(pack_e4m3x2(x[0], x[1])) | (uint32_t(pack_e4m3x2(x[2], x[3])) << 16);
     }
-    *reinterpret_cast<uint4*>(vdst + fp8_page_offset(i, c * 16, P)) = make_uint4(q[0], q[1], q[2], q[3]);
+    *reinterpret_cast<uint4*>(vdst + fp8_vpage_offset(i, c * 16)) = make_uint4(q[0], q[1], q[2], q[3]);
   }
 }
 
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kPackThreads) gather_fp8_kernel(PackArgs a, co
   for (int idx = threadIdx.x; idx < D * P / 16; idx += kPackThreads) {
     const int i = idx / (P / 16), c = idx % (P / 16);
     alignas(16) uint8_t b[16];
-    *reinterpret_cast<uint4*>(b) = *reinterpret_cast<const uint4*>(vsrc + fp8_page_offset(i, c * 16, P));
+    *reinterpret_cast<uint4*>(b) = *reinterpret_cast<const uint4*>(vsrc + fp8_vpage_offset(i, c * 16));
 #pragma unroll
     for (int e = 0; e < 16; ++e) stage[i * SP + fp8_vpos_tok(c * 16 + e)] = b[e];
   }
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(kPackThreads) gather_fp8_kernel(PackArgs a, co
     const int t = idx / (D / 16), c = idx % (D / 16);
     if (t < slot_lo(pg) || t >= slot_hi(pg)) continue;
     const int64_t row = base + int64_t(pg.abs_start + t) * a.stride_tok;
-    reinterpret_cast<uint4*>(kd + row)[c] = *reinterpret_cast<const uint4*>(ksrc + fp8_page_offset(t, c * 16, D));
+    reinterpret_cast<uint4*>(kd + row)[c] = *reinterpret_cast<const uint4*>(ksrc + fp8_kpage_offset(t, c * 16, D));
     alignas(16) uint8_t b[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) b[e] = stage[(c * 16 + e) * SP + t];
