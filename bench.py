@@ -301,11 +301,11 @@ def run_ours(args) -> None:
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(per_launch_pre / pk["bf16_tflops"], 4),
                      "peak_source": f"{pk['source']} bf16 burst",
                      "traffic": kernel_traffic("prefill_tc_kernel", csrc / "kernels_prefill_tc.cu", wl.name)},
-        "roofline_decode": {"kernel": "decode_bf16_kernel", "bound": "hbm",
+        "roofline_decode": {"kernel": "decode_mma_kernel", "bound": "hbm",
                             "achieved": round(vis_dec / (ms["decode"] * 1e-3) / 1e9, 1), "peak": pk["hbm_gbs"],
                             "unit": "GB/s", "frac": round(vis_dec / (ms["decode"] * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                             "peak_source": f"{pk['source']} HBM copy",
-                            "traffic": kernel_traffic("decode_bf16_kernel", csrc / "kernels_decode.cu", wl.name)},
+                            "traffic": kernel_traffic("decode_mma_kernel", csrc / "kernels_decode.cu", wl.name)},
         "decode_e4m3": {"ms": round(fp8_ms, 5), "visible_kv_bytes": vis_dec // eb,
                         "GB/s": round(weak_rate(vis_dec // eb, world, fp8_ms) / 1e9, 1),
                         "frac_hbm": round(vis_dec // eb / (fp8_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),

@@ -51,7 +51,7 @@ struct DecodeSmem {
 };
 
 template <int D, int NST, bool FP8>
-__global__ void __launch_bounds__(kDecodeThreads) decode_bf16_kernel(DecodeLaunch a) {
+__global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch a) {
   using S = DecodeSmem<D, NST, FP8>;
   constexpr int P = 64;
   constexpr int PB = S::kPageBytes;
@@ -542,10 +542,10 @@ constexpr int kStagesBf16 = 2;
 constexpr int kStagesFp8 = 4;  // half-size pages: twice the stages for the same bytes in flight
 
 template <int D, bool FP8>
-cudaError_t launch_bf16(const DecodeLaunch& a, cudaStream_t s) {
+cudaError_t launch_mma(const DecodeLaunch& a, cudaStream_t s) {
   constexpr int NST = FP8 ? kStagesFp8 : kStagesBf16;
   using Sm = DecodeSmem<D, NST, FP8>;
-  auto kern = decode_bf16_kernel<D, NST, FP8>;
+  auto kern = decode_mma_kernel<D, NST, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kBytes);
   if (e != cudaSuccess) return e;
   kern<<<a.n_ctas, kDecodeThreads, Sm::kBytes, s>>>(a);  // split heads are merged in-kernel
@@ -569,8 +569,8 @@ cudaError_t launch_f32(const DecodeLaunch& a, cudaStream_t s) {
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t s) {
   if (a.n_ctas == 0) return cudaSuccess;
-  if (a.fp8) return a.D == 128 ? launch_bf16<128, true>(a, s) : launch_bf16<64, true>(a, s);
-  if (a.bf16) return a.D == 128 ? launch_bf16<128, false>(a, s) : launch_bf16<64, false>(a, s);
+  if (a.fp8) return a.D == 128 ? launch_mma<128, true>(a, s) : launch_mma<64, true>(a, s);
+  if (a.bf16) return a.D == 128 ? launch_mma<128, false>(a, s) : launch_mma<64, false>(a, s);
   if (a.P == 16) return a.D == 128 ? launch_f32<128, 16>(a, s) : launch_f32<64, 16>(a, s);
   return a.D == 128 ? launch_f32<128, 64>(a, s) : launch_f32<64, 64>(a, s);
 }
