@@ -59,7 +59,8 @@ def config_of(wl, n_gpus: int) -> dict:
     return {
         "workload": ("Llama-70B-shaped layer, 32K context" if wl.name.startswith("llama")
                      else {"mistral": "Mistral-7B-shaped layer, 8K context", "mha": "MHA-style layer, 128K context",
-                           "ragged": "ragged decode batch"}.get(wl.name, wl.name)),
+                           "ragged": "ragged decode batch, 32 sequences, context log-uniform in [1K, 64K]"}
+                     .get(wl.name, wl.name)),
         "batch": wl.batch, "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
         "context": max(wl.ctx_lens), "page_size": wl.page_size, "prefill_chunk": wl.prefill_chunk,
         "heads": {"global": kinds.get("global", 0), "local": kinds.get("local", 0)},
@@ -176,14 +177,19 @@ def run_ours(args) -> None:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     wl = workload(args.workload, rank)
-    dec, pre = wl.decode_problem(), wl.prefill_problem()
+    # A configuration without a prefill chunk (the ragged decode batch) is decode only:
+    # its step is pack + decode, and the decode kernel is its dominant kernel.
+    has_pre = wl.prefill_chunk is not None
+    dec = wl.decode_problem()
+    pre = wl.prefill_problem() if has_pre else None
     k, v = W.dense_kv(dec, device=dev, gen_device=dev)
     qd = W.queries(dec, device=dev, gen_device=dev)
-    qp = W.queries(pre, device=dev, gen_device=dev)
     Ld = layer_for(dec, device=dev)
-    Lp = layer_for(pre, device=dev)
     od, lsed = torch.empty_like(qd), torch.empty(qd.shape[:2], dtype=torch.float32, device=dev)
-    op, lsep = torch.empty_like(qp), torch.empty(qp.shape[:2], dtype=torch.float32, device=dev)
+    if has_pre:
+        qp = W.queries(pre, device=dev, gen_device=dev)
+        Lp = layer_for(pre, device=dev)
+        op, lsep = torch.empty_like(qp), torch.empty(qp.shape[:2], dtype=torch.float32, device=dev)
     flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(128 << 20, dtype=torch.float32, device=dev)
 
@@ -191,9 +197,11 @@ def run_ours(args) -> None:
         flush_w.zero_()
         flush_r.sum()
 
-    calls = [lambda: Ld.build(k, v), lambda: Ld.attention(qd, od, lsed), lambda: Lp.build(k, v),
-             lambda: Lp.attention(qp, op, lsep)]
-    names = ["pack_decode", "decode", "pack_prefill", "prefill"]
+    calls = [lambda: Ld.build(k, v), lambda: Ld.attention(qd, od, lsed)]
+    names = ["pack_decode", "decode"]
+    if has_pre:
+        calls += [lambda: Lp.build(k, v), lambda: Lp.attention(qp, op, lsep)]
+        names += ["pack_prefill", "prefill"]
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in calls]
 
     def step(record: bool):
@@ -208,7 +216,7 @@ def run_ours(args) -> None:
     for _ in range(args.warmup):
         step(False)
     torch.cuda.synchronize()
-    for lay in (Ld, Lp):
+    for lay in ((Ld, Lp) if has_pre else (Ld,)):
         assert lay.device_status() == 0, "device status word set during warm-up"
 
     if world > 1:
@@ -231,13 +239,15 @@ def run_ours(args) -> None:
 
     # ---- dense-plus-mask variant (same kernels, every head stores its whole context) ----
     Ldm = layer_for(dec, device=dev, flags=S.SP_FLAG_DENSE_MASKED)
-    Lpm = layer_for(pre, device=dev, flags=S.SP_FLAG_DENSE_MASKED)
     Ldm.build(k, v)
-    Lpm.build(k, v)
-    dm = {"decode": median_ms(lambda: Ldm.attention(qd, od, lsed), flush, 10),
-          "prefill": median_ms(lambda: Lpm.attention(qp, op, lsep), flush, 3)}
-    dm = dict(zip(("decode", "prefill"), reduce_max([dm["decode"], dm["prefill"]], world, dev)))
-    del Ldm, Lpm
+    dm = {"decode": median_ms(lambda: Ldm.attention(qd, od, lsed), flush, 10)}
+    del Ldm
+    if has_pre:
+        Lpm = layer_for(pre, device=dev, flags=S.SP_FLAG_DENSE_MASKED)
+        Lpm.build(k, v)
+        dm["prefill"] = median_ms(lambda: Lpm.attention(qp, op, lsep), flush, 3)
+        del Lpm
+    dm = dict(zip(dm.keys(), reduce_max(list(dm.values()), world, dev)))
 
     # ---- E4M3 pages: the same decode on 1-byte pages (per-tensor scales amax / 448) ----
     k_scale = float(k.abs().max()) / 448.0
@@ -255,22 +265,41 @@ def run_ours(args) -> None:
     e2e, append_us = run_e2e_serving(args, dev, wl, dec, k, v, world)
     e2e["dense_upload_variant"] = e2e_dense
 
-    zd, zp = Ld.sizes, Lp.sizes
+    zd = Ld.sizes
+    zp = Lp.sizes if has_pre else None
     eb = 2
     vis_dec = zd.stored_token_heads * 2 * wl.head_dim * eb          # K + V rows the decode must read
-    flops_pre = 4 * wl.head_dim * zp.visible_pairs                  # QK^T + PV on visible pairs
     pack_bytes = lambda z: z.stored_token_heads * 2 * wl.head_dim * eb + 2 * z.num_pages * z.page_bytes
     pk = peaks()
     dec_gbs = weak_rate(vis_dec, world, ms["decode"]) / 1e9
-    pre_tflops = weak_rate(flops_pre, world, ms["prefill"]) / 1e12
-    launches_per_step = 1 + zd.kernel_launches() + 1 + zp.kernel_launches()
+    launches_per_step = 1 + zd.kernel_launches() + ((1 + zp.kernel_launches()) if has_pre else 0)
 
     if rank != 0:
         if world > 1:
             dist.destroy_process_group()
         return
-    per_launch_pre = flops_pre / (ms["prefill"] * 1e-3) / 1e12
     csrc = ROOT / "head_aware_paged_build_b200" / "csrc"
+    roof_dec = {"kernel": "decode_mma_kernel", "bound": "hbm",
+                "achieved": round(vis_dec / (ms["decode"] * 1e-3) / 1e9, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": round(vis_dec / (ms["decode"] * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                "peak_source": f"{pk['source']} HBM copy",
+                "traffic": kernel_traffic("decode_mma_kernel", csrc / "kernels_decode.cu", wl.name)}
+    if has_pre:
+        flops_pre = 4 * wl.head_dim * zp.visible_pairs              # QK^T + PV on visible pairs
+        pre_tflops = weak_rate(flops_pre, world, ms["prefill"]) / 1e12
+        per_launch_pre = flops_pre / (ms["prefill"] * 1e-3) / 1e12
+        # Each kernel is timed alone (L2 flushes between them), so the burst GEMM figure is
+        # the denominator; the sustained one is reported beside it in "prefill".
+        pre_peak = pk["bf16_tflops"]
+        prefill = {"ms": round(ms["prefill"], 4), "visible_flops": flops_pre, "TFLOP/s": round(pre_tflops, 1),
+                   "frac_bf16_burst": round(pre_tflops / world / pk["bf16_tflops"], 4),
+                   "frac_bf16_sustained": round(pre_tflops / world / pk["bf16_tflops_sustained"], 4)}
+        roof = {"kernel": "prefill_tc_kernel", "bound": "tensor", "achieved": round(per_launch_pre, 1),
+                "peak": pre_peak, "unit": "TFLOP/s", "frac": round(per_launch_pre / pre_peak, 4),
+                "peak_source": f"{pk['source']} bf16 burst",
+                "traffic": kernel_traffic("prefill_tc_kernel", csrc / "kernels_prefill_tc.cu", wl.name)}
+    else:
+        prefill, roof = None, roof_dec  # decode-only configuration: the decode kernel dominates
     line = {
         "metric": METRIC,
         "value": round(dec_gbs, 1),
@@ -287,25 +316,17 @@ def run_ours(args) -> None:
         "config": config_of(wl, world),
         "decode": {"ms": round(ms["decode"], 5), "visible_kv_bytes": vis_dec, "GB/s": round(dec_gbs, 1),
                    "frac_hbm": round(dec_gbs / world / pk["hbm_gbs"], 4), "launches": zd.kernel_launches()},
-        "prefill": {"ms": round(ms["prefill"], 4), "visible_flops": flops_pre, "TFLOP/s": round(pre_tflops, 1),
-                    "frac_bf16_burst": round(pre_tflops / world / pk["bf16_tflops"], 4),
-                    "frac_bf16_sustained": round(pre_tflops / world / pk["bf16_tflops_sustained"], 4)},
-        "pack": {"decode_ms": round(ms["pack_decode"], 5), "prefill_ms": round(ms["pack_prefill"], 5),
+        "prefill": prefill,
+        "pack": {"decode_ms": round(ms["pack_decode"], 5),
                  "decode_GB/s": round(pack_bytes(zd) / (ms["pack_decode"] * 1e-3) / 1e9, 1),
-                 "prefill_GB/s": round(pack_bytes(zp) / (ms["pack_prefill"] * 1e-3) / 1e9, 1)},
-        "dense_masked": {"decode_ms": round(dm["decode"], 5), "prefill_ms": round(dm["prefill"], 4),
-                         "decode_skip": round(dm["decode"] / ms["decode"], 3),
-                         "prefill_skip": round(dm["prefill"] / ms["prefill"], 3),
+                 **({"prefill_ms": round(ms["pack_prefill"], 5),
+                     "prefill_GB/s": round(pack_bytes(zp) / (ms["pack_prefill"] * 1e-3) / 1e9, 1)} if has_pre else {})},
+        "dense_masked": {"decode_ms": round(dm["decode"], 5), "decode_skip": round(dm["decode"] / ms["decode"], 3),
+                         **({"prefill_ms": round(dm["prefill"], 4),
+                             "prefill_skip": round(dm["prefill"] / ms["prefill"], 3)} if has_pre else {}),
                          "kv_saving": round(1 - zd.stored_token_heads / zd.dense_token_heads, 4)},
-        "roofline": {"kernel": "prefill_tc_kernel", "bound": "tensor", "achieved": round(per_launch_pre, 1),
-                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(per_launch_pre / pk["bf16_tflops"], 4),
-                     "peak_source": f"{pk['source']} bf16 burst",
-                     "traffic": kernel_traffic("prefill_tc_kernel", csrc / "kernels_prefill_tc.cu", wl.name)},
-        "roofline_decode": {"kernel": "decode_mma_kernel", "bound": "hbm",
-                            "achieved": round(vis_dec / (ms["decode"] * 1e-3) / 1e9, 1), "peak": pk["hbm_gbs"],
-                            "unit": "GB/s", "frac": round(vis_dec / (ms["decode"] * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-                            "peak_source": f"{pk['source']} HBM copy",
-                            "traffic": kernel_traffic("decode_mma_kernel", csrc / "kernels_decode.cu", wl.name)},
+        "roofline": roof,
+        "roofline_decode": roof_dec,
         "decode_e4m3": {"ms": round(fp8_ms, 5), "visible_kv_bytes": vis_dec // eb,
                         "GB/s": round(weak_rate(vis_dec // eb, world, fp8_ms) / 1e9, 1),
                         "frac_hbm": round(vis_dec // eb / (fp8_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
@@ -330,13 +351,15 @@ def run_e2e_serving(args, dev, wl, dec, k, v, world) -> tuple[dict, float]:
     A ring plan of the decode layer is built once (untimed).  Every timed step
     copies that step's inputs from pinned host memory (the new token's K and V
     rows and its queries), appends the token (segpaged_decode_append),
-    runs decode attention and copies O and LSE back to the host.
+    runs decode attention and copies O and LSE back to the host.  The step is
+    measured replayed from a CUDA graph (runtime.DecodeStepGraph: the same
+    library calls, captured once) and issued eagerly call by call.
     """
     import torch
 
     from head_aware_paged_build_b200 import segpaged as S
     from head_aware_paged_build_b200 import workloads as W
-    from head_aware_paged_build_b200.runtime import layer_for
+    from head_aware_paged_build_b200.runtime import DecodeStepGraph, layer_for
 
     n_steps = args.warmup + max(3, args.steps // 2)
     start = W.Problem(wl, tuple(L - n_steps for L in dec.ctx_lens), tuple(L - n_steps - 1 for L in dec.ctx_lens))
@@ -384,15 +407,32 @@ def run_e2e_serving(args, dev, wl, dec, k, v, world) -> tuple[dict, float]:
         eb.record(s)
         torch.cuda.synchronize()
         app.append(ea.elapsed_time(eb) * 1e3)
-    assert layer.device_status() == 0 and probe.device_status() == 0
-    ms = reduce_max([statistics.median(times)], world, dev)[0]
+    # the same steps replayed from a CUDA graph on a fresh ring plan
+    glayer = layer_for(start, device=dev, flags=S.SP_FLAG_RING, append_capacity=n_steps)
+    glayer.build(k, v)
+    step = DecodeStepGraph(glayer)
+    gtimes = []
+    for i in range(n_steps):
+        step.k_in.copy_(kin[i]), step.v_in.copy_(vin[i]), step.q_in.copy_(qin[i])  # host-side refill
+        e0.record(s)
+        step.replay()
+        e1.record(s)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            gtimes.append(e0.elapsed_time(e1))
+    assert layer.device_status() == 0 and probe.device_status() == 0 and glayer.device_status() == 0
+    ms, ms_eager = reduce_max([statistics.median(gtimes), statistics.median(times)], world, dev)
     vis = layer.sizes.stored_token_heads * 2 * d * k.element_size()
     h2d = (kin[0].numel() + vin[0].numel() + qin[0].numel()) * kin.element_size()
     d2h = oh.numel() * oh.element_size() + lh.numel() * 4
+    path = ("pinned host q, k_new, v_new -> segpaged_decode_append -> segpaged_attention (decode, cache resident) "
+            "-> host O, LSE")
     return ({"value": round(weak_rate(vis, world, ms) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 4),
-             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-             "path": "pinned host q, k_new, v_new -> segpaged_decode_append -> segpaged_attention (decode, "
-                     "cache resident) -> host O, LSE"}, statistics.median(app))
+             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "path": path + ", replayed from a CUDA graph",
+             "eager_variant": {"value": round(weak_rate(vis, world, ms_eager) / 1e9, 2), "unit": "GB/s",
+                               "ms_per_step": round(ms_eager, 4), "h2d_bytes_per_step": h2d,
+                               "d2h_bytes_per_step": d2h, "path": path + ", issued call by call"}},
+            statistics.median(app))
 
 
 def run_e2e_dense(args, dev, layer, k, v, qd, od, lsed, world) -> dict:
@@ -509,7 +549,7 @@ def main() -> None:
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="llama", choices=("llama", "mistral", "mha", "llama_b1"))
+    ap.add_argument("--workload", default="llama", choices=("llama", "mistral", "mha", "ragged", "llama_b1"))
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="time budget of the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

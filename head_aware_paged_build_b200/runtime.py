@@ -115,3 +115,58 @@ def layer_for(prob, device="cuda", flags: int = 0, **kw) -> SegPagedLayer:
     return SegPagedLayer(batch=wl.batch, num_q_heads=wl.num_q_heads, num_kv_heads=wl.num_kv_heads,
                          head_dim=wl.head_dim, page_size=wl.page_size, dtype=wl.dtype, ctx_len=prob.ctx_lens,
                          q_start=prob.q_starts, policy=wl.policy, device=device, flags=flags, **kw)
+
+
+class DecodeStepGraph:
+    """One serving decode step of a ring-plan layer, captured once in a CUDA graph.
+
+    A step copies the new token's K and V rows ([B, Hkv, d]) and its queries
+    ([B, Hq, d]) from the pinned host buffers ``k_in``, ``v_in``, ``q_in``,
+    appends the token (``segpaged_decode_append``), runs decode attention and
+    copies O and LSE into the pinned host buffers ``out`` and ``lse``.  The
+    caller refills the inputs, then calls ``replay()``; every replay appends
+    one more token (the device table advances in place).  The graph holds the
+    same library calls an eager step makes; it removes the per-call launch
+    gaps between them.
+    """
+
+    def __init__(self, layer: SegPagedLayer, stream: torch.cuda.Stream | None = None):
+        if layer.problem.flags & S.SP_FLAG_RING == 0:
+            raise ValueError("DecodeStepGraph needs a ring plan (flags=SP_FLAG_RING)")
+        if not layer.sizes.is_decode:
+            raise ValueError("DecodeStepGraph needs a decode plan")
+        B, Hkv, Hq, d = layer.problem.batch, layer.num_kv_heads, layer.num_q_heads, layer.head_dim
+        dt, dev = layer.torch_dtype, layer.device
+        self.layer = layer
+        # Inputs and outputs each live in one staging buffer (host and device), so a
+        # step moves them with one copy each way; the named tensors are views.
+        eb = torch.empty((), dtype=dt).element_size()
+        kb, qb = B * Hkv * d * eb, B * Hq * d * eb
+        self._host_in = torch.empty(2 * kb + qb, dtype=torch.uint8).pin_memory()
+        self._dev_in = torch.empty(2 * kb + qb, dtype=torch.uint8, device=dev)
+        self._host_out = torch.empty(qb + B * Hq * 4, dtype=torch.uint8).pin_memory()
+        self._dev_out = torch.empty(qb + B * Hq * 4, dtype=torch.uint8, device=dev)
+
+        def views(buf, shapes):
+            out, off = [], 0
+            for shape, t in shapes:
+                n = int(torch.Size(shape).numel()) * torch.empty((), dtype=t).element_size()
+                out.append(buf[off:off + n].view(t).view(shape))
+                off += n
+            return out
+
+        ins = [((B, Hkv, d), dt), ((B, Hkv, d), dt), ((B, Hq, d), dt)]
+        outs = [((B, Hq, d), dt), ((B, Hq), torch.float32)]
+        self.k_in, self.v_in, self.q_in = views(self._host_in, ins)
+        self._k, self._v, self._q = views(self._dev_in, ins)
+        self.out, self.lse = views(self._host_out, outs)
+        self._o, self._lse = views(self._dev_out, outs)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=stream):
+            self._dev_in.copy_(self._host_in, non_blocking=True)
+            layer.append(self._k, self._v)
+            layer.attention(self._q, self._o, self._lse)
+            self._host_out.copy_(self._dev_out, non_blocking=True)
+
+    def replay(self) -> None:
+        self.graph.replay()

@@ -90,3 +90,41 @@ def test_ring_append_beyond_capacity_reports_and_skips():
     layer.append(k[:, :, 64].contiguous(), v[:, :, 64].contiguous())
     torch.cuda.synchronize()
     assert layer.device_status() == 6
+
+
+@pytest.mark.parametrize("kv_dtype", [None, "e4m3"])
+def test_decode_step_graph_matches_eager_steps(kv_dtype):
+    """A serving step replayed from a CUDA graph gives bitwise the eager step's O and LSE, step after step."""
+    from head_aware_paged_build_b200.runtime import DecodeStepGraph
+    L0, N = (300, 77, 130), 40
+    pol = [("local", 4, 64), ("global", 0, 0)] * len(L0)
+    final = tuple(L + N for L in L0)
+    wl = W.custom("graph", 67, len(L0), 8, 2, 128, "bf16", 64, final, pol)
+    k, v = W.dense_kv(W.Problem(wl, final, tuple(L - 1 for L in final)), device="cuda")
+    qprob = W.Problem(wl, final, tuple(L - 1 for L in L0))
+    qall, qoff = W.queries(qprob, device="cuda"), qprob.q_offsets
+    kw = dict(kv_dtype="e4m3", k_scale=0.02, v_scale=0.02) if kv_dtype else {}
+    start = W.Problem(wl, L0, tuple(L - 1 for L in L0))
+    eager = layer_for(start, flags=S.SP_FLAG_RING, append_capacity=N, **kw)
+    graphed = layer_for(start, flags=S.SP_FLAG_RING, append_capacity=N, **kw)
+    eager.build(k, v)
+    graphed.build(k, v)
+    step = DecodeStepGraph(graphed)
+    out = torch.empty(len(L0), 8, 128, dtype=k.dtype, device="cuda")
+    lse = torch.empty(len(L0), 8, dtype=torch.float32, device="cuda")
+    for i in range(N):
+        pos = [L + i for L in L0]
+        kn = torch.stack([k[b, :, p] for b, p in enumerate(pos)]).contiguous()
+        vn = torch.stack([v[b, :, p] for b, p in enumerate(pos)]).contiguous()
+        q = torch.stack([qall[qoff[b] + 1 + i] for b in range(len(L0))]).contiguous()
+        eager.append(kn, vn)
+        eager.attention(q, out, lse)
+        step.k_in.copy_(kn.cpu()), step.v_in.copy_(vn.cpu()), step.q_in.copy_(q.cpu())
+        step.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(step.out, out.cpu()), i
+        assert torch.equal(step.lse, lse.cpu()), i
+    assert eager.device_status() == 0 and graphed.device_status() == 0
+    if kv_dtype is None:  # and the last step against the oracle
+        prob = W.Problem(wl, tuple(p + 1 for p in pos), tuple(pos))
+        assert_close(compare(prob, q, k, v, step.out, step.lse), "bf16")
