@@ -195,6 +195,19 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
+// Named barrier `id` over `count` threads (whole warps) that also ANDs a
+// predicate across them: every participant gets the same answer.
+__device__ __forceinline__ bool bar_red_and(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 // 2^x on the SFU (ex2.approx, flush-to-zero); 2^-inf = 0.
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

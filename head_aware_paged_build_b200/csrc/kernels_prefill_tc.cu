@@ -11,7 +11,7 @@
 // edge, sink page, a segment's partial last page) are masked, per row, by
 // visible column intervals.
 //
-// Warp roles (320 threads):
+// Warp roles (576 threads):
 //   warp 0      producer: both Q tiles by TMA (128-byte swizzle); K and V
 //               pages by 1-D bulk copies (pool pages are stored in the tensor
 //               cores' swizzled K-major operand layout, V transposed), one
@@ -23,11 +23,13 @@
 //                 PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
 //               so that the tensor core alternates between the two tiles while
 //               their softmax warpgroups run
-//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: one row per
-//               thread; S read with tcgen05.ld, online softmax in the log2
-//               domain with a lazy rescale of O (only when the row maximum
-//               grows by more than 2^8), P written back as bf16 over the first
-//               64 columns of its own S buffer; then the epilogue (O / l, LSE).
+//   warps 2-9   softmax of tile A, warps 10-17 softmax of tile B: two threads
+//               per row, each owning one of the KV tile's two pages (64
+//               columns); S read with tcgen05.ld, online softmax in the log2
+//               domain with the row maximum exchanged between the two halves
+//               through shared memory, a lazy rescale of O (only when the row
+//               maximum grows by more than 2^8), P written back as bf16 over
+//               the half's own first 32 S columns; then the epilogue (O / l, LSE).
 // The commit that signals S_x(j) also covers P_x(j-1) V, so a softmax thread
 // holding S_x(j) may rescale O_x and overwrite P_x with no further wait.
 // Every wait is bounded; a wait that runs out records a status code, and the
@@ -44,7 +46,7 @@ namespace sp {
 namespace {
 
 constexpr int kTile = kPrefillTileTokensBf16;  // 128 query rows, 128 KV tokens
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by more than 2^8
 constexpr float kLn2 = 0.6931471805599453f;
@@ -64,7 +66,8 @@ struct TcSmem {
   static constexpr int kOffQ = 0;
   static constexpr int kOffStage = kOffQ + 2 * kQ;
   static constexpr int kOffBar = kOffStage + NS * kStage;
-  static constexpr int kBytes = kOffBar + 256 + 1024;  // barriers + 1 KB alignment slack
+  static constexpr int kOffX = kOffBar + 256;                // softmax halves' exchange: 2 tiles x 6 x 128 floats
+  static constexpr int kBytes = kOffX + 2 * 6 * 128 * 4 + 1024;  // + 1 KB alignment slack
 };
 
 struct Bars {
@@ -118,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   uint64_t* kv_free = kv_full + NS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(kv_free + NS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xbuf = reinterpret_cast<float*>(smem + Sm::kOffX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const PrefillItem it = a.items[blockIdx.x];
@@ -132,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     mbar_init(&bars->done, 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->s_full[x], 1);
-      mbar_init(&bars->p_full[x], 128);
+      mbar_init(&bars->p_full[x], 256);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -213,8 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       auto issue_pv = [&](int x, int st, bool acc) {
         const uint32_t va = st_addr + st * Sm::kStage + Sm::kK;
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          tc::mma_bf16_ts(t_o(x), t_s(x) + kk * 8,
+        for (int kk = 0; kk < kTile / 16; ++kk)  // P of page h sits at columns [64 h, 64 h + 32)
+          tc::mma_bf16_ts(t_o(x), t_s(x) + (kk >> 2) * 64 + (kk & 3) * 8,
                           tc::smem_desc_sw128(va + (kk >> 2) * (D * 128) + (kk & 3) * 32), idesc_o,
                           (acc || kk > 0) ? 1u : 0u);
       };
@@ -254,85 +258,73 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     __syncwarp();
   } else {
     // ------------------------------ softmax ------------------------------
-    const int x = (warp - 2) >> 2;  // query tile of this warpgroup
+    // Eight warps per query tile, two threads per row: half h takes the tile's
+    // page h (columns [64 h, 64 h + 64)).  The halves exchange row maxima
+    // through shared memory at a barrier that also votes on every wait, so
+    // both halves always take the same path.
+    const int x = (warp - 2) >> 3;       // query tile of this warp
+    const int h = ((warp - 2) >> 2) & 1;  // page (column half) of the KV tile
     if (x == 0 || two) {
-      const int quarter = warp & 3;
+      const int quarter = warp & 3;  // TMEM lane quarter this warp may access
       const int r = quarter * 32 + lane;
       const uint32_t lane_off = uint32_t(quarter * 32) << 16;
       const int p = it.p0[x] + r;
       const int p_first = it.p0[x], p_last = it.p0[x] + it.n_rows[x] - 1;
       const float sl2 = a.scale_log2;
+      const int bar_id = 1 + x;
+      float* xch = xbuf + x * 6 * kTile;  // [parity][half][row] row maxima, then [half][row] row sums
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
-      // The page descriptors of tile j + 1 are fetched while tile j is processed.
-      auto fetch_descs = [&](int j, PageDesc& d0, PageDesc& d1) {
-        const int t = tile_of(j);
-        d0 = a.pages[hd.vpage_begin + 2 * t];
-        d1 = a.pages[hd.vpage_begin + min(2 * t + 1, hd.n_vpages - 1)];
+      PageDesc nx{};
+      auto fetch_desc = [&](int j, PageDesc& d) {
+        const int vp = 2 * tile_of(j) + h;
+        d = vp < hd.n_vpages ? a.pages[hd.vpage_begin + vp] : PageDesc{0, 0, 0, 0};
       };
-      PageDesc nx0{}, nx1{};
-      if (n > 0) fetch_descs(0, nx0, nx1);
+      if (n > 0) fetch_desc(0, nx);
       for (int j = 0; j < n; ++j) {
-        const int t = tile_of(j);
-        const bool have1 = 2 * t + 1 < hd.n_vpages;
-        const PageDesc pg0 = nx0;
-        const PageDesc pg1 = have1 ? nx1 : PageDesc{0, 0, 0, 0};
-        if (j + 1 < n) fetch_descs(j + 1, nx0, nx1);
-        const bool full = page_fully_visible(pg0, true, hd, p_first, p_last) &&
-                          page_fully_visible(pg1, have1, hd, p_first, p_last);
-        // tcgen05.ld / st are warp-collective (.sync.aligned): every branch that
-        // guards one is taken by the whole warp, so wait outcomes are voted.
-        if (!__all_sync(kFull, mbar_wait(&bars->s_full[x], j & 1))) {
+        const bool have = 2 * tile_of(j) + h < hd.n_vpages;
+        const PageDesc pg = nx;
+        if (j + 1 < n) fetch_desc(j + 1, nx);
+        const bool full = page_fully_visible(pg, have, hd, p_first, p_last);
+        // tcgen05.ld / st are warp-collective: the wait outcome is voted per warp,
+        // then across the tile's eight warps at the exchange barrier below.
+        const bool got = __all_sync(kFull, mbar_wait(&bars->s_full[x], j & 1));
+        // pass 1: this half's row maximum (S stays in TMEM), one 32-column chunk at a time
+        int h1 = 64, l2 = 0, h2 = 0;
+        if (!full) visible_slots(pg, have, hd, p, h1, l2, h2);
+        auto mask32 = [&](float (&w)[32], int c) {  // chunk c: page slots [32 c, 32 c + 32)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int t = 32 * c + e;
+            if (!(t < h1 || (t >= l2 && t < h2))) w[e] = -INFINITY;
+          }
+        };
+        float mx = -INFINITY;
+        if (got) {
+          tc::fence_after_sync();
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float w[32];
+            tc::tmem_ld32(t_s(x) + lane_off + 64 * h + 32 * c, w);
+            tc::tmem_wait_ld();
+            if (!full) mask32(w, c);
+            float m4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m4[i] = fmax3(w[i], w[i + 4], mx);
+#pragma unroll
+            for (int e = 8; e < 32; e += 8)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) m4[i] = fmax3(m4[i], w[e + i], w[e + 4 + i]);
+            mx = fmax3(fmax3(m4[0], m4[1], m4[2]), m4[3], mx);
+          }
+        }
+        xch[(j & 1) * 2 * kTile + h * kTile + r] = mx;
+        if (!bar_red_and(bar_id, 8 * 32, got)) {
           fail(kDevTimeoutMma);
           ok = false;
           break;
         }
-        tc::fence_after_sync();
-        // Visible slots of this row in the tile's two pages (boundary tiles only).
-        int h1a = 64, l2a = 0, h2a = 0, h1b = 64, l2b = 0, h2b = 0;
-        if (!full) {
-          visible_slots(pg0, true, hd, p, h1a, l2a, h2a);
-          visible_slots(pg1, have1, hd, p, h1b, l2b, h2b);
-        }
-        auto mask32 = [&](float (&v)[32], int chunk) {  // chunk c covers columns [32 c, 32 c + 32)
-          const int h1 = chunk < 2 ? h1a : h1b, l2 = chunk < 2 ? l2a : l2b, h2 = chunk < 2 ? h2a : h2b;
-          const int c0 = (chunk & 1) * 32;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c = c0 + e;
-            if (!(c < h1 || (c >= l2 && c < h2))) v[e] = -INFINITY;
-          }
-        };
-        // pass 1: the row maximum (S stays in TMEM).  The second pair of loads is
-        // in flight while the first pair is reduced.
-        float mx[4];
-        {
-          float va[32], vb[32], vc[32], vd[32];
-          tc::tmem_ld32(t_s(x) + lane_off, va);
-          tc::tmem_ld32(t_s(x) + lane_off + 32, vb);
-          tc::tmem_wait_ld();
-          tc::tmem_ld32(t_s(x) + lane_off + 64, vc);
-          tc::tmem_ld32(t_s(x) + lane_off + 96, vd);
-          if (!full) {
-            mask32(va, 0);
-            mask32(vb, 1);
-          }
-#pragma unroll
-          for (int i = 0; i < 4; ++i) mx[i] = fmax3(va[i], vb[i], -INFINITY);
-#pragma unroll
-          for (int e = 4; e < 32; ++e) mx[e & 3] = fmax3(mx[e & 3], va[e], vb[e]);
-          tc::tmem_wait_ld();
-          if (!full) {
-            mask32(vc, 2);
-            mask32(vd, 3);
-          }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx[e & 3] = fmax3(mx[e & 3], vc[e], vd[e]);
-        }
-        // pass 2's first chunk loads while the maximum is finished
-        float vbuf[2][32];
-        tc::tmem_ld32(t_s(x) + lane_off, vbuf[0]);
-        const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), mx[3], -INFINITY);
+        const float mt = fmaxf(mx, xch[(j & 1) * 2 * kTile + (1 - h) * kTile + r]);
         const float mts = mt * sl2;
         float alpha = 1.f;
         bool need = false;
@@ -341,37 +333,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           need = m_run != -INFINITY;
           m_run = mts;
         }
-        // O_x is stable here: the commit behind s_full also covered P_x(j-1) V.
-        // The decision is per row; the TMEM round trip runs for the whole warp.
-        if (__any_sync(kFull, need)) {
-          const float f = need ? alpha : 1.f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tc::tmem_ld32(t_o(x) + lane_off + c * 32, o);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= f;
-            tc::tmem_st32(t_o(x) + lane_off + c * 32, o);
-          }
-        }
-        // pass 2: P = 2^(s - m) in bf16, written over S columns already consumed:
-        // chunk c of S (columns [32 c, 32 c + 32)) becomes P columns [16 c, 16 c + 16).
-        // Chunk c + 1 is loading while chunk c is exponentiated; one pair in four
-        // takes its 2^x on the FMA pipe so that the SFU is not the bottleneck.
+        // pass 2: P = 2^(s - m) in bf16.  This half's page (columns [64 h, 64 h + 64))
+        // becomes P columns [64 h, 64 h + 32), over its own scores already read; one
+        // pair in kPolyPeriod takes its 2^x on the FMA pipe.
         const float base = m_run == -INFINITY ? 0.f : m_run;
         const uint64_t scale2 = f2_pack(sl2, sl2), nbase2 = f2_pack(-base, -base);
         uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-        tc::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) {
-          float (&v)[32] = vbuf[c & 1];
-          if (c + 1 < kTile / 32) tc::tmem_ld32(t_s(x) + lane_off + (c + 1) * 32, vbuf[(c + 1) & 1]);
-          if (!full) mask32(v, c);
+        for (int c = 0; c < 2; ++c) {
+          float w[32];
+          tc::tmem_ld32(t_s(x) + lane_off + 64 * h + 32 * c, w);
+          tc::tmem_wait_ld();
+          if (!full) mask32(w, c);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const uint64_t x2 = f2_fma(f2_pack(v[2 * e], v[2 * e + 1]), scale2, nbase2);
+            const uint64_t x2 = f2_fma(f2_pack(w[2 * e], w[2 * e + 1]), scale2, nbase2);
             float e0, e1;
             if (kPolyPeriod > 0 && (e % (kPolyPeriod > 0 ? kPolyPeriod : 1)) == kPolyPeriod - 1) {
               exp2_poly_pair(x2, e0, e1);
@@ -383,30 +360,48 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             sum2[e & 1] = f2_add(sum2[e & 1], f2_pack(e0, e1));
             pk[e] = pack_bf16x2(e0, e1);
           }
-          tc::tmem_st16(t_s(x) + lane_off + c * 16, pk);
-          if (c + 1 < kTile / 32) tc::tmem_wait_ld();
+          tc::tmem_st16(t_s(x) + lane_off + 64 * h + 16 * c, pk);
         }
         float s0, s1, s2, s3;
         f2_unpack(sum2[0], s0, s1);
         f2_unpack(sum2[1], s2, s3);
         l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
+        // O_x is stable here: the commit behind s_full also covered P_x(j-1) V, and
+        // P_x(j) V is issued only after this thread arrives on p_full.  This half
+        // rescales its half of the row's O columns (after P, when the scores'
+        // registers are free).
+        if (__any_sync(kFull, need)) {
+          const float f = need ? alpha : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            float o[32];
+            tc::tmem_ld32(t_o(x) + lane_off + h * (D / 2) + c * 32, o);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= f;
+            tc::tmem_st32(t_o(x) + lane_off + h * (D / 2) + c * 32, o);
+          }
+        }
         tc::tmem_wait_st();
         tc::fence_before_sync();
         mbar_arrive(&bars->p_full[x]);
       }
       // ------------------------------ epilogue ------------------------------
-      bool go = ok && n > 0 && mbar_wait(&bars->o_done, 0);
-      go = __all_sync(kFull, go && !*abort_flag);
+      // The row sum is the two halves' sums; the barrier also votes on the O wait.
+      xch[4 * kTile + h * kTile + r] = l_run;
+      const bool got = ok && n > 0 && mbar_wait(&bars->o_done, 0);
+      const bool go = bar_red_and(bar_id, 8 * 32, got && !*abort_flag);
       if (go) {
         tc::fence_after_sync();
+        const float l_tot = xch[4 * kTile + r] + xch[5 * kTile + r];
         const bool row_ok = r < it.n_rows[x];
-        const float inv_l = 1.f / l_run;
-        __nv_bfloat16* orow =
-            static_cast<__nv_bfloat16*>(a.out) + (int64_t(it.q_row[x] + r) * a.num_q_heads + it.qh[x]) * D;
+        const float inv_l = 1.f / l_tot;
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) +
+                              (int64_t(it.q_row[x] + r) * a.num_q_heads + it.qh[x]) * D + h * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           float o[32];
-          tc::tmem_ld32(t_o(x) + lane_off + c * 32, o);
+          tc::tmem_ld32(t_o(x) + lane_off + h * (D / 2) + c * 32, o);
           tc::tmem_wait_ld();
           if (row_ok) {
             uint32_t w[16];
@@ -417,8 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
           }
         }
-        if (row_ok && a.lse)
-          a.lse[int64_t(it.q_row[x] + r) * a.num_q_heads + it.qh[x]] = (m_run + log2f(l_run)) * kLn2;
+        if (h == 0 && row_ok && a.lse)
+          a.lse[int64_t(it.q_row[x] + r) * a.num_q_heads + it.qh[x]] = (m_run + log2f(l_tot)) * kLn2;
       } else if (ok && n > 0) {
         fail(kDevTimeoutMma);
       }
