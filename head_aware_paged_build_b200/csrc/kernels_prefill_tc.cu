@@ -170,9 +170,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const uint8_t* kpool = static_cast<const uint8_t*>(a.kpool);
       const uint8_t* vpool = static_cast<const uint8_t*>(a.vpool);
       mbar_arrive_expect_tx(&bars->q, (two ? 2 : 1) * Sm::kQ);
-      for (int x = 0; x < (two ? 2 : 1); ++x)
-        for (int h = 0; h < D / 64; ++h)
-          tc::tma_load_3d(q_s + x * Sm::kQ + h * 16384, &qmap, h * 64, it.qh[x], it.q_row[x], &bars->q);
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+        if (x == 0 || two)
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h)
+            tc::tma_load_3d(q_s + x * Sm::kQ + h * 16384, &qmap, h * 64, it.qh[x], it.q_row[x], &bars->q);
       int issued = 0;
       for (int j = 0; j < n && !*abort_flag; ++j) {
         const int st = j % NS;
@@ -268,8 +271,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const int quarter = warp & 3;  // TMEM lane quarter this warp may access
       const int r = quarter * 32 + lane;
       const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-      const int p = it.p0[x] + r;
-      const int p_first = it.p0[x], p_last = it.p0[x] + it.n_rows[x] - 1;
+      // this tile's fields by select, not by index: the item stays in registers
+      const int p0x = x ? it.p0[1] : it.p0[0], rows_x = x ? it.n_rows[1] : it.n_rows[0];
+      const int qrow_x = x ? it.q_row[1] : it.q_row[0], qh_x = x ? it.qh[1] : it.qh[0];
+      const int p = p0x + r;
+      const int p_first = p0x, p_last = p0x + rows_x - 1;
       const float sl2 = a.scale_log2;
       const int bar_id = 1 + x;
       float* xch = xbuf + x * 6 * kTile;  // [parity][half][row] row maxima, then [half][row] row sums
@@ -394,10 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       if (go) {
         tc::fence_after_sync();
         const float l_tot = xch[4 * kTile + r] + xch[5 * kTile + r];
-        const bool row_ok = r < it.n_rows[x];
+        const bool row_ok = r < rows_x;
         const float inv_l = 1.f / l_tot;
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) +
-                              (int64_t(it.q_row[x] + r) * a.num_q_heads + it.qh[x]) * D + h * (D / 2);
+                              (int64_t(qrow_x + r) * a.num_q_heads + qh_x) * D + h * (D / 2);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           float o[32];
@@ -413,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           }
         }
         if (h == 0 && row_ok && a.lse)
-          a.lse[int64_t(it.q_row[x] + r) * a.num_q_heads + it.qh[x]] = (m_run + log2f(l_tot)) * kLn2;
+          a.lse[int64_t(qrow_x + r) * a.num_q_heads + qh_x] = (m_run + log2f(l_tot)) * kLn2;
       } else if (ok && n > 0) {
         fail(kDevTimeoutMma);
       }
