@@ -53,7 +53,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kFull = 0xffffffffu;
 // One exponent pair in every kPolyPeriod is computed on the FMA pipe (0: none).
 #ifndef SP_EXP2_POLY_PERIOD
-#define SP_EXP2_POLY_PERIOD 4
+#define SP_EXP2_POLY_PERIOD 16
 #endif
 constexpr int kPolyPeriod = SP_EXP2_POLY_PERIOD;
 
