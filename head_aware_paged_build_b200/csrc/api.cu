@@ -135,6 +135,7 @@ sp_status segpaged_attention(const sp_plan* plan, const void* d_table, const voi
     L.num_q_heads = plan->prob.num_q_heads;
     L.bf16 = plan->prob.dtype == SP_BF16;
     L.page_bytes = plan->sizes.page_bytes;
+    L.pool_pages = plan->sizes.pool_pages;
     L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
     L.scale_log2 = plan->fp8 ? scale_log2 * plan->k_scale : scale_log2;
     L.fp8 = plan->fp8;
@@ -156,6 +157,7 @@ sp_status segpaged_attention(const sp_plan* plan, const void* d_table, const voi
     L.total_rows = int32_t(plan->sizes.num_queries);
     L.bf16 = plan->prob.dtype == SP_BF16;
     L.page_bytes = plan->sizes.page_bytes;
+    L.pool_pages = plan->sizes.pool_pages;
     L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
     L.scale_log2 = scale_log2;
     L.status = status;
@@ -193,6 +195,7 @@ sp_status segpaged_decode_append(const sp_plan* plan, void* d_table, const void*
   L.stride_seq = stride_seq;
   L.stride_head = stride_head;
   L.page_bytes = plan->sizes.page_bytes;
+  L.pool_pages = plan->sizes.pool_pages;
   L.k_new = k_new, L.v_new = v_new, L.kpool = k_pool, L.vpool = v_pool;
   L.status = static_cast<int32_t*>(workspace);
   const cudaError_t e = launch_append(L, static_cast<cudaStream_t>(stream));

@@ -38,6 +38,7 @@ struct DecodeLaunch {
   int32_t D, P, group, num_q_heads;
   bool bf16;
   int64_t page_bytes;
+  int64_t pool_pages;  // pages a pool must hold; a table page id outside [0, pool_pages) is reported
   const void* kpool;
   const void* vpool;
   const void* q;  // [B, Hq, D]
@@ -60,6 +61,7 @@ struct PrefillLaunch {
   int32_t D, P, group, num_q_heads, total_rows;
   bool bf16;
   int64_t page_bytes;
+  int64_t pool_pages;  // pages a pool must hold; a table page id outside [0, pool_pages) is reported
   const void* kpool;
   const void* vpool;
   const void* q;  // [rows, Hq, D]
@@ -79,6 +81,7 @@ struct AppendLaunch {
   bool fp8;            // E4M3 pages: the new bf16 rows are quantised on the way in
   float k_inv, v_inv;  // 1 / k_scale, 1 / v_scale
   int64_t stride_seq, stride_head, page_bytes;
+  int64_t pool_pages;
   const void* k_new;  // [B, Hkv, D] with the given strides (elements)
   const void* v_new;
   void* kpool;

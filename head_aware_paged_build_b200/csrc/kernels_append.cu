@@ -42,6 +42,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendLaunch a) 
   }
   PageDesc* pg = a.pages + hd->vpage_begin + vp;
   const int64_t phys = pg->phys;
+  if (phys < 0 || phys >= a.pool_pages) {  // corrupted table: report, write nothing
+    if (threadIdx.x == 0) record_error(a.status, kDevBadPage);
+    return;
+  }
   const T* kn = static_cast<const T*>(a.k_new) + int64_t(hd->b) * a.stride_seq + int64_t(hd->kv) * a.stride_head;
   const T* vn = static_cast<const T*>(a.v_new) + int64_t(hd->b) * a.stride_seq + int64_t(hd->kv) * a.stride_head;
   uint8_t* kdst = static_cast<uint8_t*>(a.kpool) + phys * a.page_bytes;

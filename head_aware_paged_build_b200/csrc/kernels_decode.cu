@@ -108,6 +108,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch
             record_error(a.status, kDevTimeoutEmpty);
             good = 0;
           } else {
+            if (pgd.phys < 0 || pgd.phys >= a.pool_pages) {  // corrupted table: report, read nothing
+              record_error(a.status, kDevBadPage);
+              pgd.span = 0;
+            }
             sdesc[s] = pgd;
             uint8_t* kd = stage + s * 2 * PB;
             if (slot_hi(pgd) > slot_lo(pgd)) {
@@ -433,6 +437,10 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(DecodeLaunch a)
     for (int j = 0; j < ACC; ++j) acc[j] = 0.f;
     for (int g = item.vp_begin; g < item.vp_end; ++g) {
       const PageDesc pg = a.pages[g];
+      if (pg.phys < 0 || pg.phys >= a.pool_pages) {  // corrupted table: report, read nothing
+        if (threadIdx.x == 0) record_error(a.status, kDevBadPage);
+        continue;
+      }
       __syncthreads();
       const uint4* ks = reinterpret_cast<const uint4*>(kpool + int64_t(pg.phys) * a.page_bytes);
       const uint4* vs = reinterpret_cast<const uint4*>(vpool + int64_t(pg.phys) * a.page_bytes);

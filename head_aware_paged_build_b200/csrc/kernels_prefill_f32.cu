@@ -51,8 +51,12 @@ __global__ void __launch_bounds__(kRows) prefill_f32_kernel(PrefillLaunch a) {
       __syncthreads();
       for (int j = 0; j < PPT; ++j) {
         const int vp = t * PPT + j;
-        const bool have = vp < hd.n_vpages;
+        bool have = vp < hd.n_vpages;
         const PageDesc pg = have ? a.pages[hd.vpage_begin + vp] : PageDesc{0, 0, 0, 0};
+        if (have && (pg.phys < 0 || pg.phys >= a.pool_pages)) {  // corrupted table: report, read nothing
+          if (threadIdx.x == 0) record_error(a.status, kDevBadPage);
+          have = false;
+        }
         const float* kp = reinterpret_cast<const float*>(kpool + int64_t(pg.phys) * a.page_bytes);
         const float* vpp = reinterpret_cast<const float*>(vpool + int64_t(pg.phys) * a.page_bytes);
         for (int e = threadIdx.x; e < P * D; e += kRows) {

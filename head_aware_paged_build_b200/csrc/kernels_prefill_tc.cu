@@ -186,6 +186,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const int t = tile_of(j);
         const int vp0 = 2 * t, vp1 = (2 * t + 1 < hd.n_vpages) ? 2 * t + 1 : 2 * t;
         const int64_t ph[2] = {a.pages[hd.vpage_begin + vp0].phys, a.pages[hd.vpage_begin + vp1].phys};
+        if (ph[0] < 0 || ph[0] >= a.pool_pages || ph[1] < 0 || ph[1] >= a.pool_pages) {
+          fail(kDevBadPage);  // corrupted table: read nothing; the other roles' bounded waits end the CTA
+          break;
+        }
         uint8_t* k_s = stage_s + st * Sm::kStage;
         uint8_t* v_s = k_s + Sm::kK;
         mbar_arrive_expect_tx(&kv_full[st], Sm::kStage);

@@ -105,6 +105,7 @@ extern "C" sp_status segpaged_attention_decode_noalloc(const sp_plan* plan, cons
   L.num_q_heads = plan->prob.num_q_heads;
   L.bf16 = plan->prob.dtype == SP_BF16;
   L.page_bytes = plan->sizes.page_bytes;
+  L.pool_pages = plan->sizes.pool_pages;
   L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
   L.scale_log2 = scale * 1.4426950408889634f * (plan->fp8 ? plan->k_scale : 1.f);
   L.fp8 = plan->fp8;

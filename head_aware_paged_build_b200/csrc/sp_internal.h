@@ -33,7 +33,7 @@ enum DeviceCode : int32_t {
   kDevTimeoutEmpty = 2,    // the producer gave up waiting for a free stage
   kDevTimeoutMma = 3,      // a wait on a tensor-core commit ran out
   kDevTimeoutSoftmax = 4,  // the MMA issuer gave up waiting for P
-  kDevBadPage = 5,         // a page id outside the pool (debug builds)
+  kDevBadPage = 5,         // a table page id outside [0, pool_pages): nothing read or written there
   kDevAppendFull = 6,      // an append found no reserved page left (ring plans)
 };
 

@@ -285,8 +285,14 @@ SP_API sp_status segpaged_decode_append(const sp_plan* plan, void* d_table, cons
                                         void* workspace, void* stream);
 
 /* Device status word: kernels never trap; a failed device-side check or a
- * bounded wait that ran out records a non-zero code.  read synchronises
- * `stream` and returns the code in *code (0 = no error); clear zeroes it. */
+ * bounded wait that ran out records a non-zero code (the first one sticks):
+ *   1, 2  a wait on a page copy (full / empty stage) ran out
+ *   3     a wait on the tensor cores ran out      4  a wait on the softmax ran out
+ *   5     a page id in the device table lies outside [0, pool_pages): the
+ *         kernel read or wrote nothing there (a corrupted table)
+ *   6     a ring append found no reserved page left (the append was skipped)
+ * read synchronises `stream` and returns the code in *code (0 = no error);
+ * clear zeroes it. */
 SP_API sp_status segpaged_read_device_status(const void* workspace, int32_t* code, void* stream);
 SP_API sp_status segpaged_clear_device_status(void* workspace, void* stream);
 
