@@ -339,7 +339,9 @@ def run_ours(args) -> None:
         "wall_s_timed": round(wall, 3),
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, dec, k, v, qd, args.cpu_seconds)
+        Ld.attention(qd, od, lsed)  # the measured decode's output, checked on the oracle's sample
+        torch.cuda.synchronize()
+        line["cpu_baseline"] = cpu_baseline(wl, dec, k, v, qd, args.cpu_seconds, gpu=(od, lsed))
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -467,14 +469,22 @@ def run_e2e_dense(args, dev, layer, k, v, qd, od, lsed, world) -> dict:
             "path": "pinned host K/V/Q -> build_segpaged_cache -> segpaged_attention (decode) -> host O, LSE"}
 
 
-def oracle_decode_sample(wl, dec, k, v, qd, budget_s: float, max_heads: int | None = None) -> tuple[float, int, int]:
+def oracle_decode_sample(wl, dec, k, v, qd, budget_s: float, max_heads: int | None = None,
+                         gpu: tuple | None = None) -> tuple[float, int, int, dict | None]:
     """Run the CPU oracle on whole (sequence, kv-head) groups until the time budget is spent.
 
-    Returns (seconds spent inside the oracle, visible KV bytes covered, groups done).
+    Returns (seconds spent inside the oracle, visible KV bytes covered, groups done, parity), where
+    parity compares the GPU decode output `gpu` = (out, lse) with the oracle on the same groups
+    (per q-head cosine and max abs error of O, max abs error of LSE), or is None without `gpu`.
     """
+    import numpy as np
+
     import oracle
 
     spent, vis, groups = 0.0, 0, 0
+    cos_min, abs_max, lse_max = 1.0, 0.0, 0.0
+    if gpu is not None:
+        gout, glse = gpu[0].double().cpu().numpy(), gpu[1].double().cpu().numpy()
     order = [(b, kv) for b in range(wl.batch) for kv in range(wl.num_kv_heads)]
     for b, kv in order:
         if spent >= budget_s or (max_heads is not None and groups >= max_heads):
@@ -486,19 +496,28 @@ def oracle_decode_sample(wl, dec, k, v, qd, budget_s: float, max_heads: int | No
         qq = qd[b, kv * wl.group:(kv + 1) * wl.group].double().cpu().numpy()
         t0 = time.perf_counter()
         # the group's q-heads share the kv-head: one call, one query row per q-head (OpenMP over rows)
-        oracle.attention_rows(qq, [L - 1] * wl.group, kk, vv, kind, s, w)
+        o_ref, l_ref = oracle.attention_rows(qq, [L - 1] * wl.group, kk, vv, kind, s, w)
         spent += time.perf_counter() - t0
         vis += int(oracle.stored_mask(kind, s, w, L, L - 1).sum()) * 2 * wl.head_dim * 2
         groups += 1
-    return spent, vis, groups
+        if gpu is not None:
+            for i in range(wl.group):
+                a, r = gout[b, kv * wl.group + i], o_ref[i]
+                cos_min = min(cos_min, float(a @ r / (np.linalg.norm(a) * np.linalg.norm(r))))
+                abs_max = max(abs_max, float(np.max(np.abs(a - r))))
+                lse_max = max(lse_max, abs(float(glse[b, kv * wl.group + i]) - float(l_ref[i])))
+    parity = ({"min_cos": round(cos_min, 7), "max_abs": float(f"{abs_max:.3g}"), "max_lse_abs": float(f"{lse_max:.3g}"),
+               "heads": groups * wl.group, "against": "fp64 oracle, same inputs"} if gpu is not None else None)
+    return spent, vis, groups, parity
 
 
-def cpu_baseline(wl, dec, k, v, qd, budget_s: float) -> dict:
+def cpu_baseline(wl, dec, k, v, qd, budget_s: float, gpu: tuple | None = None) -> dict:
     import oracle
-    spent, vis, groups = oracle_decode_sample(wl, dec, k, v, qd, budget_s)
+    spent, vis, groups, parity = oracle_decode_sample(wl, dec, k, v, qd, budget_s, gpu=gpu)
     return {"value": round(vis / spent / 1e9, 4), "unit": "GB/s", "cores": min(oracle.num_threads(), wl.group),
             "kind": "oracle",
             "seconds": round(spent, 2),
+            "decode_parity": parity,
             "sample": f"decode of {groups} of {wl.batch * wl.num_kv_heads} (sequence, kv-head) groups, "
                       f"all {wl.group} q-heads each (fp64 dense attention with explicit mask)"}
 
@@ -524,7 +543,7 @@ def run_reference(args) -> None:
     spent = vis = 0.0
     t_steps = []
     for _ in range(args.steps):
-        s, b, _ = oracle_decode_sample(wl, dec, k, v, qd, 1e9, max_heads=per_step)
+        s, b, _, _ = oracle_decode_sample(wl, dec, k, v, qd, 1e9, max_heads=per_step)
         spent += s
         vis += b
         t_steps.append(s)
