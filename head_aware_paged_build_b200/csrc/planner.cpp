@@ -28,6 +28,7 @@ sp_status fail(sp_status st, const std::string& msg) {
 namespace {
 
 constexpr int kDefaultDecodeCtas = 2 * 148;
+constexpr int64_t kItemCostPages100 = 200;  // a head start costs as much as two pages (measured)
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -268,13 +269,29 @@ sp_status plan_build(sp_plan& pl) {
   for (int64_t i = 0; i < n_pages; ++i)
     pl.pages[i].phys = int32_t(p.first_page + (p.page_ids ? p.page_ids[i] : i));
 
-  // --- decode: equal page ranges per CTA, cut at head boundaries ------------
+  // --- decode: balanced page ranges per CTA, cut at head boundaries ---------
   int n_slots = 0;
   if (decode) {
     const int64_t G = std::min<int64_t>(p.target_ctas ? p.target_ctas : kDefaultDecodeCtas, n_pages);
+    // A CTA pays for every head it starts (Q load, warp merge, partial publish) on
+    // top of its pages: cut the page list at equal shares of (pages + two pages
+    // per head start), so CTAs that cross a head boundary take fewer pages.
+    // Costs are in hundredths of a page.
+    std::vector<int64_t> cost(n_pages + 1, 0);  // cost of pages [0, i)
+    for (int64_t i = 0; i < n_pages; ++i) {
+      const HeadDesc& hd = pl.heads[pl.pages[i].head];
+      cost[i + 1] = cost[i] + kItemCostPages100 * (i == hd.vpage_begin ? 1 : 0) + 100;
+    }
+    std::vector<int64_t> cut(G + 1, n_pages);
+    for (int64_t c = 0, i = 0; c <= G; ++c) {
+      const int64_t total = cost[n_pages];  // ceil(total * c / G) without overflow
+      const int64_t want = total / G * c + ((total % G) * c + G - 1) / G;
+      while (i < n_pages && cost[i] < want) ++i;
+      cut[c] = c == G ? n_pages : i;
+    }
     pl.decode_cta_begin.assign(1, 0);
     for (int64_t c = 0; c < G; ++c) {
-      int64_t lo = c * n_pages / G, hi = (c + 1) * n_pages / G;
+      int64_t lo = cut[c], hi = cut[c + 1];
       while (lo < hi) {
         const int h = pl.pages[lo].head;
         const int64_t end = std::min<int64_t>(hi, pl.heads[h].vpage_begin + pl.heads[h].n_vpages);
