@@ -108,8 +108,10 @@ typedef struct {
  *   page_ids    NULL, or [num_pages] distinct non-negative ids (logical page i
  *               goes to physical page first_page + page_ids[i]); num_pages is
  *               reported by segpaged_plan_sizes of a plan made with NULL
- *   target_ctas decode work is split into this many equal page ranges; 0 picks
- *               2 x 148 (two CTAs on each B200 SM)
+ *   target_ctas decode work is split into this many CTAs (at most one per
+ *               page): contiguous ranges of the heads' concatenated page
+ *               lists, balanced on pages plus a two-page cost for each head
+ *               a range starts; 0 picks 2 x 148 (two CTAs on each B200 SM)
  *   append_capacity  SP_FLAG_RING plans: extra tokens per sequence that
  *               segpaged_decode_append may add (GLOBAL heads reserve pages for
  *               them); must be 0 otherwise
