@@ -507,9 +507,9 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(DecodeLaunch a)
 }
 
 // ---------------------------------------------------------------------------
-// Combine: one warp per (split head, q-head of its group).
+// Combine (fp32 path): one warp per (split head, q-head of its group).
 // ---------------------------------------------------------------------------
-template <typename TOut, int D, bool FAST>
+template <int D>
 __global__ void __launch_bounds__(128) combine_kernel(DecodeLaunch a) {
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const int G = a.group;
@@ -528,7 +528,7 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeLaunch a) {
   for (int i = 0; i < ci.n_slots; ++i) {
     const float* slot = a.partial + int64_t(ci.slot_begin + i) * partial_slot_floats(G, D);
     const float mi = slot[G * D + row * 2];
-    const float f = FAST ? fast_exp2(mi - base) : exp2f(mi - base);
+    const float f = exp2f(mi - base);
     L += f * slot[G * D + row * 2 + 1];
 #pragma unroll
     for (int j = 0; j < D / 32; ++j) acc[j] += f * slot[row * D + j * 32 + lane];
@@ -536,13 +536,7 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeLaunch a) {
   const int qh = hd.kv * G + row;
   const int64_t o_idx = (int64_t(hd.q_row0) * a.num_q_heads + qh) * D;
 #pragma unroll
-  for (int j = 0; j < D / 32; ++j) {
-    const float v = acc[j] / L;
-    if constexpr (sizeof(TOut) == 2)
-      static_cast<__nv_bfloat16*>(a.out)[o_idx + j * 32 + lane] = __float2bfloat16_rn(v);
-    else
-      static_cast<float*>(a.out)[o_idx + j * 32 + lane] = v;
-  }
+  for (int j = 0; j < D / 32; ++j) static_cast<float*>(a.out)[o_idx + j * 32 + lane] = acc[j] / L;
   if (lane == 0 && a.lse) a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh] = (M + log2f(L)) * kLn2;
 }
 
@@ -569,7 +563,7 @@ cudaError_t launch_f32(const DecodeLaunch& a, cudaStream_t s) {
   kern<<<a.n_ctas, kF32Threads, bytes, s>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess || a.n_combine == 0) return e;
-  combine_kernel<float, D, false><<<(a.n_combine * a.group + 3) / 4, 128, 0, s>>>(a);
+  combine_kernel<D><<<(a.n_combine * a.group + 3) / 4, 128, 0, s>>>(a);
   return cudaGetLastError();
 }
 
