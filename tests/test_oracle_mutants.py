@@ -28,6 +28,14 @@ MUTANTS = {
     "lse_without_max": ("lse[r] = m + log(denom);", "lse[r] = log(denom);"),
     "dense_treated_as_local": ("if (kind != ORACLE_LOCAL) return 1;", "if (kind == ORACLE_GLOBAL) return 1;"),
     "stored_only_last_query": ("for (int64_t p = q0; p < L && !keep; ++p)", "for (int64_t p = L - 1; p < L && !keep; ++p)"),
+    # FP8 E4M3 encoder / decoder
+    "e4m3_bias_8": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "e4m3_subnormal_step": ("ldexp((double)m, -9)", "ldexp((double)m, -10)"),
+    "e4m3_ties_up": ("(down < up || (down == up && ((lo - 1) & 1) == 0))", "(down < up)"),
+    "e4m3_saturates_to_nan": ("if (a >= 448.0) return sgn | 0x7E;", "if (a >= 448.0) return sgn | 0x7F;"),
+    "e4m3_inv_scale_dropped": ("oracle_e4m3_encode_f32(x[i] * inv_scale)", "oracle_e4m3_encode_f32(x[i])"),
+    "e4m3_decode_scale_dropped": ("values[i] = oracle_e4m3_value(codes[i]) * scale;",
+                                  "values[i] = oracle_e4m3_value(codes[i]);"),
 }
 
 

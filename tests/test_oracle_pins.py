@@ -246,6 +246,8 @@ def test_e4m3_codes_fixed_by_the_format():
     assert oracle.e4m3_encode(vals, 1.0).tolist() == want
     back = oracle.e4m3_decode(np.array(want, np.uint8), 1.0)
     np.testing.assert_array_equal(back, [0, 1, -1, 448, 448, -448, 2 ** -9, 2 ** -6, 1.125, 0.875 * 2 ** -6, 240, 256])
+    # a decoded value is the code's value times the scale: 1.0 (0x38) at scale 0.25, -448 (0xFE) at 2
+    np.testing.assert_array_equal(oracle.e4m3_decode(np.array([0x38, 0xFE], np.uint8), 0.25), [0.25, -112.0])
 
 
 def test_e4m3_rounds_to_nearest_even_and_saturates():
