@@ -5,6 +5,7 @@
 // fallback: a dtype / shape without a kernel returns SP_ERR_UNSUPPORTED.
 #include <cmath>
 #include <cstdint>
+#include <limits>
 #include <string>
 
 #include "kernels.h"
@@ -91,6 +92,51 @@ sp_status build_segpaged_cache(const sp_plan* plan, const void* d_table, const v
                                void* v_pool, void* stream) {
   return sp::pack_common(plan, d_table, k_dense, v_dense, k_pool, v_pool, false, stride_seq, stride_head,
                          stride_tok, stream);
+}
+
+sp_status build_segpaged_cache_layers(int32_t n_layers, const sp_plan* const* plans, const void* const* d_tables,
+                                      const void* const* k_dense, const void* const* v_dense, int64_t stride_seq,
+                                      int64_t stride_head, int64_t stride_tok, void* k_pool, void* v_pool,
+                                      void* stream) {
+  using namespace sp;
+  if (n_layers < 1 || n_layers > kMaxPackLayers)
+    return fail(SP_ERR_INVALID_ARG, "n_layers must be in [1, " + std::to_string(kMaxPackLayers) + "]");
+  if (!plans || !d_tables || !k_dense || !v_dense) return fail(SP_ERR_INVALID_ARG, "arrays must be non-NULL");
+  if (!k_pool || !v_pool || !aligned(k_pool, 16) || !aligned(v_pool, 16))
+    return fail(SP_ERR_INVALID_ARG, "pools must be non-NULL and 16-byte aligned");
+  const sp_plan* p0 = plans[0];
+  if (!p0) return fail(SP_ERR_INVALID_ARG, "plans[0] is NULL");
+  const int64_t eb = p0->elem_bytes;
+  if (stride_head < 0 || stride_tok < 0 || (stride_seq < 0 && stride_seq != SP_VARLEN))
+    return fail(SP_ERR_INVALID_ARG, "strides must be >= 0 (stride_seq may be SP_VARLEN)");
+  if ((stride_head * eb) % 16 || (stride_tok * eb) % 16 || (stride_seq > 0 && (stride_seq * eb) % 16))
+    return fail(SP_ERR_INVALID_ARG, "strides must give 16-byte aligned rows");
+  PackLayersArgs la{};
+  la.n_layers = n_layers;
+  la.stride_seq = stride_seq, la.stride_head = stride_head, la.stride_tok = stride_tok;
+  la.page_bytes = p0->sizes.page_bytes;
+  int64_t total = 0;
+  for (int32_t i = 0; i < n_layers; ++i) {
+    const sp_plan* p = plans[i];
+    sp_status st = check_table(p, d_tables[i]);
+    if (st != SP_OK) return st;
+    if (p->prob.dtype != p0->prob.dtype || p->prob.head_dim != p0->prob.head_dim ||
+        p->prob.page_size != p0->prob.page_size || p->fp8 != p0->fp8)
+      return fail(SP_ERR_INVALID_ARG, "every layer needs the same dtype, head_dim, page_size and page type");
+    if (!k_dense[i] || !v_dense[i] || !aligned(k_dense[i], 16) || !aligned(v_dense[i], 16))
+      return fail(SP_ERR_INVALID_ARG, "dense K/V pointers must be non-NULL and 16-byte aligned");
+    la.page_begin[i] = int32_t(total);
+    la.heads[i] = section<HeadDesc>(d_tables[i], p->hdr.off_heads);
+    la.pages[i] = section<PageDesc>(d_tables[i], p->hdr.off_pages);
+    la.kd[i] = k_dense[i], la.vd[i] = v_dense[i];
+    la.k_inv[i] = 1.0f / p->k_scale, la.v_inv[i] = 1.0f / p->v_scale;
+    total += p->hdr.n_vpages;
+    if (total > std::numeric_limits<int32_t>::max()) return fail(SP_ERR_UNSUPPORTED, "more than 2^31 pages");
+  }
+  la.page_begin[n_layers] = int32_t(total);
+  const cudaError_t e = launch_pack_layers(la, p0->prob.dtype == SP_BF16, p0->fp8, p0->prob.head_dim,
+                                           p0->prob.page_size, k_pool, v_pool, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SP_OK : cuda_fail(e, "build_segpaged_cache_layers launch");
 }
 
 sp_status segpaged_gather(const sp_plan* plan, const void* d_table, const void* k_pool, const void* v_pool,

@@ -28,6 +28,21 @@ struct PackLaunch {
 };
 void launch_pack(const PackLaunch& L, cudaStream_t s);
 
+// Pack of several layers in one launch (kernel parameter, passed by value).
+constexpr int kMaxPackLayers = 128;
+struct PackLayersArgs {
+  int32_t n_layers;
+  int32_t page_begin[kMaxPackLayers + 1];  // prefix sums of the layers' page counts
+  const HeadDesc* heads[kMaxPackLayers];
+  const PageDesc* pages[kMaxPackLayers];
+  const void* kd[kMaxPackLayers];
+  const void* vd[kMaxPackLayers];
+  float k_inv[kMaxPackLayers], v_inv[kMaxPackLayers];  // E4M3 pages: 1 / scale per layer
+  int64_t stride_seq, stride_head, stride_tok, page_bytes;
+};
+cudaError_t launch_pack_layers(const PackLayersArgs& la, bool bf16, bool fp8, int D, int P, void* kpool, void* vpool,
+                               cudaStream_t s);
+
 struct DecodeLaunch {
   const HeadDesc* heads;
   const PageDesc* pages;

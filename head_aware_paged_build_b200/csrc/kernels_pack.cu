@@ -48,16 +48,16 @@ __device__ __forceinline__ int64_t vpage_chunk(int i, int c16, int P) {
 }
 
 template <typename T, int D, int P>
-__global__ void __launch_bounds__(kPackThreads) pack_kernel(PackArgs a, const T* __restrict__ kd,
-                                                            const T* __restrict__ vd, uint8_t* __restrict__ kpool,
-                                                            uint8_t* __restrict__ vpool) {
+__device__ __forceinline__ void pack_page(const PackArgs& a, int page, const T* __restrict__ kd,
+                                          const T* __restrict__ vd, uint8_t* __restrict__ kpool,
+                                          uint8_t* __restrict__ vpool) {
   constexpr int CR = D * int(sizeof(T)) / 16;   // 16-byte chunks per dense row
   constexpr int EPC = 16 / int(sizeof(T));      // elements per chunk
   constexpr int PW = vstage_pitch_words<T>(D);  // staging pitch (32-bit words)
   constexpr int VR = P / EPC;                   // chunks per transposed V row
   __shared__ uint32_t stage[P * PW];
 
-  const PageDesc pg = a.pages[blockIdx.x];
+  const PageDesc pg = a.pages[page];
   const HeadDesc hd = a.heads[pg.head];
   const int64_t base = (a.stride_seq >= 0 ? int64_t(hd.b) * a.stride_seq : int64_t(hd.ctx_row0) * a.stride_tok) +
                        int64_t(hd.kv) * a.stride_head;
@@ -86,6 +86,13 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(PackArgs a, const T*
     for (int e = 0; e < EPC; ++e) vals[e] = st[(c * EPC + e) * (PW * 4 / int(sizeof(T))) + i];
     *reinterpret_cast<uint4*>(vdst + vpage_chunk<T>(i, c, P)) = *reinterpret_cast<const uint4*>(vals);
   }
+}
+
+template <typename T, int D, int P>
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(PackArgs a, const T* __restrict__ kd,
+                                                            const T* __restrict__ vd, uint8_t* __restrict__ kpool,
+                                                            uint8_t* __restrict__ vpool) {
+  pack_page<T, D, P>(a, blockIdx.x, kd, vd, kpool, vpool);
 }
 
 template <typename T, int D, int P>
@@ -140,16 +147,15 @@ __device__ __forceinline__ uint32_t quant4(uint32_t w0, uint32_t w1, float inv) 
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPackThreads) pack_fp8_kernel(PackArgs a, float k_inv, float v_inv,
-                                                                const __nv_bfloat16* __restrict__ kd,
-                                                                const __nv_bfloat16* __restrict__ vd,
-                                                                uint8_t* __restrict__ kpool,
-                                                                uint8_t* __restrict__ vpool) {
+__device__ __forceinline__ void pack_fp8_page(const PackArgs& a, int page, float k_inv, float v_inv,
+                                              const __nv_bfloat16* __restrict__ kd,
+                                              const __nv_bfloat16* __restrict__ vd, uint8_t* __restrict__ kpool,
+                                              uint8_t* __restrict__ vpool) {
   constexpr int P = 64;
   constexpr int CR = D * 2 / 16;                            // 16-byte bf16 chunks per dense row
   constexpr int PW = vstage_pitch_words<__nv_bfloat16>(D);  // staging pitch (32-bit words)
   __shared__ uint32_t stage[P * PW];
-  const PageDesc pg = a.pages[blockIdx.x];
+  const PageDesc pg = a.pages[page];
   const HeadDesc hd = a.heads[pg.head];
   const int64_t base = (a.stride_seq >= 0 ? int64_t(hd.b) * a.stride_seq : int64_t(hd.ctx_row0) * a.stride_tok) +
                        int64_t(hd.kv) * a.stride_head;
@@ -182,6 +188,35 @@ __global__ void __launch_bounds__(kPackThreads) pack_fp8_kernel(PackArgs a, floa
     }
     *reinterpret_cast<uint4*>(vdst + fp8_vpage_offset(i, c * 16)) = make_uint4(q[0], q[1], q[2], q[3]);
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPackThreads) pack_fp8_kernel(PackArgs a, float k_inv, float v_inv,
+                                                                const __nv_bfloat16* __restrict__ kd,
+                                                                const __nv_bfloat16* __restrict__ vd,
+                                                                uint8_t* __restrict__ kpool,
+                                                                uint8_t* __restrict__ vpool) {
+  pack_fp8_page<D>(a, blockIdx.x, k_inv, v_inv, kd, vd, kpool, vpool);
+}
+
+// Several layers in one launch: CTA i packs page i of the layers' concatenated
+// page lists; the layer is found by a binary search of the page offsets.
+template <typename T, int D, int P, bool FP8>
+__global__ void __launch_bounds__(kPackThreads) pack_layers_kernel(PackLayersArgs la, uint8_t* __restrict__ kpool,
+                                                                   uint8_t* __restrict__ vpool) {
+  int lo = 0, hi = la.n_layers - 1;
+  while (lo < hi) {  // last layer whose first page <= blockIdx.x
+    const int mid = (lo + hi + 1) / 2;
+    if (la.page_begin[mid] <= int(blockIdx.x)) lo = mid;
+    else hi = mid - 1;
+  }
+  const PackArgs a{la.heads[lo], la.pages[lo], la.stride_seq, la.stride_head, la.stride_tok, la.page_bytes};
+  const int page = int(blockIdx.x) - la.page_begin[lo];
+  if constexpr (FP8)
+    pack_fp8_page<D>(a, page, la.k_inv[lo], la.v_inv[lo], static_cast<const __nv_bfloat16*>(la.kd[lo]),
+                     static_cast<const __nv_bfloat16*>(la.vd[lo]), kpool, vpool);
+  else
+    pack_page<T, D, P>(a, page, static_cast<const T*>(la.kd[lo]), static_cast<const T*>(la.vd[lo]), kpool, vpool);
 }
 
 template <int D>
@@ -249,6 +284,28 @@ void launch_pack_t(const PackLaunch& L, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t launch_pack_layers(const PackLayersArgs& la, bool bf16, bool fp8, int D, int P, void* kpool, void* vpool,
+                               cudaStream_t s) {
+  const int n = la.page_begin[la.n_layers];
+  if (n == 0) return cudaSuccess;
+  uint8_t* kp = static_cast<uint8_t*>(kpool);
+  uint8_t* vp = static_cast<uint8_t*>(vpool);
+  if (fp8) {
+    if (D == 128) pack_layers_kernel<__nv_bfloat16, 128, 64, true><<<n, kPackThreads, 0, s>>>(la, kp, vp);
+    else pack_layers_kernel<__nv_bfloat16, 64, 64, true><<<n, kPackThreads, 0, s>>>(la, kp, vp);
+  } else if (bf16) {
+    if (D == 128) pack_layers_kernel<__nv_bfloat16, 128, 64, false><<<n, kPackThreads, 0, s>>>(la, kp, vp);
+    else pack_layers_kernel<__nv_bfloat16, 64, 64, false><<<n, kPackThreads, 0, s>>>(la, kp, vp);
+  } else if (P == 16) {
+    if (D == 128) pack_layers_kernel<float, 128, 16, false><<<n, kPackThreads, 0, s>>>(la, kp, vp);
+    else pack_layers_kernel<float, 64, 16, false><<<n, kPackThreads, 0, s>>>(la, kp, vp);
+  } else {
+    if (D == 128) pack_layers_kernel<float, 128, 64, false><<<n, kPackThreads, 0, s>>>(la, kp, vp);
+    else pack_layers_kernel<float, 64, 64, false><<<n, kPackThreads, 0, s>>>(la, kp, vp);
+  }
+  return cudaGetLastError();
+}
 
 void launch_pack(const PackLaunch& L, cudaStream_t s) {
   if (L.n_pages == 0) return;

@@ -117,6 +117,27 @@ def layer_for(prob, device="cuda", flags: int = 0, **kw) -> SegPagedLayer:
                          q_start=prob.q_starts, policy=wl.policy, device=device, flags=flags, **kw)
 
 
+def build_layers(layers: Sequence[SegPagedLayer], k_dense: Sequence[torch.Tensor], v_dense: Sequence[torch.Tensor],
+                 varlen: bool = False, stream=None) -> None:
+    """Pack several layers that share one pair of pools with a single launch.
+
+    ``layers[i]`` packs ``k_dense[i]`` / ``v_dense[i]`` (all with the same strides); the
+    layers must hold the same pools (``pools=`` at construction, distinct ``first_page``).
+    """
+    k0 = k_dense[0]
+    if varlen:
+        ss, sh, st = S.SP_VARLEN, k0.stride(1), k0.stride(0)
+    else:
+        ss, sh, st = k0.stride(0), k0.stride(1), k0.stride(2)
+    for lay, k, v in zip(layers, k_dense, v_dense):
+        assert k.stride() == k0.stride() and v.stride() == k0.stride() and k0.stride(-1) == 1
+        assert lay.k_pool.data_ptr() == layers[0].k_pool.data_ptr(), "layers must share the pools"
+        assert lay.v_pool.data_ptr() == layers[0].v_pool.data_ptr(), "layers must share the pools"
+    S.build_segpaged_cache_layers([lay.plan for lay in layers], [lay.table.data_ptr() for lay in layers],
+                                  [k.data_ptr() for k in k_dense], [v.data_ptr() for v in v_dense], ss, sh, st,
+                                  layers[0].k_pool.data_ptr(), layers[0].v_pool.data_ptr(), _stream(stream))
+
+
 class DecodeStepGraph:
     """One serving decode step of a ring-plan layer, captured once in a CUDA graph.
 

@@ -29,7 +29,7 @@ DTYPE_CODES = {"f32": SP_F32, "bf16": SP_BF16, "e4m3": SP_E4M3}
 # every symbol include/segpaged.h declares
 EXPORTED = ("segpaged_plan_create", "segpaged_plan_destroy", "segpaged_plan_sizes",
             "segpaged_plan_head_segments", "segpaged_plan_head_pages", "segpaged_table_write",
-            "build_segpaged_cache", "segpaged_gather", "segpaged_attention",
+            "build_segpaged_cache", "build_segpaged_cache_layers", "segpaged_gather", "segpaged_attention",
             "segpaged_attention_decode_noalloc", "segpaged_decode_append", "segpaged_read_device_status", "segpaged_clear_device_status", "segpaged_status_string",
             "segpaged_last_error", "segpaged_abi_version")
 
@@ -97,6 +97,8 @@ def load(path: Path | str | None = None) -> ctypes.CDLL:
         "segpaged_plan_head_pages": ([vp, i32, i32, ctypes.POINTER(i64), i32, ctypes.POINTER(i32)], i32),
         "segpaged_table_write": ([vp, vp, sz, vp], i32),
         "build_segpaged_cache": ([vp, vp, vp, vp, i64, i64, i64, vp, vp, vp], i32),
+        "build_segpaged_cache_layers": ([i32, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                         ctypes.POINTER(vp), i64, i64, i64, vp, vp, vp], i32),
         "segpaged_gather": ([vp, vp, vp, vp, vp, vp, i64, i64, i64, vp], i32),
         "segpaged_attention": ([vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp], i32),
         "segpaged_attention_decode_noalloc": ([vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp], i32),
@@ -202,6 +204,16 @@ def build_segpaged_cache(plan: int, d_table: int, k_dense: int, v_dense: int, st
                          stride_tok: int, k_pool: int, v_pool: int, stream: int = 0) -> None:
     _check(load().build_segpaged_cache(plan, d_table, k_dense, v_dense, stride_seq, stride_head, stride_tok,
                                        k_pool, v_pool, stream), "build_segpaged_cache")
+
+
+def build_segpaged_cache_layers(plans: Sequence[int], d_tables: Sequence[int], k_dense: Sequence[int],
+                                v_dense: Sequence[int], stride_seq: int, stride_head: int, stride_tok: int,
+                                k_pool: int, v_pool: int, stream: int = 0) -> None:
+    n = len(plans)
+    arr = lambda xs: (ctypes.c_void_p * max(1, n))(*xs)
+    _check(load().build_segpaged_cache_layers(n, arr(plans), arr(d_tables), arr(k_dense), arr(v_dense), stride_seq,
+                                              stride_head, stride_tok, k_pool, v_pool, stream),
+           "build_segpaged_cache_layers")
 
 
 def segpaged_gather(plan: int, d_table: int, k_pool: int, v_pool: int, k_out: int, v_out: int, stride_seq: int,

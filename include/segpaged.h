@@ -211,6 +211,23 @@ SP_API sp_status build_segpaged_cache(const sp_plan* plan, const void* d_table, 
                                const void* v_dense, int64_t stride_seq, int64_t stride_head,
                                int64_t stride_tok, void* k_pool, void* v_pool, void* stream);
 
+/* build_segpaged_cache for several layers in one launch.  Every (layer,
+ * kv-head) pair has its own policy ("SegPagedAttention runtime design", §2:
+ * e.g. 80 layers x 8 kv-heads for a 70B model), so a model's cache is one
+ * table per layer; this call packs several of them with a single launch (the
+ * pages have no counterpart: it only saves launches).  Layer i uses
+ * plans[i] / d_tables[i] and its dense K/V k_dense[i] / v_dense[i]; all
+ * layers share dtype, head_dim, page_size, page type, the dense strides and
+ * the pools (give each layer's plan its own first_page so that their pages do
+ * not overlap; the pools must hold every layer's pool_pages).  The result is
+ * bit for bit that of n_layers separate build_segpaged_cache calls.
+ * 1 <= n_layers <= 128.  Arguments are checked as in build_segpaged_cache,
+ * for every layer, before the launch. */
+SP_API sp_status build_segpaged_cache_layers(int32_t n_layers, const sp_plan* const* plans,
+                                             const void* const* d_tables, const void* const* k_dense,
+                                             const void* const* v_dense, int64_t stride_seq, int64_t stride_head,
+                                             int64_t stride_tok, void* k_pool, void* v_pool, void* stream);
+
 /* Inverse of build_segpaged_cache, for checking: writes each stored row back
  * into dense-shaped k_out / v_out (same addressing rules); rows that are not
  * stored are left untouched.  With SP_E4M3 pages it writes the 1-byte codes

@@ -1,6 +1,7 @@
 """C-ABI library and host planner tests (no GPU: only host-side entry points run)."""
 from __future__ import annotations
 
+import ctypes
 import re
 from pathlib import Path
 
@@ -300,3 +301,24 @@ def test_e4m3_pages_plan_and_validation():
                      (dict(BASE, kv_dtype="e4m3"), S.SP_ERR_UNSUPPORTED)):  # fp32 queries
         st, pl = S.segpaged_plan_create_status(S.make_problem(**kw))
         assert st == code and not pl, (kw, S.last_error())
+
+
+def test_multi_layer_build_checks_before_launch():
+    base = dict(batch=1, num_q_heads=4, num_kv_heads=2, head_dim=64, page_size=64, dtype="bf16", ctx_len=[300],
+                q_start=[299], policy=[("global", 0, 0), ("local", 4, 64)])
+    a = S.segpaged_plan_create(S.make_problem(**base))
+    b = S.segpaged_plan_create(S.make_problem(**dict(base, head_dim=128)))
+    lib = S.load()
+    arr = lambda xs: (ctypes.c_void_p * len(xs))(*xs)
+    ok = arr([256, 512])
+    # no layers, too many layers, NULL arrays, mismatched head_dim: refused on the host
+    assert lib.build_segpaged_cache_layers(0, arr([a]), arr([256]), arr([256]), arr([256]), 0, 0, 64, 256, 256,
+                                           None) == S.SP_ERR_INVALID_ARG
+    assert lib.build_segpaged_cache_layers(129, arr([a] * 129), arr([256] * 129), arr([256] * 129),
+                                           arr([256] * 129), 0, 0, 64, 256, 256, None) == S.SP_ERR_INVALID_ARG
+    assert lib.build_segpaged_cache_layers(2, None, ok, ok, ok, 0, 0, 64, 256, 256, None) == S.SP_ERR_INVALID_ARG
+    assert lib.build_segpaged_cache_layers(2, arr([a, b]), ok, ok, ok, 0, 0, 64, 256, 256,
+                                           None) == S.SP_ERR_INVALID_ARG
+    assert "same dtype" in S.last_error()
+    S.segpaged_plan_destroy(a)
+    S.segpaged_plan_destroy(b)

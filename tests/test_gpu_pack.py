@@ -133,3 +133,44 @@ def test_two_layers_share_one_pool_through_first_page():
         out, lse = lay.attention(q)
         torch.cuda.synchronize()
         assert_close(compare(prob, q, k, v, out, lse), "bf16")
+
+
+@pytest.mark.parametrize("kv_dtype", [None, "e4m3"])
+def test_pack_several_layers_in_one_launch(kv_dtype):
+    """build_segpaged_cache_layers: one launch for three layers sharing the pools gives the
+    same pool bytes as three build_segpaged_cache calls, and every layer gathers back bit-exact."""
+    from head_aware_paged_build_b200.runtime import build_layers
+    probs = [W.llama(layer=i, batch=1).decode_problem() for i in range(3)]
+    kw = lambda i: dict(kv_dtype="e4m3", k_scale=0.01 * (i + 1), v_scale=0.02 * (i + 1)) if kv_dtype else {}
+    first, firsts = 0, []
+    for i, prob in enumerate(probs):
+        firsts.append(first)
+        first += layer_for(prob, first_page=first, **kw(i)).sizes.pool_pages - first
+    probe = layer_for(probs[0], **kw(0))
+    nbytes = first * probe.sizes.page_bytes
+    dense = [W.dense_kv(prob, device="cuda") for prob in probs]
+    pools = []
+    for one_launch in (True, False):
+        kpool = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+        vpool = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+        layers = [layer_for(prob, first_page=f, pools=(kpool, vpool), **kw(i))
+                  for i, (prob, f) in enumerate(zip(probs, firsts))]
+        if one_launch:
+            build_layers(layers, [k for k, _ in dense], [v for _, v in dense])
+        else:
+            for lay, (k, v) in zip(layers, dense):
+                lay.build(k, v)
+        torch.cuda.synchronize()
+        pools.append((kpool, vpool, layers))
+    assert torch.equal(pools[0][0], pools[1][0]) and torch.equal(pools[0][1], pools[1][1])
+    if kv_dtype is None:
+        for lay, prob, (k, v) in zip(pools[0][2], probs, dense):
+            ko, vo = torch.full_like(k, float("nan")), torch.full_like(v, float("nan"))
+            lay.gather(ko, vo)
+            torch.cuda.synchronize()
+            for kv in range(prob.wl.num_kv_heads):
+                kind, s, w = prob.wl.policy[kv]
+                L = prob.ctx_lens[0]
+                m = torch.from_numpy(oracle.stored_mask(kind, s, w, L, L - 1)).cuda()
+                assert torch.equal(_bits(ko[0, kv, :L][m]), _bits(k[0, kv, :L][m])), kv
+                assert torch.equal(_bits(vo[0, kv, :L][m]), _bits(v[0, kv, :L][m])), kv
