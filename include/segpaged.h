@@ -60,8 +60,9 @@ typedef enum {
 
 /* Head kinds ("RedKnot head classification", four-kind table).  DENSE reads
  * the full causal context like GLOBAL (its RoPE re-alignment belongs to KV
- * reuse, outside attention).  RETRIEVAL (top-p token selection) is not
- * implemented: the pages give no scoring rule; it returns SP_ERR_UNSUPPORTED. */
+ * reuse, outside attention).  RETRIEVAL (pages fetched on demand) is not
+ * implemented: the pages give no rule for choosing the pages; it returns
+ * SP_ERR_UNSUPPORTED. */
 typedef enum { SP_GLOBAL = 0, SP_LOCAL = 1, SP_DENSE = 2, SP_RETRIEVAL = 3 } sp_kind;
 
 /* SP_E4M3 is a page type only (sp_problem.kv_dtype): FP8 E4M3 codes, 1 byte. */
