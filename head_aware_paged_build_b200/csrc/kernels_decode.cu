@@ -50,6 +50,100 @@ struct DecodeSmem {
   static constexpr int kBytes = kDescOff + NST * 16;
 };
 
+// Final merge of a split head, run by its last CTA over the n_slots partials
+// (m, l, acc) at p0 (standard split-KV: O = sum_i 2^(m_i - M) acc_i / L with
+// M = max_i m_i, L = sum_i 2^(m_i - M) l_i).  The consumer warps run it.
+//   1. one warp per row: (M, L) in one pass over the slots' (m, l) pairs,
+//      merged online per lane and then across lanes (a fixed butterfly, so
+//      every lane ends with the same bits);
+//   2. per 32-slot chunk, the slot weights 2^(m_i - M) go to shared memory
+//      (the first chunk's straight from step 1), and each thread adds NE
+//      (row, 4-column) entries over the chunk's slots, BATCH slots' loads in
+//      flight at a time, slots in increasing order.
+// All summation orders are fixed: results are bitwise reproducible.
+template <int D, int NE, int BATCH, bool FP8>
+__device__ __forceinline__ void merge_split_head(const DecodeLaunch& a, const HeadDesc& hd, int qh0, int G, int ns,
+                                                 const float* p0, float* wts, float* rowml, int warp, int lane) {
+  constexpr int kT = kConsumerWarps * 32;
+  constexpr int kChunk = 32;
+  const int64_t stride = partial_slot_floats(G, D);
+  float* row_m = rowml;              // [G] merged max (log2 units)
+  float* row_l = rowml + kMaxGroup;  // [G] merged sum
+  for (int row = warp; row < G; row += kConsumerWarps) {
+    float m = -INFINITY, l = 0.f, m_first = -INFINITY;
+    for (int i = lane; i < ns; i += 32) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p0 + i * stride + G * D + row * 2));
+      if (i == lane) m_first = ml.x;
+      const float mn = fmaxf(m, ml.x), b = mn == -INFINITY ? 0.f : mn;
+      l = l * fast_exp2(m - b) + ml.y * fast_exp2(ml.x - b);
+      m = mn;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m, o), lo = __shfl_xor_sync(0xffffffffu, l, o);
+      const float mn = fmaxf(m, mo), b = mn == -INFINITY ? 0.f : mn;
+      l = l * fast_exp2(m - b) + lo * fast_exp2(mo - b);
+      m = mn;
+    }
+    const float base = m == -INFINITY ? 0.f : m;
+    wts[row * kChunk + lane] = lane < ns ? fast_exp2(m_first - base) : 0.f;
+    if (lane == 0) row_m[row] = m, row_l[row] = l;
+  }
+  float4 acc[NE];
+#pragma unroll
+  for (int t = 0; t < NE; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c0 = 0; c0 < ns; c0 += kChunk) {
+    if (c0 > 0) {
+      asm volatile("bar.sync 1, %0;" ::"n"(kT) : "memory");  // the previous chunk's weights are consumed
+      for (int e = threadIdx.x; e < G * kChunk; e += kT) {
+        const int row = e / kChunk, i = c0 + e % kChunk;
+        const float M = row_m[row], base = M == -INFINITY ? 0.f : M;
+        wts[e] = i < ns ? fast_exp2(__ldcg(p0 + i * stride + G * D + row * 2) - base) : 0.f;
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kT) : "memory");
+    const int c1 = min(ns, c0 + kChunk);
+    for (int i = c0; i < c1; i += BATCH) {
+      float4 v[NE][BATCH];
+#pragma unroll
+      for (int t = 0; t < NE; ++t) {
+        const int e4 = threadIdx.x + t * kT, row = e4 / (D / 4), col = (e4 % (D / 4)) * 4;
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u)
+          v[t][u] = e4 < G * D / 4 && i + u < c1
+                        ? __ldcg(reinterpret_cast<const float4*>(p0 + (i + u) * stride + row * D + col))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int t = 0; t < NE; ++t) {
+        const int e4 = threadIdx.x + t * kT, row = e4 / (D / 4);
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+          if (e4 < G * D / 4 && i + u < c1) {
+            const float f = wts[row * kChunk + (i + u - c0)];
+            acc[t].x += f * v[t][u].x, acc[t].y += f * v[t][u].y;
+            acc[t].z += f * v[t][u].z, acc[t].w += f * v[t][u].w;
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < NE; ++t) {
+    const int e4 = threadIdx.x + t * kT, row = e4 / (D / 4), col = (e4 % (D / 4)) * 4;
+    if (e4 < G * D / 4) {
+      const float inv = (FP8 ? a.v_scale : 1.f) / row_l[row];
+      __nv_bfloat16* o =
+          static_cast<__nv_bfloat16*>(a.out) + (int64_t(hd.q_row0) * a.num_q_heads + qh0 + row) * D + col;
+      reinterpret_cast<uint2*>(o)[0] = make_uint2(pack_bf16x2(acc[t].x * inv, acc[t].y * inv),
+                                                  pack_bf16x2(acc[t].z * inv, acc[t].w * inv));
+    }
+  }
+  if (threadIdx.x < G && a.lse)
+    a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + threadIdx.x] =
+        (row_m[threadIdx.x] + log2f(row_l[threadIdx.x])) * kLn2;
+}
+
 template <int D, int NST, bool FP8>
 __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch a) {
   using S = DecodeSmem<D, NST, FP8>;
@@ -354,48 +448,61 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch
       if (s_last) {
         __threadfence();
         const int ns = item.n_slots;
-        const int64_t stride = partial_slot_floats(G, D);
-        const float* p0 = a.partial + int64_t(item.slot0) * stride;
-        float* row_m = mlbuf;              // [G] merged max
-        float* row_l = mlbuf + kMaxGroup;  // [G] merged sum
-        // per row: max and weighted sum over the slots, one warp per row
-        for (int row = warp; row < G; row += kConsumerWarps) {
-          float m = -INFINITY;
-          for (int i = lane; i < ns; i += 32) m = fmaxf(m, __ldcg(p0 + i * stride + G * D + row * 2));
+        if constexpr (!FP8) {
+          // 16 float4 loads in flight per thread: 8 slots of two (row, 4-column)
+          // entries, or 4 slots of four.
+          const float* p0 = a.partial + int64_t(item.slot0) * partial_slot_floats(G, D);
+          if (G * D / 4 <= 2 * kConsumerWarps * 32)
+            merge_split_head<D, 2, 8, false>(a, hd, qh0, G, ns, p0, mbuf, mlbuf, warp, lane);
+          else
+            merge_split_head<D, 4, 4, false>(a, hd, qh0, G, ns, p0, mbuf, mlbuf, warp, lane);
+        } else {
+          // E4M3 pages keep a serial merge (four slots' loads in flight): with the
+          // batched one inlined, the kernel's register allocation grew from 153 to
+          // 200 and its page loop ran 38% slower (measured on the 32K layer).
+          const int64_t stride = partial_slot_floats(G, D);
+          const float* p0 = a.partial + int64_t(item.slot0) * stride;
+          float* row_m = mlbuf;              // [G] merged max
+          float* row_l = mlbuf + kMaxGroup;  // [G] merged sum
+          // per row: max and weighted sum over the slots, one warp per row
+          for (int row = warp; row < G; row += kConsumerWarps) {
+            float m = -INFINITY;
+            for (int i = lane; i < ns; i += 32) m = fmaxf(m, __ldcg(p0 + i * stride + G * D + row * 2));
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-          const float base = m == -INFINITY ? 0.f : m;
-          float l = 0.f;
-          for (int i = lane; i < ns; i += 32) {
-            const float* ml = p0 + i * stride + G * D + row * 2;
-            l += fast_exp2(__ldcg(ml) - base) * __ldcg(ml + 1);
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            const float base = m == -INFINITY ? 0.f : m;
+            float l = 0.f;
+            for (int i = lane; i < ns; i += 32) {
+              const float* ml = p0 + i * stride + G * D + row * 2;
+              l += fast_exp2(__ldcg(ml) - base) * __ldcg(ml + 1);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+            if (lane == 0) row_m[row] = m, row_l[row] = l;
           }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-          if (lane == 0) row_m[row] = m, row_l[row] = l;
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-        // weighted sum of the slots' accumulators, four columns per thread, slots in order
-        for (int e4 = threadIdx.x; e4 < G * D / 4; e4 += kConsumerWarps * 32) {
-          const int row = e4 / (D / 4), col = (e4 % (D / 4)) * 4;
-          const float M = row_m[row], base = M == -INFINITY ? 0.f : M;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+          // weighted sum of the slots' accumulators, four columns per thread, slots in order
+          for (int e4 = threadIdx.x; e4 < G * D / 4; e4 += kConsumerWarps * 32) {
+            const int row = e4 / (D / 4), col = (e4 % (D / 4)) * 4;
+            const float M = row_m[row], base = M == -INFINITY ? 0.f : M;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-          for (int i = 0; i < ns; ++i) {
-            const float* sl = p0 + i * stride;
-            const float f = fast_exp2(__ldcg(sl + G * D + row * 2) - base);
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(sl + row * D + col));
-            acc.x += f * v.x, acc.y += f * v.y, acc.z += f * v.z, acc.w += f * v.w;
+            for (int i = 0; i < ns; ++i) {
+              const float* sl = p0 + i * stride;
+              const float f = fast_exp2(__ldcg(sl + G * D + row * 2) - base);
+              const float4 v = __ldcg(reinterpret_cast<const float4*>(sl + row * D + col));
+              acc.x += f * v.x, acc.y += f * v.y, acc.z += f * v.z, acc.w += f * v.w;
+            }
+            const float inv = a.v_scale / row_l[row];
+            __nv_bfloat16* o =
+                static_cast<__nv_bfloat16*>(a.out) + (int64_t(hd.q_row0) * a.num_q_heads + qh0 + row) * D + col;
+            reinterpret_cast<uint2*>(o)[0] = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv),
+                                                        pack_bf16x2(acc.z * inv, acc.w * inv));
           }
-          const float inv = (FP8 ? a.v_scale : 1.f) / row_l[row];
-          __nv_bfloat16* o =
-              static_cast<__nv_bfloat16*>(a.out) + (int64_t(hd.q_row0) * a.num_q_heads + qh0 + row) * D + col;
-          reinterpret_cast<uint2*>(o)[0] = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv),
-                                                      pack_bf16x2(acc.z * inv, acc.w * inv));
+          if (threadIdx.x < G && a.lse)
+            a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + threadIdx.x] =
+                (row_m[threadIdx.x] + log2f(row_l[threadIdx.x])) * kLn2;
         }
-        if (threadIdx.x < G && a.lse)
-          a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + threadIdx.x] =
-              (row_m[threadIdx.x] + log2f(row_l[threadIdx.x])) * kLn2;
         if (threadIdx.x == 0) a.counters[item.comb] = 0;
       }
     }
