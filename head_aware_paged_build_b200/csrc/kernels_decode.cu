@@ -63,7 +63,8 @@ struct DecodeSmem {
 // All summation orders are fixed: results are bitwise reproducible.
 template <int D, int NE, int BATCH, bool FP8>
 __device__ __forceinline__ void merge_split_head(const DecodeLaunch& a, const HeadDesc& hd, int qh0, int G, int ns,
-                                                 const float* p0, float* wts, float* rowml, int warp, int lane) {
+                                                 const float* p0, float* part, float* wts, float* rowml, int warp,
+                                                 int lane) {
   constexpr int kT = kConsumerWarps * 32;
   constexpr int kChunk = 32;
   const int64_t stride = partial_slot_floats(G, D);
@@ -127,6 +128,16 @@ __device__ __forceinline__ void merge_split_head(const DecodeLaunch& a, const He
         }
       }
     }
+  }
+  if (part) {  // a merge group: the merged partial (acc, M, L) in the same slot layout
+#pragma unroll
+    for (int t = 0; t < NE; ++t) {
+      const int e4 = threadIdx.x + t * kT, row = e4 / (D / 4), col = (e4 % (D / 4)) * 4;
+      if (e4 < G * D / 4) *reinterpret_cast<float4*>(part + row * D + col) = acc[t];
+    }
+    if (threadIdx.x < G)
+      part[G * D + threadIdx.x * 2] = row_m[threadIdx.x], part[G * D + threadIdx.x * 2 + 1] = row_l[threadIdx.x];
+    return;
   }
 #pragma unroll
   for (int t = 0; t < NE; ++t) {
@@ -438,24 +449,56 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch
       }
     }
     if (item.slot >= 0) {
-      // Split head: publish this partial, take a ticket; the last of the head's
-      // n_slots CTAs merges all partials in slot order (fixed order: bitwise
-      // reproducible) and returns the counter to zero for the next call.
+      // Split head: publish this partial, take a ticket; the last CTA to arrive
+      // merges in slot order (fixed order: bitwise reproducible) and returns
+      // the counter to zero for the next call.  A head with merge groups takes
+      // its ticket on its group's counter: the group's last CTA merges the
+      // group into the group's slot, then takes a ticket on the head's counter,
+      // and the last group's merger merges the group slots.
+      int grp = 0, cnt = item.comb, n_arrive = item.n_slots;
+      if constexpr (!FP8) {  // E4M3 plans have no merge groups
+        if (item.gsz > 0) {
+          grp = (item.slot - item.slot0) / item.gsz;
+          cnt = item.gcnt0 + grp;
+          n_arrive = min(item.gsz, item.n_slots - grp * item.gsz);
+        }
+      }
       __threadfence();
       asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-      if (threadIdx.x == 0) s_last = atomicAdd(&a.counters[item.comb], 1) == item.n_slots - 1;
+      if (threadIdx.x == 0) s_last = atomicAdd(&a.counters[cnt], 1) == n_arrive - 1;
       asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
       if (s_last) {
         __threadfence();
         const int ns = item.n_slots;
         if constexpr (!FP8) {
-          // 16 float4 loads in flight per thread: 8 slots of two (row, 4-column)
-          // entries, or 4 slots of four.
-          const float* p0 = a.partial + int64_t(item.slot0) * partial_slot_floats(G, D);
-          if (G * D / 4 <= 2 * kConsumerWarps * 32)
-            merge_split_head<D, 2, 8, false>(a, hd, qh0, G, ns, p0, mbuf, mlbuf, warp, lane);
-          else
-            merge_split_head<D, 4, 4, false>(a, hd, qh0, G, ns, p0, mbuf, mlbuf, warp, lane);
+          const int64_t stride = partial_slot_floats(G, D);
+          const float* src = a.partial + int64_t(item.slot0 + grp * item.gsz) * stride;
+          int n_src = n_arrive;
+          float* part = item.gsz > 0 ? a.partial + int64_t(item.gslot0 + grp) * stride : nullptr;
+          for (;;) {
+            // 16 float4 loads in flight per thread: 8 slots of two (row, 4-column)
+            // entries, or 4 slots of four.
+            if (G * D / 4 <= 2 * kConsumerWarps * 32)
+              merge_split_head<D, 2, 8, false>(a, hd, qh0, G, n_src, src, part, mbuf, mlbuf, warp, lane);
+            else
+              merge_split_head<D, 4, 4, false>(a, hd, qh0, G, n_src, src, part, mbuf, mlbuf, warp, lane);
+            if (part == nullptr) {
+              if (threadIdx.x == 0) a.counters[item.comb] = 0;
+              break;
+            }
+            // group merged: reset its counter, publish the group slot, ticket on the head
+            if (threadIdx.x == 0) a.counters[cnt] = 0;
+            const int ng = (ns + item.gsz - 1) / item.gsz;
+            __threadfence();
+            asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+            if (threadIdx.x == 0) s_last = atomicAdd(&a.counters[item.comb], 1) == ng - 1;
+            asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+            if (!s_last) break;
+            __threadfence();
+            src = a.partial + int64_t(item.gslot0) * stride;
+            n_src = ng;
+            part = nullptr;
+          }
         } else {
           // E4M3 pages keep a serial merge (four slots' loads in flight): with the
           // batched one inlined, the kernel's register allocation grew from 153 to
@@ -502,8 +545,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch
           if (threadIdx.x < G && a.lse)
             a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + threadIdx.x] =
                 (row_m[threadIdx.x] + log2f(row_l[threadIdx.x])) * kLn2;
+          if (threadIdx.x == 0) a.counters[item.comb] = 0;
         }
-        if (threadIdx.x == 0) a.counters[item.comb] = 0;
       }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");

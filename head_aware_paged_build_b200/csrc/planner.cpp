@@ -29,6 +29,7 @@ namespace {
 
 constexpr int kDefaultDecodeCtas = 2 * 148;
 constexpr int64_t kItemCostPages100 = 200;  // a head start costs as much as two pages (measured)
+constexpr int32_t kMergeOneLevel = 16;      // split heads with more items merge in two levels
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -295,30 +296,54 @@ sp_status plan_build(sp_plan& pl) {
       while (lo < hi) {
         const int h = pl.pages[lo].head;
         const int64_t end = std::min<int64_t>(hi, pl.heads[h].vpage_begin + pl.heads[h].n_vpages);
-        pl.decode_items.push_back(DecodeItem{h, int32_t(lo), int32_t(end), -1, -1, 0, 0, 0});
+        pl.decode_items.push_back(DecodeItem{h, int32_t(lo), int32_t(end), -1, -1, 0, 0, 0, 0, 0, {0, 0}});
         lo = end;
       }
       pl.decode_cta_begin.push_back(int32_t(pl.decode_items.size()));
     }
-    // items of a head are consecutive; split heads get consecutive slots
+    // items of a head are consecutive; split heads get consecutive slots.  On
+    // bf16 pages a head split into more than kMergeOneLevel items merges in two
+    // levels (groups of about sqrt(n) slots), so no single CTA reads all of a
+    // long head's partials at the end of the call.
+    const bool two_level = p.dtype == SP_BF16 && !pl.fp8;
+    int32_t n_group_counters = 0;
     size_t i = 0;
     while (i < pl.decode_items.size()) {
       size_t j = i;
       while (j < pl.decode_items.size() && pl.decode_items[j].head == pl.decode_items[i].head) ++j;
       if (j - i > 1) {
+        const int32_t ns = int32_t(j - i);
         const int32_t comb = int32_t(pl.combine.size());
-        pl.combine.push_back(CombineItem{pl.decode_items[i].head, n_slots, int32_t(j - i), 0});
+        pl.combine.push_back(CombineItem{pl.decode_items[i].head, n_slots, ns, 0});
         const int32_t slot0 = n_slots;
+        n_slots += ns;
+        int32_t gsz = 0, gslot0 = 0, gcnt0 = 0;
+        if (two_level && ns > kMergeOneLevel) {
+          gsz = 1;
+          while (gsz * gsz < ns) ++gsz;  // ceil(sqrt(ns))
+          const int32_t ng = (ns + gsz - 1) / gsz;
+          gslot0 = n_slots;
+          n_slots += ng;
+          gcnt0 = n_group_counters;
+          n_group_counters += ng;
+        }
         for (size_t k = i; k < j; ++k) {
           DecodeItem& d = pl.decode_items[k];
-          d.slot = n_slots++;
+          d.slot = slot0 + int32_t(k - i);
           d.comb = comb;
-          d.n_slots = int32_t(j - i);
+          d.n_slots = ns;
           d.slot0 = slot0;
+          d.gsz = gsz;
+          d.gslot0 = gslot0;
+          d.gcnt0 = gcnt0;
         }
       }
       i = j;
     }
+    // group counters follow the heads' counters in the workspace
+    for (DecodeItem& d : pl.decode_items)
+      if (d.gsz > 0) d.gcnt0 += int32_t(pl.combine.size());
+    pl.n_counters = int32_t(pl.combine.size()) + n_group_counters;
   } else {
     // --- prefill: query tiles x visited KV tile ranges -----------------------
     // bf16 items pair two query tiles of the same (sequence, kv-head) so that
@@ -412,9 +437,10 @@ sp_status plan_build(sp_plan& pl) {
   z.pool_pages = p.first_page + max_id + 1;
   z.page_bytes = int64_t(P) * D * (pl.fp8 ? 1 : pl.elem_bytes);
   z.table_bytes = int64_t(pl.blob.size());
-  // workspace: status word block | one arrival counter per split head | partial slots
+  // workspace: status word block | arrival counters (one per split head, then
+  // one per merge group) | partial slots (items' slots, then group slots)
   const int64_t partial = int64_t(n_slots) * partial_slot_floats(pl.group, D) * 4;
-  pl.partial_offset = kStatusBytes + ceil_div(int64_t(pl.combine.size()) * 4, 256) * 256;
+  pl.partial_offset = kStatusBytes + ceil_div(int64_t(pl.n_counters) * 4, 256) * 256;
   z.workspace_bytes = pl.partial_offset + ceil_div(partial, 256) * 256;
   z.stored_token_heads = stored;
   z.dense_token_heads = dense_rows;

@@ -79,9 +79,16 @@ struct alignas(16) DecodeItem {
   int32_t comb;      // split head index (arrival counter), -1 if not split
   int32_t n_slots;   // items the split head has
   int32_t slot0;     // first slot of the split head
-  int32_t pad;
+  // Two-level merge of a head split into many items: its slots form groups of
+  // gsz consecutive slots; the last CTA of a group merges the group into a
+  // group slot (gslot0 + group) and the last group's merger merges those.
+  // gsz = 0: the last of the n_slots CTAs merges all slots.
+  int32_t gsz;
+  int32_t gslot0;    // first group slot of the head (after its n_slots item slots)
+  int32_t gcnt0;     // arrival counter of the head's first group
+  int32_t pad[2];
 };
-static_assert(sizeof(DecodeItem) == 32, "DecodeItem layout");
+static_assert(sizeof(DecodeItem) == 48, "DecodeItem layout");
 
 // A head whose decode result is split across several items.
 struct alignas(16) CombineItem {
@@ -144,6 +151,7 @@ struct sp_plan {
   float k_scale = 1.f, v_scale = 1.f;     // E4M3 page scales
   int32_t prefill_tile = 0;
   int32_t n_partial_slots = 0;
+  int32_t n_counters = 0;      // arrival counters in the workspace (split heads, then merge groups)
   int64_t partial_offset = 0;  // workspace byte offset of the partial slots (status word, then counters)
 };
 

@@ -248,8 +248,9 @@ SP_API sp_status segpaged_gather(const sp_plan* plan, const void* d_table, const
  *   softmax_scale  <= 0 selects 1/sqrt(head_dim)
  *   workspace      device, >= workspace_bytes, 256-byte aligned, zero-filled
  *                  before its first use; it holds the device status word (first
- *                  256 bytes), one arrival counter per split decode head (the
- *                  kernels return them to zero) and the split partial results.
+ *                  256 bytes), arrival counters of split decode heads and of
+ *                  their merge groups (the kernels return them to zero) and
+ *                  the split partial results.
  *                  After a non-zero device status, zero it again before reuse.
  *                  Calls that overlap on the GPU need separate workspaces.
  * Decode plans run a split-KV kernel over each head's own pages plus a
