@@ -42,6 +42,8 @@ class SegPagedLayer:
                                       q_start, policy, first_page, page_ids, target_ctas, flags, append_capacity,
                                       kv_dtype, k_scale, v_scale)
         self.kv_dtype = kv_dtype or dtype
+        self.batch = batch
+        self.ctx_len = [int(x) for x in ctx_len]
         self.plan = S.segpaged_plan_create(self.problem)
         self.sizes = S.segpaged_plan_sizes(self.plan)
         z = self.sizes
@@ -55,18 +57,46 @@ class SegPagedLayer:
             self.k_pool, self.v_pool = pools
         self.workspace = torch.zeros(z.workspace_bytes, dtype=torch.uint8, device=self.device)
 
+    # -- argument checks (the C ABI sees only pointers and strides) ------------
+    def _check_tensor(self, t: torch.Tensor, what: str, dtype: torch.dtype) -> None:
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{what} must be a torch.Tensor")
+        if t.dtype != dtype:
+            raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+        if t.device != self.k_pool.device:
+            raise ValueError(f"{what} is on {t.device}, the layer's buffers on {self.k_pool.device}")
+
+    def _check_dense(self, k: torch.Tensor, v: torch.Tensor, varlen: bool, what: str) -> None:
+        """Dense K/V (or gather targets): every row the plan reads or writes must lie inside."""
+        self._check_tensor(k, f"{what} K", self.torch_dtype)
+        self._check_tensor(v, f"{what} V", self.torch_dtype)
+        if k.shape != v.shape or k.stride() != v.stride() or k.stride(-1) != 1:
+            raise ValueError(f"{what}: K and V need the same shape and strides, head_dim contiguous")
+        d, hkv = self.head_dim, self.num_kv_heads
+        if varlen:
+            ok = k.dim() == 3 and k.shape[0] >= sum(self.ctx_len) and k.shape[1] >= hkv and k.shape[2] == d
+            want = f"[>= {sum(self.ctx_len)}, >= {hkv}, {d}]"
+        else:
+            ok = (k.dim() == 4 and k.shape[0] >= self.batch and k.shape[1] >= hkv and
+                  k.shape[2] >= max(self.ctx_len) and k.shape[3] == d)
+            want = f"[>= {self.batch}, >= {hkv}, >= {max(self.ctx_len)}, {d}]"
+        if not ok:
+            raise ValueError(f"{what}: K/V shape {tuple(k.shape)} does not cover {want}")
+
     # -- calls --------------------------------------------------------------
     def build(self, k_dense: torch.Tensor, v_dense: torch.Tensor, varlen: bool = False, stream=None) -> None:
         """Pack dense K/V ([B, Hkv, Lmax, d], or varlen [sum L, Hkv, d] with varlen=True)."""
+        self._check_dense(k_dense, v_dense, varlen, "build")
         if varlen:
             ss, sh, st = S.SP_VARLEN, k_dense.stride(1), k_dense.stride(0)
         else:
             ss, sh, st = k_dense.stride(0), k_dense.stride(1), k_dense.stride(2)
-        assert k_dense.stride() == v_dense.stride() and k_dense.stride(-1) == 1
         S.build_segpaged_cache(self.plan, self.table.data_ptr(), k_dense.data_ptr(), v_dense.data_ptr(), ss, sh,
                                st, self.k_pool.data_ptr(), self.v_pool.data_ptr(), _stream(stream))
 
     def gather(self, k_out: torch.Tensor, v_out: torch.Tensor, varlen: bool = False, stream=None) -> None:
+        """Write every stored row back to its dense position (the inverse of build; E4M3 pages give codes)."""
+        self._check_dense(k_out, v_out, varlen, "gather")
         if varlen:
             ss, sh, st = S.SP_VARLEN, k_out.stride(1), k_out.stride(0)
         else:
@@ -77,11 +107,21 @@ class SegPagedLayer:
     def attention(self, q: torch.Tensor, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
                   scale: float = 0.0, with_lse: bool = True, stream=None):
         """q: [sum C_b, Hq, d] contiguous; returns (out, lse)."""
-        assert q.is_contiguous() and q.dtype == self.torch_dtype
+        rows = (self.sizes.num_queries, self.num_q_heads)
+        self._check_tensor(q, "q", self.torch_dtype)
+        if tuple(q.shape) != rows + (self.head_dim,) or not q.is_contiguous():
+            raise ValueError(f"q must be contiguous {rows + (self.head_dim,)}, got {tuple(q.shape)}")
         if out is None:
             out = torch.empty_like(q)
+        self._check_tensor(out, "out", self.torch_dtype)
+        if out.shape != q.shape or not out.is_contiguous():
+            raise ValueError(f"out must be contiguous {tuple(q.shape)}, got {tuple(out.shape)}")
         if lse is None and with_lse:
             lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device)
+        if lse is not None:
+            self._check_tensor(lse, "lse", torch.float32)
+            if tuple(lse.shape) != rows or not lse.is_contiguous():
+                raise ValueError(f"lse must be contiguous {rows}, got {tuple(lse.shape)}")
         S.segpaged_attention(self.plan, self.table.data_ptr(), self.k_pool.data_ptr(), self.v_pool.data_ptr(),
                              q.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None, scale,
                              self.workspace.data_ptr(), self.workspace.numel(), _stream(stream))
@@ -89,7 +129,13 @@ class SegPagedLayer:
 
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
         """Ring plans: add one token per sequence (k_new, v_new: [B, Hkv, d])."""
-        assert k_new.stride() == v_new.stride() and k_new.stride(-1) == 1
+        self._check_tensor(k_new, "k_new", self.torch_dtype)
+        self._check_tensor(v_new, "v_new", self.torch_dtype)
+        if (k_new.dim() != 3 or k_new.shape != v_new.shape or k_new.stride() != v_new.stride() or
+                k_new.stride(-1) != 1 or k_new.shape[0] < self.batch or k_new.shape[1] < self.num_kv_heads or
+                k_new.shape[2] != self.head_dim):
+            raise ValueError(f"k_new / v_new must be [{self.batch}, {self.num_kv_heads}, {self.head_dim}] "
+                             f"with the same strides, head_dim contiguous; got {tuple(k_new.shape)}")
         S.segpaged_decode_append(self.plan, self.table.data_ptr(), k_new.data_ptr(), v_new.data_ptr(),
                                  k_new.stride(0), k_new.stride(1), self.k_pool.data_ptr(), self.v_pool.data_ptr(),
                                  self.workspace.data_ptr(), _stream(stream))
@@ -124,15 +170,20 @@ def build_layers(layers: Sequence[SegPagedLayer], k_dense: Sequence[torch.Tensor
     ``layers[i]`` packs ``k_dense[i]`` / ``v_dense[i]`` (all with the same strides); the
     layers must hold the same pools (``pools=`` at construction, distinct ``first_page``).
     """
+    if not (len(layers) == len(k_dense) == len(v_dense)) or not layers:
+        raise ValueError("build_layers: one dense K and one dense V per layer, at least one layer")
     k0 = k_dense[0]
     if varlen:
         ss, sh, st = S.SP_VARLEN, k0.stride(1), k0.stride(0)
     else:
         ss, sh, st = k0.stride(0), k0.stride(1), k0.stride(2)
     for lay, k, v in zip(layers, k_dense, v_dense):
-        assert k.stride() == k0.stride() and v.stride() == k0.stride() and k0.stride(-1) == 1
-        assert lay.k_pool.data_ptr() == layers[0].k_pool.data_ptr(), "layers must share the pools"
-        assert lay.v_pool.data_ptr() == layers[0].v_pool.data_ptr(), "layers must share the pools"
+        lay._check_dense(k, v, varlen, "build_layers")
+        if k.stride() != k0.stride():
+            raise ValueError("build_layers: every layer's dense K/V needs the same strides")
+        if (lay.k_pool.data_ptr() != layers[0].k_pool.data_ptr() or
+                lay.v_pool.data_ptr() != layers[0].v_pool.data_ptr()):
+            raise ValueError("build_layers: the layers must share the pools")
     S.build_segpaged_cache_layers([lay.plan for lay in layers], [lay.table.data_ptr() for lay in layers],
                                   [k.data_ptr() for k in k_dense], [v.data_ptr() for v in v_dense], ss, sh, st,
                                   layers[0].k_pool.data_ptr(), layers[0].v_pool.data_ptr(), _stream(stream))
