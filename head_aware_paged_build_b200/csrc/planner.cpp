@@ -537,4 +537,33 @@ sp_status segpaged_plan_head_pages(const sp_plan* plan, int32_t b, int32_t kv, i
   return SP_OK;
 }
 
+sp_status segpaged_plan_decode_items(const sp_plan* plan, int32_t* records, int32_t max, int32_t* count) {
+  if (!plan || !count || (max > 0 && !records)) return sp::fail(SP_ERR_INVALID_ARG, "NULL argument");
+  const int32_t n = int32_t(plan->decode_items.size());
+  *count = n;
+  const int32_t hkv = plan->prob.num_kv_heads;
+  int32_t i = 0;
+  for (size_t c = 0; c + 1 < plan->decode_cta_begin.size(); ++c) {
+    for (int32_t it = plan->decode_cta_begin[c]; it < plan->decode_cta_begin[c + 1]; ++it, ++i) {
+      if (i >= max) return SP_OK;
+      const sp::DecodeItem& d = plan->decode_items[it];
+      const sp::HeadDesc& hd = plan->heads[d.head];
+      int32_t* r = records + int64_t(i) * SP_DECODE_ITEM_WORDS;
+      r[0] = int32_t(c);
+      r[1] = d.head / hkv;
+      r[2] = d.head % hkv;
+      r[3] = d.vp_begin - hd.vpage_begin;
+      r[4] = d.vp_end - hd.vpage_begin;
+      r[5] = d.slot;
+      r[6] = d.slot >= 0 ? d.n_slots : 1;
+      r[7] = d.slot >= 0 ? d.slot0 : -1;
+      r[8] = d.gsz;
+      r[9] = d.gsz > 0 ? d.gslot0 : -1;
+      r[10] = d.slot >= 0 ? d.comb : -1;
+      r[11] = d.gsz > 0 ? d.gcnt0 + (d.slot - d.slot0) / d.gsz : -1;
+    }
+  }
+  return SP_OK;
+}
+
 }  // extern "C"

@@ -28,7 +28,8 @@ DTYPE_CODES = {"f32": SP_F32, "bf16": SP_BF16, "e4m3": SP_E4M3}
 
 # every symbol include/segpaged.h declares
 EXPORTED = ("segpaged_plan_create", "segpaged_plan_destroy", "segpaged_plan_sizes",
-            "segpaged_plan_head_segments", "segpaged_plan_head_pages", "segpaged_table_write",
+            "segpaged_plan_head_segments", "segpaged_plan_head_pages", "segpaged_plan_decode_items",
+            "segpaged_table_write",
             "build_segpaged_cache", "build_segpaged_cache_layers", "segpaged_gather", "segpaged_attention",
             "segpaged_attention_decode_noalloc", "segpaged_decode_append", "segpaged_read_device_status", "segpaged_clear_device_status", "segpaged_status_string",
             "segpaged_last_error", "segpaged_abi_version")
@@ -95,6 +96,7 @@ def load(path: Path | str | None = None) -> ctypes.CDLL:
         "segpaged_plan_sizes": ([vp, ctypes.POINTER(sp_sizes)], i32),
         "segpaged_plan_head_segments": ([vp, i32, i32, ctypes.POINTER(sp_segment), i32, ctypes.POINTER(i32)], i32),
         "segpaged_plan_head_pages": ([vp, i32, i32, ctypes.POINTER(i64), i32, ctypes.POINTER(i32)], i32),
+        "segpaged_plan_decode_items": ([vp, ctypes.POINTER(i32), i32, ctypes.POINTER(i32)], i32),
         "segpaged_table_write": ([vp, vp, sz, vp], i32),
         "build_segpaged_cache": ([vp, vp, vp, vp, i64, i64, i64, vp, vp, vp], i32),
         "build_segpaged_cache_layers": ([i32, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
@@ -194,6 +196,21 @@ def segpaged_plan_head_pages(plan: int, b: int, kv: int) -> list[int]:
     ids = (ctypes.c_int64 * max(1, n.value))()
     _check(load().segpaged_plan_head_pages(plan, b, kv, ids, n.value, ctypes.byref(n)), "segpaged_plan_head_pages")
     return list(ids[: n.value])
+
+
+SP_DECODE_ITEM_WORDS = 12
+DECODE_ITEM_FIELDS = ("cta", "b", "kv", "page_begin", "page_end", "slot", "n_slots", "slot0", "group_size",
+                      "group_slot0", "counter", "group_counter")
+
+
+def segpaged_plan_decode_items(plan: int) -> list[dict]:
+    """The decode work split of a plan, one dict per work item in launch order."""
+    n = ctypes.c_int32()
+    _check(load().segpaged_plan_decode_items(plan, None, 0, ctypes.byref(n)), "segpaged_plan_decode_items")
+    rec = (ctypes.c_int32 * max(1, n.value * SP_DECODE_ITEM_WORDS))()
+    _check(load().segpaged_plan_decode_items(plan, rec, n.value, ctypes.byref(n)), "segpaged_plan_decode_items")
+    w = SP_DECODE_ITEM_WORDS
+    return [dict(zip(DECODE_ITEM_FIELDS, rec[i * w:(i + 1) * w])) for i in range(n.value)]
 
 
 def segpaged_table_write(plan: int, d_table: int, nbytes: int, stream: int = 0) -> None:

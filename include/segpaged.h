@@ -190,6 +190,24 @@ SP_API sp_status segpaged_plan_head_segments(const sp_plan* plan, int32_t b, int
 SP_API sp_status segpaged_plan_head_pages(const sp_plan* plan, int32_t b, int32_t kv, int64_t* page_ids,
                                    int32_t max, int32_t* count);
 
+/* Inspect the decode work split of a plan (host only; prefill plans have no
+ * decode items).  One record of SP_DECODE_ITEM_WORDS int32 per work item, in
+ * launch order:
+ *   [0] CTA   [1] b   [2] kv
+ *   [3] first page, [4] one past the last page (indices into the head's page
+ *       list, as segpaged_plan_head_pages orders it)
+ *   [5] the item's partial slot in the workspace, or -1 when the item covers
+ *       the whole head (no merge)
+ *   [6] items of the head   [7] the head's first slot
+ *   [8] merge group size: 0 for a one-level merge, else the head's slots form
+ *       groups of this many, each merged into a group slot first
+ *   [9] the head's first group slot
+ *   [10] the head's arrival counter (-1 when the head is not split)
+ *   [11] the arrival counter of the item's merge group (-1 when none)
+ * *count receives the number of items; at most `max` records are written. */
+#define SP_DECODE_ITEM_WORDS 12
+SP_API sp_status segpaged_plan_decode_items(const sp_plan* plan, int32_t* records, int32_t max, int32_t* count);
+
 /* Copy the plan's table blob to `d_table` (device, >= table_bytes, 16-byte
  * aligned) with an asynchronous host-to-device copy on `stream`. */
 SP_API sp_status segpaged_table_write(const sp_plan* plan, void* d_table, size_t bytes, void* stream);
