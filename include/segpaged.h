@@ -191,8 +191,10 @@ SP_API sp_status segpaged_plan_head_pages(const sp_plan* plan, int32_t b, int32_
                                    int32_t max, int32_t* count);
 
 /* Inspect the decode work split of a plan (host only; prefill plans have no
- * decode items).  One record of SP_DECODE_ITEM_WORDS int32 per work item, in
- * launch order:
+ * decode items).  The pages have no counterpart: this is the bookkeeping of
+ * this library's split-KV decode, exposed for tuning target_ctas and for
+ * tests.  One record of SP_DECODE_ITEM_WORDS int32 per work item, in launch
+ * order:
  *   [0] CTA   [1] b   [2] kv
  *   [3] first page, [4] one past the last page (indices into the head's page
  *       list, as segpaged_plan_head_pages orders it)
