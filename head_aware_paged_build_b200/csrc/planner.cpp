@@ -566,4 +566,25 @@ sp_status segpaged_plan_decode_items(const sp_plan* plan, int32_t* records, int3
   return SP_OK;
 }
 
+sp_status segpaged_plan_prefill_items(const sp_plan* plan, int32_t* records, int32_t max, int32_t* count) {
+  if (!plan || !count || (max > 0 && !records)) return sp::fail(SP_ERR_INVALID_ARG, "NULL argument");
+  const int32_t n = int32_t(plan->prefill.size());
+  *count = n;
+  const int32_t hkv = plan->prob.num_kv_heads;
+  for (int32_t i = 0; i < n && i < max; ++i) {
+    const sp::PrefillItem& it = plan->prefill[i];
+    int32_t* r = records + int64_t(i) * SP_PREFILL_ITEM_WORDS;
+    r[0] = it.head / hkv;
+    r[1] = it.head % hkv;
+    r[2] = plan->prefill_tile;
+    r[3] = it.qh[0], r[4] = it.qh[1];
+    r[5] = it.q_row[0], r[6] = it.qh[1] >= 0 ? it.q_row[1] : 0;
+    r[7] = it.n_rows[0], r[8] = it.qh[1] >= 0 ? it.n_rows[1] : 0;
+    r[9] = it.p0[0], r[10] = it.qh[1] >= 0 ? it.p0[1] : 0;
+    r[11] = it.t0, r[12] = it.t1, r[13] = it.t2, r[14] = it.t3;
+    r[15] = it.work;
+  }
+  return SP_OK;
+}
+
 }  // extern "C"

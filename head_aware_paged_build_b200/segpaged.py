@@ -29,7 +29,7 @@ DTYPE_CODES = {"f32": SP_F32, "bf16": SP_BF16, "e4m3": SP_E4M3}
 # every symbol include/segpaged.h declares
 EXPORTED = ("segpaged_plan_create", "segpaged_plan_destroy", "segpaged_plan_sizes",
             "segpaged_plan_head_segments", "segpaged_plan_head_pages", "segpaged_plan_decode_items",
-            "segpaged_table_write",
+            "segpaged_plan_prefill_items", "segpaged_table_write",
             "build_segpaged_cache", "build_segpaged_cache_layers", "segpaged_gather", "segpaged_attention",
             "segpaged_attention_decode_noalloc", "segpaged_decode_append", "segpaged_read_device_status", "segpaged_clear_device_status", "segpaged_status_string",
             "segpaged_last_error", "segpaged_abi_version")
@@ -97,6 +97,7 @@ def load(path: Path | str | None = None) -> ctypes.CDLL:
         "segpaged_plan_head_segments": ([vp, i32, i32, ctypes.POINTER(sp_segment), i32, ctypes.POINTER(i32)], i32),
         "segpaged_plan_head_pages": ([vp, i32, i32, ctypes.POINTER(i64), i32, ctypes.POINTER(i32)], i32),
         "segpaged_plan_decode_items": ([vp, ctypes.POINTER(i32), i32, ctypes.POINTER(i32)], i32),
+        "segpaged_plan_prefill_items": ([vp, ctypes.POINTER(i32), i32, ctypes.POINTER(i32)], i32),
         "segpaged_table_write": ([vp, vp, sz, vp], i32),
         "build_segpaged_cache": ([vp, vp, vp, vp, i64, i64, i64, vp, vp, vp], i32),
         "build_segpaged_cache_layers": ([i32, ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
@@ -211,6 +212,21 @@ def segpaged_plan_decode_items(plan: int) -> list[dict]:
     _check(load().segpaged_plan_decode_items(plan, rec, n.value, ctypes.byref(n)), "segpaged_plan_decode_items")
     w = SP_DECODE_ITEM_WORDS
     return [dict(zip(DECODE_ITEM_FIELDS, rec[i * w:(i + 1) * w])) for i in range(n.value)]
+
+
+SP_PREFILL_ITEM_WORDS = 16
+PREFILL_ITEM_FIELDS = ("b", "kv", "tile", "qh0", "qh1", "q_row0", "q_row1", "n_rows0", "n_rows1", "p0_0", "p0_1",
+                       "t0", "t1", "t2", "t3", "work")
+
+
+def segpaged_plan_prefill_items(plan: int) -> list[dict]:
+    """The prefill work list of a plan, one dict per item (one CTA) in launch order."""
+    n = ctypes.c_int32()
+    _check(load().segpaged_plan_prefill_items(plan, None, 0, ctypes.byref(n)), "segpaged_plan_prefill_items")
+    rec = (ctypes.c_int32 * max(1, n.value * SP_PREFILL_ITEM_WORDS))()
+    _check(load().segpaged_plan_prefill_items(plan, rec, n.value, ctypes.byref(n)), "segpaged_plan_prefill_items")
+    w = SP_PREFILL_ITEM_WORDS
+    return [dict(zip(PREFILL_ITEM_FIELDS, rec[i * w:(i + 1) * w])) for i in range(n.value)]
 
 
 def segpaged_table_write(plan: int, d_table: int, nbytes: int, stream: int = 0) -> None:

@@ -212,6 +212,25 @@ SP_API sp_status segpaged_plan_head_pages(const sp_plan* plan, int32_t b, int32_
 #define SP_DECODE_ITEM_WORDS 12
 SP_API sp_status segpaged_plan_decode_items(const sp_plan* plan, int32_t* records, int32_t max, int32_t* count);
 
+/* Inspect the prefill work list of a plan (host only; decode plans have no
+ * prefill items).  Each item is one CTA of the prefill kernel: one or two
+ * query tiles of the same (b, kv) and the KV tiles it visits
+ * ("SegPagedAttention runtime design", §4: only KV a head can see is
+ * visited).  One record of SP_PREFILL_ITEM_WORDS int32 per item, in launch
+ * order:
+ *   [0] b   [1] kv   [2] KV tile size in tokens (128 bf16, 64 fp32)
+ *   [3], [4] q-head of query tile 0 / 1 (-1: no second tile)
+ *   [5], [6] first query row (index into q) of tile 0 / 1
+ *   [7], [8] number of rows of tile 0 / 1
+ *   [9], [10] position of the first row of tile 0 / 1
+ *   [11]..[14] visited KV tiles [t0, t1) then [t2, t3), counted in tiles of
+ *       the head's page list (tile i = pages [i * tile / page_size,
+ *       (i + 1) * tile / page_size) in segpaged_plan_head_pages order)
+ *   [15] visited KV tiles
+ * *count receives the number of items; at most `max` records are written. */
+#define SP_PREFILL_ITEM_WORDS 16
+SP_API sp_status segpaged_plan_prefill_items(const sp_plan* plan, int32_t* records, int32_t max, int32_t* count);
+
 /* Copy the plan's table blob to `d_table` (device, >= table_bytes, 16-byte
  * aligned) with an asynchronous host-to-device copy on `stream`. */
 SP_API sp_status segpaged_table_write(const sp_plan* plan, void* d_table, size_t bytes, void* stream);
