@@ -1,4 +1,4 @@
-"""Host-side pieces of bench.py that need no GPU: the sampled decode parity bookkeeping."""
+"""Host-side pieces of bench.py that need no GPU: sampled decode parity, clocks record, traffic record, rates."""
 from __future__ import annotations
 
 import sys
@@ -43,3 +43,48 @@ def test_sampled_parity_matches_and_catches_a_wrong_head():
     bad[0, wl.num_q_heads - 1] = torch.from_numpy(np.roll(bad[0, wl.num_q_heads - 1].numpy(), 1))
     _, _, _, par = bench.oracle_decode_sample(wl, dec, k, v, q, 1e9, gpu=(bad, lse))
     assert par["min_cos"] < 0.99 and par["max_abs"] > 0
+
+
+def test_clock_sampler_takes_median_max_and_active_reasons():
+    """The clocks record of the bench line, from nvidia-smi CSV rows (no GPU: a fake process)."""
+    class Fake:
+        def terminate(self):
+            pass
+
+        def communicate(self, timeout=None):
+            rows = ["1800, 1965, 900.1, 0x4, Not Active, Not Active, Not Active, Active",
+                    "1770, 1965, 950.3, 0x4, Not Active, Not Active, Not Active, Active",
+                    "1500, 1965, 990.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+                    "[N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
+                    "garbage"]
+            return "\n".join(rows), ""
+
+    cs = object.__new__(bench.ClockSampler)
+    cs.proc = Fake()
+    rec = cs.stop()
+    assert rec == {"sm_mhz": 1770.0, "sm_max_mhz": 1965.0, "samples": 3, "reasons": ["sw_power_cap"]}
+    cs.proc = None
+    assert cs.stop() is None
+
+
+def test_kernel_traffic_only_while_the_source_is_unchanged(tmp_path):
+    """DRAM bytes come from profiles/traffic.json only for the captured workload and kernel source."""
+    import json
+    rec = json.loads((bench.ROOT / "profiles" / "traffic.json").read_text())
+    csrc = bench.ROOT / "head_aware_paged_build_b200" / "csrc"
+    for kernel, src in (("decode_mma_kernel", "kernels_decode.cu"), ("prefill_tc_kernel", "kernels_prefill_tc.cu")):
+        key = rec[kernel]["workload_key"]
+        assert bench.kernel_traffic(kernel, csrc / src, key) == rec[kernel]["bytes_per_launch"]
+        assert bench.kernel_traffic(kernel, csrc / src, key + "_other") is None
+        changed = tmp_path / src
+        changed.write_bytes((csrc / src).read_bytes() + b"\n// changed\n")
+        assert bench.kernel_traffic(kernel, changed, key) is None
+    assert bench.kernel_traffic("no_such_kernel", csrc / "kernels_decode.cu", "llama_l0") is None
+
+
+def test_weak_rate_and_config():
+    assert bench.weak_rate(1e9, 4, 2.0) == 4 * 1e9 / 2e-3
+    cfg = bench.config_of(W.llama(), 1)
+    assert cfg["workload"] == "Llama-70B-shaped layer, 32K context"
+    assert cfg["heads"] == {"global": 8, "local": 56} and cfg["local_sink_window"] == [4, 8192]
+    assert cfg["parallelism"] == "single GPU" and bench.config_of(W.llama(), 8)["parallelism"] == "replicas x8"
