@@ -66,10 +66,12 @@ class SegPagedLayer:
         if t.device != self.k_pool.device:
             raise ValueError(f"{what} is on {t.device}, the layer's buffers on {self.k_pool.device}")
 
-    def _check_dense(self, k: torch.Tensor, v: torch.Tensor, varlen: bool, what: str) -> None:
+    def _check_dense(self, k: torch.Tensor, v: torch.Tensor, varlen: bool, what: str,
+                     dtype: torch.dtype | None = None) -> None:
         """Dense K/V (or gather targets): every row the plan reads or writes must lie inside."""
-        self._check_tensor(k, f"{what} K", self.torch_dtype)
-        self._check_tensor(v, f"{what} V", self.torch_dtype)
+        dtype = dtype or self.torch_dtype
+        self._check_tensor(k, f"{what} K", dtype)
+        self._check_tensor(v, f"{what} V", dtype)
         if k.shape != v.shape or k.stride() != v.stride() or k.stride(-1) != 1:
             raise ValueError(f"{what}: K and V need the same shape and strides, head_dim contiguous")
         d, hkv = self.head_dim, self.num_kv_heads
@@ -95,8 +97,10 @@ class SegPagedLayer:
                                st, self.k_pool.data_ptr(), self.v_pool.data_ptr(), _stream(stream))
 
     def gather(self, k_out: torch.Tensor, v_out: torch.Tensor, varlen: bool = False, stream=None) -> None:
-        """Write every stored row back to its dense position (the inverse of build; E4M3 pages give codes)."""
-        self._check_dense(k_out, v_out, varlen, "gather")
+        """Write every stored row back to its dense position (the inverse of build).
+
+        E4M3 pages give their 1-byte codes: k_out / v_out are then torch.uint8."""
+        self._check_dense(k_out, v_out, varlen, "gather", torch.uint8 if self.kv_dtype == "e4m3" else None)
         if varlen:
             ss, sh, st = S.SP_VARLEN, k_out.stride(1), k_out.stride(0)
         else:

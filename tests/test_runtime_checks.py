@@ -15,9 +15,11 @@ import torch
 from head_aware_paged_build_b200.runtime import SegPagedLayer, build_layers
 
 
-def fake_layer(batch=2, hq=4, hkv=2, d=128, ctx=(100, 70), dtype=torch.bfloat16, num_queries=None):
+def fake_layer(batch=2, hq=4, hkv=2, d=128, ctx=(100, 70), dtype=torch.bfloat16, num_queries=None,
+               kv_dtype=None):
     lay = object.__new__(SegPagedLayer)
     lay.torch_dtype = dtype
+    lay.kv_dtype = kv_dtype or "bf16"
     lay.batch, lay.num_q_heads, lay.num_kv_heads, lay.head_dim = batch, hq, hkv, d
     lay.ctx_len = list(ctx)
     lay.sizes = SimpleNamespace(num_queries=batch if num_queries is None else num_queries)
@@ -68,6 +70,20 @@ def test_dense_dtype_layout_and_device_are_checked():
     with pytest.raises(ValueError):  # not where the layer's buffers are
         m = torch.empty(2, 2, 100, 128, dtype=torch.bfloat16, device="meta")
         lay._check_dense(m, m, False, "build")
+
+
+def test_gather_of_e4m3_pages_takes_byte_codes():
+    """E4M3 pages gather their 1-byte codes: uint8 targets pass the checks, bf16 ones are refused."""
+    lay = fake_layer(kv_dtype="e4m3")
+    codes = torch.zeros(2, 2, 100, 128, dtype=torch.uint8)
+    lay._check_dense(codes, codes, False, "gather", torch.uint8)
+    with pytest.raises(TypeError):
+        lay.gather(dense(2, 2, 100, 128), dense(2, 2, 100, 128))
+    with pytest.raises(ValueError):  # shape still checked
+        short = torch.zeros(2, 2, 99, 128, dtype=torch.uint8)
+        lay.gather(short, short)
+    with pytest.raises(TypeError):  # build still takes the bf16 dense K/V
+        lay.build(codes, codes)
 
 
 def test_attention_refuses_wrong_q_out_lse_before_any_call():
