@@ -15,6 +15,60 @@ namespace sp {
 cudaError_t launch_prefill_f32(const PrefillLaunch& a, cudaStream_t s);
 cudaError_t launch_prefill_bf16(const PrefillLaunch& a, cudaStream_t s);
 
+sp_status check_table(const sp_plan* plan, const void* d_table) {
+  if (!plan) return fail(SP_ERR_INVALID_ARG, "plan is NULL");
+  if (!d_table || (reinterpret_cast<uintptr_t>(d_table) % 16) != 0)
+    return fail(SP_ERR_INVALID_ARG, "d_table must be a 16-byte aligned device pointer");
+  return SP_OK;
+}
+
+sp_status check_attention_args(const sp_plan* plan, const void* d_table, const void* k_pool, const void* v_pool,
+                            const void* q, const void* out, const float* lse, float softmax_scale) {
+  sp_status st = check_table(plan, d_table);
+  if (st != SP_OK) return st;
+  auto aligned_to = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; };
+  if (!k_pool || !v_pool || !q || !out) return fail(SP_ERR_INVALID_ARG, "pool, q and out must be non-NULL");
+  if (!aligned_to(k_pool, 16) || !aligned_to(v_pool, 16) || !aligned_to(q, 16) || !aligned_to(out, 16))
+    return fail(SP_ERR_INVALID_ARG, "pools, q and out must be 16-byte aligned");
+  if (lse && !aligned_to(lse, 4)) return fail(SP_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  if (!std::isfinite(softmax_scale)) return fail(SP_ERR_INVALID_ARG, "softmax_scale must be finite");
+  return SP_OK;
+}
+
+float softmax_scale_of(const sp_plan* plan, float softmax_scale) {
+  return softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(plan->prob.head_dim));
+}
+
+DecodeLaunch decode_launch_of(const sp_plan* plan, const void* d_table, const void* k_pool, const void* v_pool,
+                              const void* q, void* out, float* lse, float softmax_scale, void* scratch,
+                              int32_t* status) {
+  const float scale_log2 = softmax_scale_of(plan, softmax_scale) * 1.4426950408889634f;
+  const uint8_t* tbl = static_cast<const uint8_t*>(d_table);
+  DecodeLaunch L{};
+  L.heads = reinterpret_cast<const HeadDesc*>(tbl + plan->hdr.off_heads);
+  L.pages = reinterpret_cast<const PageDesc*>(tbl + plan->hdr.off_pages);
+  L.items = reinterpret_cast<const DecodeItem*>(tbl + plan->hdr.off_decode_items);
+  L.cta_begin = reinterpret_cast<const int32_t*>(tbl + plan->hdr.off_decode_cta);
+  L.combine = reinterpret_cast<const CombineItem*>(tbl + plan->hdr.off_combine);
+  L.n_ctas = plan->hdr.n_decode_ctas;
+  L.n_combine = plan->hdr.n_combine;
+  L.D = plan->prob.head_dim;
+  L.P = plan->prob.page_size;
+  L.group = plan->group;
+  L.num_q_heads = plan->prob.num_q_heads;
+  L.bf16 = plan->prob.dtype == SP_BF16;
+  L.page_bytes = plan->sizes.page_bytes;
+  L.pool_pages = plan->sizes.pool_pages;
+  L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
+  L.scale_log2 = plan->fp8 ? scale_log2 * plan->k_scale : scale_log2;
+  L.fp8 = plan->fp8;
+  L.v_scale = plan->fp8 ? plan->v_scale : 1.f;
+  L.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + plan->partial_offset);
+  L.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + kStatusBytes);
+  L.status = status;
+  return L;
+}
+
 namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -28,11 +82,6 @@ sp_status cuda_fail(cudaError_t e, const char* what) {
   return fail(SP_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
 }
 
-sp_status check_table(const sp_plan* plan, const void* d_table) {
-  if (!plan) return fail(SP_ERR_INVALID_ARG, "plan is NULL");
-  if (!d_table || !aligned(d_table, 16)) return fail(SP_ERR_INVALID_ARG, "d_table must be a 16-byte aligned device pointer");
-  return SP_OK;
-}
 
 sp_status pack_common(const sp_plan* plan, const void* d_table, const void* k_in, const void* v_in, void* k_out,
                       void* v_out, bool inverse, int64_t stride_seq, int64_t stride_head, int64_t stride_tok,
@@ -150,46 +199,18 @@ sp_status segpaged_attention(const sp_plan* plan, const void* d_table, const voi
                              const void* q, void* out, float* lse, float softmax_scale, void* workspace,
                              size_t workspace_bytes, void* stream) {
   using namespace sp;
-  sp_status st = check_table(plan, d_table);
+  sp_status st = check_attention_args(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale);
   if (st != SP_OK) return st;
-  if (!k_pool || !v_pool || !q || !out) return fail(SP_ERR_INVALID_ARG, "pool, q and out must be non-NULL");
-  if (!aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(q, 16) || !aligned(out, 16))
-    return fail(SP_ERR_INVALID_ARG, "pools, q and out must be 16-byte aligned");
-  if (lse && !aligned(lse, 4)) return fail(SP_ERR_INVALID_ARG, "lse must be 4-byte aligned");
   if (!workspace || !aligned(workspace, 256)) return fail(SP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   if (int64_t(workspace_bytes) < plan->sizes.workspace_bytes)
     return fail(SP_ERR_WORKSPACE, "workspace smaller than workspace_bytes");
-  if (!(softmax_scale == softmax_scale) || std::isinf(softmax_scale))
-    return fail(SP_ERR_INVALID_ARG, "softmax_scale must be finite");
-  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(plan->prob.head_dim));
-  const float scale_log2 = scale * 1.4426950408889634f;
+  const float scale_log2 = softmax_scale_of(plan, softmax_scale) * 1.4426950408889634f;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* status = static_cast<int32_t*>(workspace);
   cudaError_t e;
   if (plan->sizes.is_decode) {
-    DecodeLaunch L{};
-    L.heads = section<HeadDesc>(d_table, plan->hdr.off_heads);
-    L.pages = section<PageDesc>(d_table, plan->hdr.off_pages);
-    L.items = section<DecodeItem>(d_table, plan->hdr.off_decode_items);
-    L.cta_begin = section<int32_t>(d_table, plan->hdr.off_decode_cta);
-    L.combine = section<CombineItem>(d_table, plan->hdr.off_combine);
-    L.n_ctas = plan->hdr.n_decode_ctas;
-    L.n_combine = plan->hdr.n_combine;
-    L.D = plan->prob.head_dim;
-    L.P = plan->prob.page_size;
-    L.group = plan->group;
-    L.num_q_heads = plan->prob.num_q_heads;
-    L.bf16 = plan->prob.dtype == SP_BF16;
-    L.page_bytes = plan->sizes.page_bytes;
-    L.pool_pages = plan->sizes.pool_pages;
-    L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
-    L.scale_log2 = plan->fp8 ? scale_log2 * plan->k_scale : scale_log2;
-    L.fp8 = plan->fp8;
-    L.v_scale = plan->fp8 ? plan->v_scale : 1.f;
-    L.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + plan->partial_offset);
-    L.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
-    L.status = status;
-    e = launch_decode(L, s);
+    e = launch_decode(decode_launch_of(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale, workspace, status),
+                      s);
   } else {
     PrefillLaunch L{};
     L.heads = section<HeadDesc>(d_table, plan->hdr.off_heads);

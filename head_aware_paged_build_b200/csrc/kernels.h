@@ -68,6 +68,18 @@ struct DecodeLaunch {
 };
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t s);
 
+// Argument checks and launch set-up shared by the attention entry points
+// (segpaged_attention and the allocation-free decode), so that both refuse
+// exactly the same arguments.
+sp_status check_table(const sp_plan* plan, const void* d_table);
+sp_status check_attention_args(const sp_plan* plan, const void* d_table, const void* k_pool, const void* v_pool,
+                               const void* q, const void* out, const float* lse, float softmax_scale);
+float softmax_scale_of(const sp_plan* plan, float softmax_scale);  // <= 0 selects 1 / sqrt(head_dim)
+// Decode launch of a plan whose scratch (status block, counters, partials) starts at `scratch`.
+DecodeLaunch decode_launch_of(const sp_plan* plan, const void* d_table, const void* k_pool, const void* v_pool,
+                              const void* q, void* out, float* lse, float softmax_scale, void* scratch,
+                              int32_t* status);
+
 struct PrefillLaunch {
   const HeadDesc* heads;
   const PageDesc* pages;

@@ -12,11 +12,13 @@
 //
 // The array lives for as long as the library is loaded, once on every GPU that
 // loads it, and is shared by every call on that GPU.  It keeps the last call's
-// contents; the parts that must start at zero (the status word and the split
-// heads' arrival counters) are cleared by each call.  Calls whose kernels overlap on the GPU (different
-// streams, or different host threads, same device) race on the array and
-// corrupt each other's partial results: serialise them.
-#include <cmath>
+// contents; the part that must start at zero (the split heads' arrival
+// counters) is cleared by each call.  Device-side errors go to a status word
+// the caller owns (d_status), so that the caller can read them.  Calls whose
+// kernels overlap on the GPU (different streams, or different host threads,
+// same device) race on the array and corrupt each other's partial results:
+// serialise them.
+#include <cstdint>
 #include <mutex>
 #include <string>
 
@@ -26,30 +28,38 @@
 namespace sp {
 namespace {
 
-// Upper bound of the scratch a decode plan may need (status word + partials).
+// Upper bound of the scratch a decode plan may need (control block + partials).
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB per GPU
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
 void* g_scratch_addr[kMaxDevices] = {};
-cudaError_t g_scratch_err[kMaxDevices] = {};
-std::once_flag g_scratch_once[kMaxDevices];
+std::mutex g_scratch_mutex;
 
 // Host code cannot use &g_noalloc_scratch as a device address (it is a host
-// stand-in).  Resolve the real address once per device, with that device
-// current.
+// stand-in).  Resolve the real address with the device current, once per
+// device: only a successful lookup is kept, so a lookup that failed (for
+// example one attempted while the stream was being captured) is simply tried
+// again by the next call.
 cudaError_t scratch_address(int dev, void** out) {
-  std::call_once(g_scratch_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
     void* p = nullptr;
-    g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) {
+      *out = nullptr;
+      return e;
+    }
+    if (!p) {
+      *out = nullptr;
+      return cudaErrorInvalidSymbol;
+    }
     g_scratch_addr[dev] = p;
-  });
+  }
   *out = g_scratch_addr[dev];
-  return g_scratch_err[dev];
+  return cudaSuccess;
 }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 }  // namespace
 }  // namespace sp
@@ -58,17 +68,13 @@ extern "C" sp_status segpaged_attention_decode_noalloc(const sp_plan* plan, cons
                                                         const void* v_pool, const void* q, void* out, float* lse,
                                                         float softmax_scale, int32_t* d_status, void* stream) {
   using namespace sp;
-  if (!plan) return fail(SP_ERR_INVALID_ARG, "plan is NULL");
+  // the same argument checks as segpaged_attention, then this call's own
+  sp_status st = check_attention_args(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale);
+  if (st != SP_OK) return st;
   if (!plan->sizes.is_decode)
     return fail(SP_ERR_UNSUPPORTED, "segpaged_attention_decode_noalloc takes decode plans only");
-  if (!d_table || !k_pool || !v_pool || !q || !out)
-    return fail(SP_ERR_INVALID_ARG, "table, pools, q and out must be non-NULL");
-  if (!aligned16(d_table) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(q) || !aligned16(out))
-    return fail(SP_ERR_INVALID_ARG, "table, pools, q and out must be 16-byte aligned");
-  if ((lse && (reinterpret_cast<uintptr_t>(lse) & 3)) || (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)))
-    return fail(SP_ERR_INVALID_ARG, "lse and d_status must be 4-byte aligned");
-  if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
-    return fail(SP_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (!d_status || (reinterpret_cast<uintptr_t>(d_status) & 3))
+    return fail(SP_ERR_INVALID_ARG, "d_status must be a 4-byte aligned device int32 owned by the caller");
   if (size_t(plan->sizes.workspace_bytes) > kNoAllocScratchBytes)
     return fail(SP_ERR_WORKSPACE, "this decode plan needs " + std::to_string(plan->sizes.workspace_bytes) +
                                       " bytes of scratch; the built-in scratch holds " +
@@ -80,39 +86,16 @@ extern "C" sp_status segpaged_attention_decode_noalloc(const sp_plan* plan, cons
   if (dev < 0 || dev >= kMaxDevices) return fail(SP_ERR_UNSUPPORTED, "device index above 63");
   void* scratch = nullptr;
   e = scratch_address(dev, &scratch);
-  if (e != cudaSuccess || !scratch)
+  if (e != cudaSuccess)
     return fail(SP_ERR_CUDA, std::string("cudaGetSymbolAddress of the built-in scratch: ") + cudaGetErrorString(e));
 
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int32_t* status = d_status ? d_status : static_cast<int32_t*>(scratch);
-  // The status word and the split heads' arrival counters must start at zero
-  // (the counters return to zero by themselves unless a call was cut short).
+  // The split heads' arrival counters must start at zero (they return to zero
+  // by themselves unless a call was cut short); the partial results need no
+  // clearing.  The status block in front of them is cleared with them.
   e = cudaMemsetAsync(scratch, 0, size_t(plan->partial_offset), s);
   if (e != cudaSuccess) return fail(SP_ERR_CUDA, std::string("clearing the control block: ") + cudaGetErrorString(e));
-  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(plan->prob.head_dim));
-  const uint8_t* tbl = static_cast<const uint8_t*>(d_table);
-  DecodeLaunch L{};
-  L.heads = reinterpret_cast<const HeadDesc*>(tbl + plan->hdr.off_heads);
-  L.pages = reinterpret_cast<const PageDesc*>(tbl + plan->hdr.off_pages);
-  L.items = reinterpret_cast<const DecodeItem*>(tbl + plan->hdr.off_decode_items);
-  L.cta_begin = reinterpret_cast<const int32_t*>(tbl + plan->hdr.off_decode_cta);
-  L.combine = reinterpret_cast<const CombineItem*>(tbl + plan->hdr.off_combine);
-  L.n_ctas = plan->hdr.n_decode_ctas;
-  L.n_combine = plan->hdr.n_combine;
-  L.D = plan->prob.head_dim;
-  L.P = plan->prob.page_size;
-  L.group = plan->group;
-  L.num_q_heads = plan->prob.num_q_heads;
-  L.bf16 = plan->prob.dtype == SP_BF16;
-  L.page_bytes = plan->sizes.page_bytes;
-  L.pool_pages = plan->sizes.pool_pages;
-  L.kpool = k_pool, L.vpool = v_pool, L.q = q, L.out = out, L.lse = lse;
-  L.scale_log2 = scale * 1.4426950408889634f * (plan->fp8 ? plan->k_scale : 1.f);
-  L.fp8 = plan->fp8;
-  L.v_scale = plan->fp8 ? plan->v_scale : 1.f;
-  L.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + plan->partial_offset);
-  L.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + kStatusBytes);
-  L.status = status;
-  e = launch_decode(L, s);
+  e = launch_decode(decode_launch_of(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale, scratch, d_status),
+                    s);
   return e == cudaSuccess ? SP_OK : fail(SP_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
 }

@@ -31,7 +31,8 @@ EXPORTED = ("segpaged_plan_create", "segpaged_plan_destroy", "segpaged_plan_size
             "segpaged_plan_head_segments", "segpaged_plan_head_pages", "segpaged_plan_decode_items",
             "segpaged_plan_prefill_items", "segpaged_table_write",
             "build_segpaged_cache", "build_segpaged_cache_layers", "segpaged_gather", "segpaged_attention",
-            "segpaged_attention_decode_noalloc", "segpaged_decode_append", "segpaged_read_device_status", "segpaged_clear_device_status", "segpaged_status_string",
+            "segpaged_attention_decode_noalloc", "segpaged_decode_append", "segpaged_read_device_status",
+            "segpaged_clear_device_status", "segpaged_eval_exp2_fma", "segpaged_status_string",
             "segpaged_last_error", "segpaged_abi_version")
 
 
@@ -108,6 +109,7 @@ def load(path: Path | str | None = None) -> ctypes.CDLL:
         "segpaged_decode_append": ([vp, vp, vp, vp, i64, i64, vp, vp, vp, vp], i32),
         "segpaged_read_device_status": ([vp, ctypes.POINTER(i32), vp], i32),
         "segpaged_clear_device_status": ([vp, vp], i32),
+        "segpaged_eval_exp2_fma": ([vp, vp, i64, vp], i32),
         "segpaged_status_string": ([i32], ctypes.c_char_p),
         "segpaged_last_error": ([], ctypes.c_char_p),
         "segpaged_abi_version": ([], i32),
@@ -262,9 +264,11 @@ def segpaged_attention(plan: int, d_table: int, k_pool: int, v_pool: int, q: int
 
 
 def segpaged_attention_decode_noalloc(plan: int, d_table: int, k_pool: int, v_pool: int, q: int, out: int,
-                                      lse: int | None, softmax_scale: float, d_status: int | None = None,
+                                      lse: int | None, softmax_scale: float, d_status: int,
                                       stream: int = 0) -> None:
-    """Decode attention with the library's built-in scratch (no workspace argument, no allocation)."""
+    """Decode attention with the library's built-in scratch (no workspace argument, no allocation).
+
+    ``d_status`` is the caller's device int32 that receives the device status code."""
     _check(load().segpaged_attention_decode_noalloc(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale,
                                                     d_status, stream), "segpaged_attention_decode_noalloc")
 
@@ -291,6 +295,11 @@ def segpaged_read_device_status(workspace: int, stream: int = 0) -> int:
 
 def segpaged_clear_device_status(workspace: int, stream: int = 0) -> None:
     _check(load().segpaged_clear_device_status(workspace, stream), "segpaged_clear_device_status")
+
+
+def segpaged_eval_exp2_fma(d_x: int, d_y: int, n: int, stream: int = 0) -> None:
+    """y = the prefill kernel's FMA-pipe 2^x of x (device float arrays of n elements)."""
+    _check(load().segpaged_eval_exp2_fma(d_x, d_y, n, stream), "segpaged_eval_exp2_fma")
 
 
 def segpaged_abi_version() -> int:

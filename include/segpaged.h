@@ -26,7 +26,9 @@
  *  - Supported: head_dim 64 or 128; dtype fp32 with page size 16 or 64; dtype
  *    bf16 with page size 64 (pages bf16, or FP8 E4M3 for decode plans);
  *    num_q_heads / num_kv_heads <= 16.  Anything else returns
- *    SP_ERR_UNSUPPORTED.
+ *    SP_ERR_UNSUPPORTED.  bf16 pages are 64 tokens only: the kernels stage a
+ *    page as one 128-byte-swizzled tensor-core operand of 64 rows (the pages'
+ *    own runtime uses page size 64, "SegPagedAttention runtime design", §6).
  */
 #ifndef SEGPAGED_H_
 #define SEGPAGED_H_
@@ -183,10 +185,21 @@ typedef struct sp_plan sp_plan;
  * The plan is immutable and may be shared by several streams. */
 SP_API sp_status segpaged_plan_create(const sp_problem* problem, sp_plan** out);
 SP_API void segpaged_plan_destroy(sp_plan* plan);
+
+/* Sizes of a plan's buffers and its ledger ("SegPagedAttention runtime
+ * design", §3: the per-head page table decides how many pages each head owns;
+ * §5 and the closing summary: KV savings = 1 - stored / dense).  Host only;
+ * fills *out with the fields of sp_sizes: pages each pool must hold, table and
+ * workspace bytes, stored and dense token-heads, visible (query, key) pairs
+ * (the prefill FLOP ledger is 4 * head_dim * visible_pairs) and the launch
+ * shape.  SP_ERR_INVALID_ARG if plan or out is NULL. */
 SP_API sp_status segpaged_plan_sizes(const sp_plan* plan, sp_sizes* out);
 
-/* Inspect the segments / physical page ids of (b, kv).  *count receives the
- * number available; at most `max` are written. */
+/* Inspect the segments / physical page ids of (b, kv) ("SegPagedAttention
+ * runtime design", §3: (layer, head, segment) -> contiguous virtual pages ->
+ * physical pages).  Host only.  *count receives the number available; at most
+ * `max` are written (segs / page_ids may be NULL when max is 0).
+ * SP_ERR_INVALID_ARG for a NULL plan or count, or (b, kv) out of range. */
 SP_API sp_status segpaged_plan_head_segments(const sp_plan* plan, int32_t b, int32_t kv,
                                       sp_segment* segs, int32_t max, int32_t* count);
 SP_API sp_status segpaged_plan_head_pages(const sp_plan* plan, int32_t b, int32_t kv, int64_t* page_ids,
@@ -231,8 +244,16 @@ SP_API sp_status segpaged_plan_decode_items(const sp_plan* plan, int32_t* record
 #define SP_PREFILL_ITEM_WORDS 16
 SP_API sp_status segpaged_plan_prefill_items(const sp_plan* plan, int32_t* records, int32_t max, int32_t* count);
 
-/* Copy the plan's table blob to `d_table` (device, >= table_bytes, 16-byte
- * aligned) with an asynchronous host-to-device copy on `stream`. */
+/* Upload the SegmentPageTable ("SegPagedAttention runtime design", §3: page
+ * ids per head segment plus per-head policy, built once when KV is written;
+ * §5: never rebuilt per attention call).  Copies the plan's table blob to
+ * `d_table` (device, caller-owned, >= table_bytes, 16-byte aligned) with one
+ * asynchronous host-to-device copy on `stream`; the host plan stays valid and
+ * unchanged.  The blob holds the heads' descriptors, their page records and
+ * the decode / prefill work lists.  SP_ERR_WORKSPACE if `bytes` is smaller
+ * than table_bytes, SP_ERR_INVALID_ARG for a NULL or misaligned pointer,
+ * SP_ERR_CUDA if the copy cannot be enqueued.  Writing it again restores a
+ * table that segpaged_decode_append has advanced. */
 SP_API sp_status segpaged_table_write(const sp_plan* plan, void* d_table, size_t bytes, void* stream);
 
 /* build_segpaged_cache ("SegPagedAttention runtime design", §3: build the
@@ -270,10 +291,14 @@ SP_API sp_status build_segpaged_cache_layers(int32_t n_layers, const sp_plan* co
                                              const void* const* v_dense, int64_t stride_seq, int64_t stride_head,
                                              int64_t stride_tok, void* k_pool, void* v_pool, void* stream);
 
-/* Inverse of build_segpaged_cache, for checking: writes each stored row back
- * into dense-shaped k_out / v_out (same addressing rules); rows that are not
- * stored are left untouched.  With SP_E4M3 pages it writes the 1-byte codes
- * (strides then count bytes). */
+/* Inverse of build_segpaged_cache, for checking the packing bit for bit
+ * ("SegPagedAttention runtime design", §3: each head's store holds exactly
+ * the tokens it can see; §4: the result is verified against a dense
+ * baseline).  Writes each stored (b, kv, position) row of the pools back into
+ * dense-shaped k_out / v_out (device, caller-owned; same addressing rules and
+ * alignment checks as build_segpaged_cache); rows that are not stored are left
+ * untouched.  With SP_E4M3 pages it writes the 1-byte codes (strides then
+ * count bytes).  Errors as build_segpaged_cache. */
 SP_API sp_status segpaged_gather(const sp_plan* plan, const void* d_table, const void* k_pool,
                           const void* v_pool, void* k_out, void* v_out, int64_t stride_seq,
                           int64_t stride_head, int64_t stride_tok, void* stream);
@@ -306,24 +331,29 @@ SP_API sp_status segpaged_attention(const sp_plan* plan, const void* d_table, co
  * call above.)  Some callers cannot hand this library a workspace: engines
  * whose device memory is divided into a fixed arena before serving starts,
  * and latency-critical loops that must not call cudaMalloc because it can
- * synchronise the device.  This call runs the same split-KV decode and
- * combine kernels as segpaged_attention on a decode plan, but takes their
- * scratch (status word + partial results) from a 4 MiB array built into the
+ * synchronise the device.  This call runs the same split-KV decode kernels as
+ * segpaged_attention on a decode plan, but takes their scratch (split heads'
+ * arrival counters + partial results) from a 4 MiB array built into the
  * library's device image, one per GPU, held until the process exits.  It
- * calls no cudaMalloc, cudaFree or allocating library routine.
+ * calls no cudaMalloc, cudaFree or allocating library routine.  For the same
+ * plan and inputs its output is bit for bit that of segpaged_attention.
  *   - Decode plans only (SP_ERR_UNSUPPORTED otherwise).  A plan whose
  *     workspace_bytes exceed 4 MiB is rejected with SP_ERR_WORKSPACE before
  *     any launch (lower target_ctas, or use segpaged_attention).
  *   - It runs on the current CUDA device.  The first call on a device looks
  *     up the array's device address (cudaGetSymbolAddress) with that device
- *     current; make that first call before any stream capture.
+ *     current; make that first call before any stream capture.  A lookup
+ *     that fails is reported (SP_ERR_CUDA) and tried again by the next call.
  *   - All calls on one GPU share the array and leave their contents in it.
- *     Each call clears the status word and the split heads' arrival
- *     counters; the partial results need no clearing.  Calls whose kernels overlap on the GPU race on the array:
- *     serialise them.
- *   - d_status: NULL, or a device int32 the caller owns (and clears) that
- *     receives the device status code instead of the built-in word.
- * Other arguments as segpaged_attention. */
+ *     Each call clears the split heads' arrival counters; the partial results
+ *     need no clearing.  Calls whose kernels overlap on the GPU race on the
+ *     array: serialise them.
+ *   - d_status: required, a 4-byte aligned device int32 the caller owns (a
+ *     word of its arena) that receives the device status code (the codes of
+ *     segpaged_read_device_status; the first error sticks).  The call does not
+ *     clear it: the caller zeroes it once and again after reading an error.
+ *     NULL returns SP_ERR_INVALID_ARG.
+ * Other arguments as segpaged_attention, checked the same way. */
 SP_API sp_status segpaged_attention_decode_noalloc(const sp_plan* plan, const void* d_table, const void* k_pool,
                                                    const void* v_pool, const void* q, void* out, float* lse,
                                                    float softmax_scale, int32_t* d_status, void* stream);
@@ -346,17 +376,32 @@ SP_API sp_status segpaged_decode_append(const sp_plan* plan, void* d_table, cons
                                         int64_t stride_seq, int64_t stride_head, void* k_pool, void* v_pool,
                                         void* workspace, void* stream);
 
-/* Device status word: kernels never trap; a failed device-side check or a
- * bounded wait that ran out records a non-zero code (the first one sticks):
+/* Device status word.  The pages have no counterpart: this is the failure
+ * detection of this library's kernels.  Kernels never trap; a failed
+ * device-side check or a bounded wait that ran out records a non-zero code in
+ * the first int32 of the workspace (the first one sticks):
  *   1, 2  a wait on a page copy (full / empty stage) ran out
  *   3     a wait on the tensor cores ran out      4  a wait on the softmax ran out
  *   5     a page id in the device table lies outside [0, pool_pages): the
  *         kernel read or wrote nothing there (a corrupted table)
  *   6     a ring append found no reserved page left (the append was skipped)
- * read synchronises `stream` and returns the code in *code (0 = no error);
- * clear zeroes it. */
+ * read synchronises `stream`, copies the word to *code (host) and returns
+ * SP_OK for 0, SP_ERR_DEVICE_CHECK for a recorded code (SP_ERR_CUDA if the
+ * synchronisation or the copy fails); clear zeroes the word's 256-byte block
+ * asynchronously on `stream`.  `workspace` is the one given to the kernels. */
 SP_API sp_status segpaged_read_device_status(const void* workspace, int32_t* code, void* stream);
 SP_API sp_status segpaged_clear_device_status(void* workspace, void* stream);
+
+/* segpaged_eval_exp2_fma: y[i] = 2^x[i] as the bf16 prefill kernel computes
+ * it on the FMA pipe for one exponent pair in sixteen (the pages have no
+ * counterpart: it is this library's own 2^x, a cubic on [-1/2, 1/2] fitted by
+ * relative-error least squares, maximum relative error 7.8e-5 in fp32 for
+ * x in [-125, 8], below the 2^-8 rounding of P to bf16; x below -126,
+ * including -inf, gives a value in [0, 2^-125]).  Exposed so that the bound
+ * can be tested on the device that runs the kernel.  d_x, d_y: device,
+ * caller-owned, n floats each, 4-byte aligned; enqueued on `stream`.
+ * SP_ERR_INVALID_ARG for n < 0 or bad pointers. */
+SP_API sp_status segpaged_eval_exp2_fma(const float* d_x, float* d_y, int64_t n, void* stream);
 
 SP_API const char* segpaged_status_string(sp_status status);
 SP_API const char* segpaged_last_error(void);
