@@ -25,9 +25,20 @@ MUTANTS = {
     "scale_dropped": ("s[j] = scale * acc;", "s[j] = acc;"),
     "values_from_keys": ("o[t] += e * v[j * d + t];", "o[t] += e * k[j * d + t];"),
     "transposed_key_index": ("acc += qr[t] * k[j * d + t];", "acc += qr[t] * k[t * d + j % d];"),
-    "lse_without_max": ("lse[r] = m + log(denom);", "lse[r] = log(denom);"),
-    "dense_treated_as_local": ("if (kind != ORACLE_LOCAL) return 1;", "if (kind == ORACLE_GLOBAL) return 1;"),
+    "lse_without_max": ("*lse = m + log(denom);", "*lse = log(denom);"),
+    "dense_treated_as_local": ("if (kind == ORACLE_GLOBAL || kind == ORACLE_DENSE) return 1;",
+                               "if (kind == ORACLE_GLOBAL) return 1;"),
     "stored_only_last_query": ("for (int64_t p = q0; p < L && !keep; ++p)", "for (int64_t p = L - 1; p < L && !keep; ++p)"),
+    # RETRIEVAL heads: visibility of kept blocks and the top-p block selection
+    "retrieval_kept_blocks_ignored": ("return kind == ORACLE_RETRIEVAL && sel[j / block] != 0;", "return 0;"),
+    "retrieval_kept_block_shifted": ("&& sel[j / block] != 0;", "&& sel[(j + 1) / block] != 0;"),
+    "retrieval_ties_to_higher_block": ("if (best < 0 || mass[i] > mass[best]) best = i;",
+                                       "if (best < 0 || mass[i] >= mass[best]) best = i;"),
+    "retrieval_least_important_first": ("mass[i] > mass[best]", "mass[i] < mass[best]"),
+    "retrieval_threshold_strict": ("if (run >= target) {", "if (run > target) {"),
+    "retrieval_sink_blocks_are_candidates": ("if (taken[i] || (i + 1) * block <= sink) continue;",
+                                             "if (taken[i]) continue;"),
+    "retrieval_top_p_one_drops_empty_blocks": ("} else if (top_p < 1.0f) {", "} else if (top_p <= 1.0f) {"),
     # FP8 E4M3 encoder / decoder
     "e4m3_bias_8": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
     "e4m3_subnormal_step": ("ldexp((double)m, -9)", "ldexp((double)m, -10)"),

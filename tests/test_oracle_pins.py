@@ -139,6 +139,31 @@ def test_equal_keys_average_visible_values_and_count(sink, window):
         np.testing.assert_allclose(out[i, 2:], v[vis, 2:].mean(0), rtol=0, atol=1e-12)
 
 
+def test_batched_rows_of_mixed_groups_match_brute_force():
+    """The batched call (many groups, each with its own context length and policy) against brute force,
+    and bit for bit against one call per group (each row is computed by the same code whichever call runs it)."""
+    rng = np.random.default_rng(21)
+    d = 8
+    groups = []
+    for gi, (kind, sink, window) in enumerate(POLICIES):
+        L = 5 + 7 * gi
+        q0 = max(0, L - 1 - 3 * gi)
+        groups.append((_rand(rng, L - q0, d), np.arange(q0, L), _rand(rng, L, d), _rand(rng, L, d), kind, sink,
+                       window))
+    res = oracle.attention_batch(groups)
+    scale = 1.0 / math.sqrt(d)
+    for (q, pos, k, v, kind, sink, window), (out, lse) in zip(groups, res):
+        for i, p in enumerate(pos):
+            bo, bl = brute.attention_row(q[i].tolist(), k.tolist(), v.tolist(), kind, sink, window, int(p), scale)
+            np.testing.assert_allclose(out[i], bo, rtol=0, atol=1e-12)
+            assert abs(lse[i] - bl) <= 1e-12
+        o1, l1 = oracle.attention_rows(q, pos, k, v, kind, sink, window)
+        assert np.array_equal(o1, out) and np.array_equal(l1, lse)
+    with pytest.raises(ValueError):
+        q, pos, k, v, kind, sink, window = groups[0]
+        oracle.attention_batch([(q, pos + 100, k, v, kind, sink, window)])
+
+
 def test_gqa_equals_mha_with_repeated_kv_heads():
     """Query head h uses kv-head h // g: repeating each kv-head g times gives the same result."""
     rng = np.random.default_rng(11)
@@ -289,3 +314,108 @@ def test_e4m3_every_midpoint_goes_to_the_even_neighbour():
     c = oracle.e4m3_encode(x, 1.0)
     best = np.abs(x[:, None].astype(np.float64) - np.concatenate([vals, -vals])[None, :]).min(1)
     assert np.all(np.abs(x.astype(np.float64) - oracle.e4m3_decode(c, 1.0)) == best)
+
+
+# ---------------------------------------------------------------------------
+# RETRIEVAL heads: sink + recent window + the top-p blocks by importance
+# ---------------------------------------------------------------------------
+
+def _masses(rng, n, integer):
+    return (rng.integers(0, 6, n) if integer else rng.exponential(1.0, n)).astype(np.float32)
+
+
+@pytest.mark.parametrize("integer", [True, False])
+@pytest.mark.parametrize("top_p", [0.0, 0.25, 0.5, 0.7, 0.9, 1.0])
+@pytest.mark.parametrize("L,block,sink", [(1, 4, 0), (13, 4, 0), (29, 4, 3), (32, 8, 8), (40, 8, 11), (37, 16, 0)])
+def test_retrieval_selection_matches_exhaustive_search(integer, top_p, L, block, sink):
+    """The kept blocks are the fewest whose importance reaches top_p of the total (exhaustive search)."""
+    rng = np.random.default_rng(hash((integer, top_p, L, block, sink)) % (1 << 32))
+    n = -(-L // block)
+    for _ in range(4):
+        mass = _masses(rng, n, integer)
+        sel = oracle.retrieval_select(L, block, sink, top_p, mass)
+        want = brute.kept_blocks(L, block, sink, float(np.float32(top_p)), [float(x) for x in mass])
+        assert set(np.flatnonzero(sel).tolist()) == want, (mass, top_p)
+
+
+def test_retrieval_selection_closed_forms():
+    """Uniform importance keeps ceil(top_p * candidates) blocks, lowest first; a single heavy block is kept alone."""
+    for n_cand, top_p in [(10, 0.25), (10, 0.5), (7, 0.75), (16, 0.5), (5, 1.0), (5, 0.0)]:
+        L, block, sink = 64 * (n_cand + 1), 64, 64  # block 0 is all sink: not a candidate
+        sel = oracle.retrieval_select(L, block, sink, top_p, np.ones(n_cand + 1, np.float32))
+        k = math.ceil(top_p * n_cand)
+        assert not sel[0] and sel.sum() == k and np.array_equal(np.flatnonzero(sel), np.arange(1, k + 1))
+    mass = np.zeros(9, np.float32)
+    mass[6] = 3.5
+    for top_p in (0.01, 0.5, 0.99):
+        assert np.flatnonzero(oracle.retrieval_select(9 * 32, 32, 4, top_p, mass)).tolist() == [6]
+    with pytest.raises(ValueError):
+        oracle.retrieval_select(64, 32, 0, 0.5, np.array([1.0, -1.0], np.float32))
+    with pytest.raises(ValueError):
+        oracle.retrieval_select(64, 32, 0, 0.5, np.array([1.0, np.inf], np.float32))
+
+
+@pytest.mark.parametrize("top_p", [0.3, 0.6, 0.95])
+@pytest.mark.parametrize("sink,window", [(0, 1), (2, 3), (4, 8), (9, 2)])
+@pytest.mark.parametrize("L,q0,block", [(17, 0, 4), (33, 20, 4), (40, 39, 8), (29, 10, 8)])
+def test_retrieval_attention_matches_brute_force(top_p, sink, window, L, q0, block):
+    rng = np.random.default_rng(L * 1000 + q0 * 10 + sink + window)
+    d = 8
+    q, k, v = _rand(rng, L - q0, d), _rand(rng, L, d), _rand(rng, L, d)
+    mass = _masses(rng, -(-L // block), False)
+    sel = oracle.retrieval_select(L, block, sink, top_p, mass)
+    kept = set(np.flatnonzero(sel).tolist())
+    pos = np.arange(q0, L)
+    out, lse = oracle.attention_rows(q, pos, k, v, "retrieval", sink, window, sel=sel, block=block)
+    scale = 1.0 / math.sqrt(d)
+    for i, p in enumerate(pos):
+        bo, bl = brute.attention_row(q[i].tolist(), k.tolist(), v.tolist(), "retrieval", sink, window, int(p), scale,
+                                     kept, block)
+        np.testing.assert_allclose(out[i], bo, rtol=0, atol=1e-12)
+        assert abs(lse[i] - bl) <= 1e-12
+    # the stored set is the union of the rows' visible sets, the pair count their sizes
+    stored = oracle.stored_mask("retrieval", sink, window, L, q0, sel=sel, block=block)
+    assert set(np.flatnonzero(stored).tolist()) == brute.stored_positions("retrieval", sink, window, L, q0, kept,
+                                                                          block)
+    pairs = sum(len(brute.visible_positions("retrieval", sink, window, int(p), kept, block)) for p in pos)
+    assert oracle.visible_pairs("retrieval", sink, window, L, q0, sel=sel, block=block) == pairs
+
+
+@pytest.mark.parametrize("sink,window", [(0, 1), (4, 8), (3, 100)])
+def test_retrieval_top_p_one_is_global_and_zero_is_local(sink, window):
+    rng = np.random.default_rng(31 + sink)
+    L, d, block, q0 = 70, 16, 8, 30
+    q, k, v = _rand(rng, L - q0, d), _rand(rng, L, d), _rand(rng, L, d)
+    mass = _masses(rng, -(-L // block), False)
+    mass[3] = 0.0  # a zero-importance block is still kept at top_p = 1
+    pos = np.arange(q0, L)
+    s1 = oracle.retrieval_select(L, block, sink, 1.0, mass)
+    o1, l1 = oracle.attention_rows(q, pos, k, v, "retrieval", sink, window, sel=s1, block=block)
+    og, lg = oracle.attention_rows(q, pos, k, v, "global", 0, 0)
+    assert np.array_equal(o1, og) and np.array_equal(l1, lg)
+    s0 = oracle.retrieval_select(L, block, sink, 0.0, mass)
+    assert not s0.any()
+    o0, l0 = oracle.attention_rows(q, pos, k, v, "retrieval", sink, window, sel=s0, block=block)
+    ol, ll = oracle.attention_rows(q, pos, k, v, "local", sink, window)
+    assert np.array_equal(o0, ol) and np.array_equal(l0, ll)
+
+
+def test_retrieval_equal_keys_average_the_kept_values():
+    """All keys equal: every visible weight is the same, so O is the mean of the visible values and
+    |V(p)| = (kept or sink positions before the window) + (window positions up to p)."""
+    rng = np.random.default_rng(44)
+    L, d, block, sink, window = 48, 4, 8, 2, 5
+    k = np.tile(_rand(rng, 1, d), (L, 1))
+    v = _rand(rng, L, d)
+    q = _rand(rng, L, d)
+    mass = np.array([0, 9, 0, 4, 0, 1], np.float32)
+    sel = oracle.retrieval_select(L, block, sink, 0.9, mass)
+    assert np.flatnonzero(sel).tolist() == [1, 3]  # 9 + 4 = 13 >= 0.9 * 14
+    out, lse = oracle.attention_rows(q, np.arange(L), k, v, "retrieval", sink, window, sel=sel, block=block)
+    for p in range(L):
+        lo = max(0, p - window + 1)
+        early = [j for j in range(lo) if j < sink or sel[j // block]]
+        vis = early + list(range(lo, p + 1))
+        np.testing.assert_allclose(out[p], v[vis].mean(0), rtol=0, atol=1e-12)
+        s0 = float(q[p] @ k[0]) / math.sqrt(d)
+        assert abs(lse[p] - (s0 + math.log(len(vis)))) < 1e-12
