@@ -339,9 +339,14 @@ def run_ours(args) -> None:
         "wall_s_timed": round(wall, 3),
     }
     if world == 1 and not args.no_cpu_baseline:
-        Ld.attention(qd, od, lsed)  # the measured decode's output, checked on the oracle's sample
+        Ld.attention(qd, od, lsed)  # the measured kernels' outputs, checked on the oracle's samples
+        if has_pre:
+            Lp.attention(qp, op, lsep)
         torch.cuda.synchronize()
-        line["cpu_baseline"] = cpu_baseline(wl, dec, k, v, qd, args.cpu_seconds, gpu=(od, lsed))
+        line["cpu_baseline"] = cpu_baseline(wl, dec, k, v, qd, args.cpu_seconds, gpu=(od, lsed),
+                                            pre=pre, qp=qp if has_pre else None,
+                                            gpu_pre=(op, lsep) if has_pre else None,
+                                            prefill_full=args.cpu_prefill_full)
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -469,57 +474,177 @@ def run_e2e_dense(args, dev, layer, k, v, qd, od, lsed, world) -> dict:
             "path": "pinned host K/V/Q -> build_segpaged_cache -> segpaged_attention (decode) -> host O, LSE"}
 
 
-def oracle_decode_sample(wl, dec, k, v, qd, budget_s: float, max_heads: int | None = None,
+def host_cores() -> int:
+    """Host cores this process may run on (its CPU affinity), the oracle's OpenMP default."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _f64(t):
+    return t.double().cpu().numpy()
+
+
+def _cos(a, r) -> float:
+    import numpy as np
+    return float(a.ravel() @ r.ravel() / (np.linalg.norm(a) * np.linalg.norm(r)))
+
+
+def oracle_decode_sample(wl, dec, k, v, qd, budget_s: float, max_groups: int | None = None,
                          gpu: tuple | None = None) -> tuple[float, int, int, dict | None]:
     """Run the CPU oracle on whole (sequence, kv-head) groups until the time budget is spent.
 
-    Returns (seconds spent inside the oracle, visible KV bytes covered, groups done, parity), where
-    parity compares the GPU decode output `gpu` = (out, lse) with the oracle on the same groups
-    (per q-head cosine and max abs error of O, max abs error of LSE), or is None without `gpu`.
+    Groups go to the oracle several at a time in one batched call, so that every host core
+    works on their rows (one decode row per q-head).  Returns (seconds spent inside the
+    oracle, visible KV bytes covered, groups done, parity), where parity compares the GPU
+    decode output `gpu` = (out, lse) with the oracle on the same groups (per q-head cosine and
+    max abs error of O, max abs error of LSE), or is None without `gpu`.
     """
     import numpy as np
 
     import oracle
 
-    spent, vis, groups = 0.0, 0, 0
+    spent, vis, done = 0.0, 0, 0
     cos_min, abs_max, lse_max = 1.0, 0.0, 0.0
     if gpu is not None:
-        gout, glse = gpu[0].double().cpu().numpy(), gpu[1].double().cpu().numpy()
+        gout, glse = _f64(gpu[0]), _f64(gpu[1])
     order = [(b, kv) for b in range(wl.batch) for kv in range(wl.num_kv_heads)]
-    for b, kv in order:
-        if spent >= budget_s or (max_heads is not None and groups >= max_heads):
+    if max_groups is not None:
+        order = order[:max_groups]
+    per_call = max(1, int(1.5e9 // (2 * max(dec.ctx_lens) * wl.head_dim * 8)))  # <= 1.5 GB of fp64 K/V per call
+    for c0 in range(0, len(order), per_call):
+        if spent >= budget_s:
             break
-        L = dec.ctx_lens[b]
-        kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
-        kk = k[b, kv, :L].double().cpu().numpy()
-        vv = v[b, kv, :L].double().cpu().numpy()
-        qq = qd[b, kv * wl.group:(kv + 1) * wl.group].double().cpu().numpy()
+        chunk = order[c0:c0 + per_call]
+        groups = []
+        for b, kv in chunk:
+            L = dec.ctx_lens[b]
+            kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+            groups.append((_f64(qd[b, kv * wl.group:(kv + 1) * wl.group]), [L - 1] * wl.group,
+                           _f64(k[b, kv, :L]), _f64(v[b, kv, :L]), kind, s, w))
         t0 = time.perf_counter()
-        # the group's q-heads share the kv-head: one call, one query row per q-head (OpenMP over rows)
-        o_ref, l_ref = oracle.attention_rows(qq, [L - 1] * wl.group, kk, vv, kind, s, w)
+        res = oracle.attention_batch(groups)
         spent += time.perf_counter() - t0
-        vis += int(oracle.stored_mask(kind, s, w, L, L - 1).sum()) * 2 * wl.head_dim * 2
-        groups += 1
-        if gpu is not None:
-            for i in range(wl.group):
-                a, r = gout[b, kv * wl.group + i], o_ref[i]
-                cos_min = min(cos_min, float(a @ r / (np.linalg.norm(a) * np.linalg.norm(r))))
-                abs_max = max(abs_max, float(np.max(np.abs(a - r))))
-                lse_max = max(lse_max, abs(float(glse[b, kv * wl.group + i]) - float(l_ref[i])))
+        for (b, kv), (o_ref, l_ref), gr in zip(chunk, res, groups):
+            L = dec.ctx_lens[b]
+            vis += int(oracle.stored_mask(gr[4], gr[5], gr[6], L, L - 1).sum()) * 2 * wl.head_dim * 2
+            done += 1
+            if gpu is not None:
+                for i in range(wl.group):
+                    a, r = gout[b, kv * wl.group + i], o_ref[i]
+                    cos_min = min(cos_min, _cos(a, r))
+                    abs_max = max(abs_max, float(np.max(np.abs(a - r))))
+                    lse_max = max(lse_max, abs(float(glse[b, kv * wl.group + i]) - float(l_ref[i])))
     parity = ({"min_cos": round(cos_min, 7), "max_abs": float(f"{abs_max:.3g}"), "max_lse_abs": float(f"{lse_max:.3g}"),
-               "heads": groups * wl.group, "against": "fp64 oracle, same inputs"} if gpu is not None else None)
-    return spent, vis, groups, parity
+               "heads": done * wl.group, "against": "fp64 oracle, same inputs"} if gpu is not None else None)
+    return spent, vis, done, parity
 
 
-def cpu_baseline(wl, dec, k, v, qd, budget_s: float, gpu: tuple | None = None) -> dict:
+def oracle_prefill_sample(wl, pre, k, v, qp, budget_s: float, full: bool = False, rows_per_head: int = 48,
+                          gpu: tuple | None = None) -> dict:
+    """The CPU oracle on the prefill chunk: visible-pair FLOPs per second of host time.
+
+    Groups (sequence, kv-head) are taken in a seeded random order; from each, `rows_per_head`
+    seeded random rows of every q-head of the group (all rows with `full`), several groups per
+    batched oracle call, until the time budget is spent (or, with `full`, every row is done).
+    The rate counts 4 * head_dim FLOPs per visible (query, key) pair, as the GPU prefill's;
+    the time of the whole chunk is that work divided by the rate (extrapolated unless `full`).
+    With `gpu` = (out, lse) of the GPU prefill the same rows are compared with the oracle.
+    """
+    import numpy as np
+
+    import oracle
+
+    rng = np.random.default_rng(12345)
+    order = [(b, kv) for b in range(wl.batch) for kv in range(wl.num_kv_heads)]
+    order = [order[i] for i in rng.permutation(len(order))]
+    off = pre.q_offsets
+    per_call = max(1, int(1.5e9 // (2 * max(pre.ctx_lens) * wl.head_dim * 8)))
+    spent, pairs, rows_done, done = 0.0, 0, 0, 0
+    cos_min, abs_max, lse_max = 1.0, 0.0, 0.0
+    if gpu is not None:
+        gout, glse = gpu
+    for c0 in range(0, len(order), per_call):
+        if spent >= budget_s and not full:
+            break
+        chunk = order[c0:c0 + per_call]
+        groups, meta = [], []
+        for b, kv in chunk:
+            L, q0 = pre.ctx_lens[b], pre.q_starts[b]
+            C = L - q0
+            kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+            rows = np.arange(C) if full else np.sort(rng.choice(C, min(C, rows_per_head), replace=False))
+            kk, vv = _f64(k[b, kv, :L]), _f64(v[b, kv, :L])
+            for h in range(kv * wl.group, (kv + 1) * wl.group):
+                idx = torch_index(off[b] + rows, qp.device)
+                groups.append((_f64(qp[idx, h]), q0 + rows, kk, vv, kind, s, w))
+                meta.append((b, h, rows, kind, s, w))
+        t0 = time.perf_counter()
+        res = oracle.attention_batch(groups)
+        spent += time.perf_counter() - t0
+        done += len(chunk)
+        for (b, h, rows, kind, s, w), (o_ref, l_ref) in zip(meta, res):
+            q0 = pre.q_starts[b]
+            pos = q0 + rows
+            if kind == "local":  # |visible(p)| = min(p + 1, s + w); global: p + 1
+                pairs += int(np.minimum(pos + 1, s + w).sum())
+            else:
+                pairs += int((pos + 1).sum())
+            rows_done += len(rows)
+            if gpu is not None:
+                idx = torch_index(off[b] + rows, gout.device)
+                a = _f64(gout[idx, h])
+                cos_min = min(cos_min, _cos(a, o_ref))
+                abs_max = max(abs_max, float(np.max(np.abs(a - o_ref))))
+                lse_max = max(lse_max, float(np.max(np.abs(_f64(glse[idx, h]) - l_ref))))
+    flops = 4 * wl.head_dim * pairs
+    total_rows = pre.total_queries * wl.num_q_heads
+    rate = flops / spent
+    return {"value": round(rate / 1e12, 6), "unit": "TFLOP/s", "cores": host_cores(),
+            "threads": oracle.num_threads(), "kind": "oracle", "seconds": round(spent, 2),
+            "extrapolated": not (full and rows_done == total_rows),
+            "chunk_s_at_this_rate": round(4 * wl.head_dim * pre_visible_pairs(wl, pre) / rate, 1),
+            "sample": (f"prefill rows: {rows_done} of {total_rows} (query row, q-head) pairs, "
+                       + ("all rows" if full else f"{rows_per_head} seeded random rows of every q-head")
+                       + f" of {done} of {len(order)} (sequence, kv-head) groups in seeded random order; "
+                         "rate = 4 * head_dim * visible pairs / oracle time (fp64 dense attention with "
+                         "explicit mask)"),
+            **({"parity": {"min_cos": round(cos_min, 7), "max_abs": float(f"{abs_max:.3g}"),
+                           "max_lse_abs": float(f"{lse_max:.3g}"), "rows": rows_done,
+                           "against": "fp64 oracle, same inputs"}} if gpu is not None else {})}
+
+
+def torch_index(rows, device):
+    import torch
+    return torch.as_tensor(rows, dtype=torch.long, device=device)
+
+
+def pre_visible_pairs(wl, pre) -> int:
+    """Visible (query, key) pairs of the whole chunk over all q-heads (global p + 1, local min(p + 1, s + w))."""
+    n = 0
+    for b, (L, q0) in enumerate(zip(pre.ctx_lens, pre.q_starts)):
+        for kv in range(wl.num_kv_heads):
+            kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+            for p in range(q0, L):
+                n += min(p + 1, s + w) if kind == "local" else p + 1
+    return n * wl.group
+
+
+def cpu_baseline(wl, dec, k, v, qd, budget_s: float, gpu: tuple | None = None, pre=None, qp=None,
+                 gpu_pre: tuple | None = None, prefill_full: bool = False) -> dict:
     import oracle
     spent, vis, groups, parity = oracle_decode_sample(wl, dec, k, v, qd, budget_s, gpu=gpu)
-    return {"value": round(vis / spent / 1e9, 4), "unit": "GB/s", "cores": min(oracle.num_threads(), wl.group),
-            "kind": "oracle",
-            "seconds": round(spent, 2),
-            "decode_parity": parity,
-            "sample": f"decode of {groups} of {wl.batch * wl.num_kv_heads} (sequence, kv-head) groups, "
-                      f"all {wl.group} q-heads each (fp64 dense attention with explicit mask)"}
+    out = {"value": round(vis / spent / 1e9, 4), "unit": "GB/s", "cores": host_cores(),
+           "threads": oracle.num_threads(), "kind": "oracle",
+           "seconds": round(spent, 2),
+           "decode_parity": parity,
+           "sample": f"decode of {groups} of {wl.batch * wl.num_kv_heads} (sequence, kv-head) groups, "
+                     f"all {wl.group} q-heads each, several groups per batched call on all host cores "
+                     "(fp64 dense attention with explicit mask)"}
+    if pre is not None:
+        out["prefill"] = oracle_prefill_sample(wl, pre, k, v, qp, budget_s, full=prefill_full, gpu=gpu_pre)
+    return out
 
 
 def run_reference(args) -> None:
@@ -539,24 +664,23 @@ def run_reference(args) -> None:
     qd = W.queries(dec)
     per_step = max(1, wl.num_kv_heads // 2)
     for _ in range(args.warmup):
-        oracle_decode_sample(wl, dec, k, v, qd, 1e9, max_heads=1)
+        oracle_decode_sample(wl, dec, k, v, qd, 1e9, max_groups=1)
     spent = vis = 0.0
-    t_steps = []
     for _ in range(args.steps):
-        s, b, _, _ = oracle_decode_sample(wl, dec, k, v, qd, 1e9, max_heads=per_step)
+        s, b, _, _ = oracle_decode_sample(wl, dec, k, v, qd, 1e9, max_groups=per_step)
         spent += s
         vis += b
-        t_steps.append(s)
     value = vis / spent / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * spent / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(wl, 1),
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": min(oracle.num_threads(), wl.group),
-                         "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": host_cores(),
+                         "threads": oracle.num_threads(), "kind": "oracle",
                          "sample": f"per step: decode of {per_step} (sequence, kv-head) groups of sequence 0 "
-                                   f"(all {wl.group} q-heads each), fp64 dense attention with explicit mask"},
+                                   f"(all {wl.group} q-heads each) in one batched call on all host cores, "
+                                   "fp64 dense attention with explicit mask"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -571,6 +695,8 @@ def main() -> None:
     ap.add_argument("--workload", default="llama", choices=("llama", "mistral", "mha", "ragged", "llama_b1"))
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="time budget of the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-prefill-full", action="store_true",
+                    help="run the oracle over every prefill row (Mistral-sized layers) instead of a sample")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -37,23 +37,48 @@ def oracle_rows(prob, q_host, k_host, v_host, b, h, rows=None):
 def compare(prob, q_host, k_host, v_host, out, lse, rows_per_seq=None, heads=None, seqs=None):
     """Compare GPU out / lse (device or host tensors) with the oracle.
 
+    The checked (sequence, q-head, rows) go to the oracle grouped by kv-head, several
+    kv-heads per batched call (all host cores; at most ~2 GB of fp64 K/V at a time).
     Returns dict(min_cos, max_abs, max_lse, worst) over the checked (b, h).
     """
     wl = prob.wl
     out_h = out.float().cpu()
     lse_h = lse.float().cpu() if lse is not None else None
     heads = range(wl.num_q_heads) if heads is None else heads
-    min_cos, max_abs, max_lse, worst = 1.0, 0.0, 0.0, None
+    tasks = {}  # (b, kv) -> [(h, rows)]
     for b in (range(wl.batch) if seqs is None else seqs):
         rows = None if rows_per_seq is None else rows_per_seq[b]
         if rows is not None and len(rows) == 0:
             continue
         C = prob.ctx_lens[b] - prob.q_starts[b]
         ridx = np.arange(C) if rows is None else np.asarray(rows)
-        off = prob.q_offsets[b]
         for h in heads:
-            o_ref, l_ref = oracle_rows(prob, q_host, k_host, v_host, b, h, ridx)
-            o = out_h[off + ridx, h].double().numpy()
+            tasks.setdefault((b, h // wl.group), []).append((h, ridx))
+    min_cos, max_abs, max_lse, worst = 1.0, 0.0, 0.0, None
+    keys = list(tasks)
+    budget = 2e9
+    i = 0
+    while i < len(keys):
+        chunk, used = [], 0
+        while i < len(keys) and (not chunk or used + 16 * prob.ctx_lens[keys[i][0]] * wl.head_dim <= budget):
+            chunk.append(keys[i])
+            used += 16 * prob.ctx_lens[keys[i][0]] * wl.head_dim
+            i += 1
+        groups, meta = [], []
+        for b, kv in chunk:
+            kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+            L, q0 = prob.ctx_lens[b], prob.q_starts[b]
+            off = prob.q_offsets[b]
+            k = k_host[b, kv, :L].cpu().double().numpy()
+            v = v_host[b, kv, :L].cpu().double().numpy()
+            for h, ridx in tasks[(b, kv)]:
+                # inputs may live on the GPU (large layers are generated there): copy the slices
+                q = q_host[torch.as_tensor(off + ridx, device=q_host.device), h].cpu().double().numpy()
+                groups.append((q, q0 + ridx, k, v, kind, s, w))
+                meta.append((b, h, off + ridx))
+        res = oracle.attention_batch(groups)
+        for (b, h, idx), (o_ref, l_ref) in zip(meta, res):
+            o = out_h[idx, h].double().numpy()
             a, r = o.ravel(), o_ref.ravel()
             cos = float(a @ r / (np.linalg.norm(a) * np.linalg.norm(r)))
             err = float(np.max(np.abs(o - o_ref)))
@@ -61,7 +86,7 @@ def compare(prob, q_host, k_host, v_host, out, lse, rows_per_seq=None, heads=Non
                 min_cos, worst = cos, (b, h)
             max_abs = max(max_abs, err)
             if lse_h is not None:
-                max_lse = max(max_lse, float(np.max(np.abs(lse_h[off + ridx, h].double().numpy() - l_ref))))
+                max_lse = max(max_lse, float(np.max(np.abs(lse_h[idx, h].double().numpy() - l_ref))))
     return dict(min_cos=min_cos, max_abs=max_abs, max_lse=max_lse, worst=worst)
 
 
@@ -73,7 +98,7 @@ def assert_close(res, dtype):
 
 
 def sample_rows(C: int, stride: int = 128, n_random: int = 16, seed: int = 0) -> np.ndarray:
-    """First / last rows, rows around multiples of `stride` (tile edges), and seeded random rows."""
+    """First / last rows, rows at multiples of `stride` and one either side (tile edges), seeded random rows."""
     rng = np.random.default_rng(seed)
     pick = {0, 1, C - 1, C - 2}
     for m in range(stride, C, stride):

@@ -45,6 +45,35 @@ def test_sampled_parity_matches_and_catches_a_wrong_head():
     assert par["min_cos"] < 0.99 and par["max_abs"] > 0
 
 
+def test_prefill_sample_rate_ledger_parity_and_cores():
+    """The prefill CPU baseline: full run over the tiny layer's chunk counts every visible pair
+    (the closed form 21,238,784 FLOPs), matches an oracle-made output exactly and reports the
+    host's affinity core count; a planted wrong row is caught."""
+    wl = W.tiny()
+    pre = wl.prefill_problem()
+    k, v = W.dense_kv(pre)
+    q = W.queries(pre)
+    out = torch.zeros(q.shape, dtype=torch.float64)
+    lse = torch.zeros(q.shape[:2], dtype=torch.float64)
+    L, q0 = pre.ctx_lens[0], pre.q_starts[0]
+    for h in range(wl.num_q_heads):
+        kind, s, w = wl.policy[h // wl.group]
+        o, l = oracle.attention_rows(q[:, h].double().numpy(), np.arange(q0, L), k[0, h // wl.group, :L].double().numpy(),
+                                     v[0, h // wl.group, :L].double().numpy(), kind, s, w)
+        out[:, h], lse[:, h] = torch.from_numpy(o), torch.from_numpy(l)
+    rec = bench.oracle_prefill_sample(wl, pre, k, v, q, 1e9, full=True, gpu=(out, lse))
+    assert rec["extrapolated"] is False and rec["parity"]["rows"] == pre.total_queries * wl.num_q_heads
+    assert rec["parity"]["max_abs"] == 0.0 and rec["parity"]["max_lse_abs"] == 0.0
+    assert bench.pre_visible_pairs(wl, pre) * 4 * wl.head_dim == 21_238_784
+    assert rec["cores"] == len(__import__("os").sched_getaffinity(0)) and rec["value"] > 0
+    bad = out.clone()
+    bad[5, 1] = -bad[5, 1]
+    rec = bench.oracle_prefill_sample(wl, pre, k, v, q, 1e9, full=True, gpu=(bad, lse))
+    assert rec["parity"]["min_cos"] < 0.999
+    samp = bench.oracle_prefill_sample(wl, pre, k, v, q, 1e9, rows_per_head=8)
+    assert samp["extrapolated"] is True and "8 seeded random rows" in samp["sample"]
+
+
 def test_clock_sampler_takes_median_max_and_active_reasons():
     """The clocks record of the bench line, from nvidia-smi CSV rows (no GPU: a fake process)."""
     class Fake:

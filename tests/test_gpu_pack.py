@@ -53,6 +53,60 @@ def check_pack(prob, flags=0, **kw):
     return layer
 
 
+def check_pack_full_size(prob):
+    """check_pack at full size: inputs generated on the GPU, every comparison made there.
+
+    The oracle's stored mask depends only on (kind, sink, window, L, q0): it is computed
+    once per distinct key and reused for every (sequence, kv-head) that has it.
+    """
+    wl = prob.wl
+    k, v = W.dense_kv(prob, device="cuda")
+    layer = layer_for(prob)
+    layer.build(k, v)
+    ko = torch.full_like(k, float("nan"))
+    vo = torch.full_like(v, float("nan"))
+    layer.gather(ko, vo)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    kb, vb, kob, vob = _bits(k), _bits(v), _bits(ko), _bits(vo)
+    sentinel = int(_bits(torch.full((1,), float("nan"), dtype=k.dtype))[0])
+    masks, stored_total = {}, 0
+    for b in range(wl.batch):
+        L, q0 = prob.ctx_lens[b], prob.q_starts[b]
+        for kv in range(wl.num_kv_heads):
+            kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+            key = (kind, s, w, L, q0)
+            if key not in masks:
+                masks[key] = torch.from_numpy(oracle.stored_mask(kind, s, w, L, q0)).cuda()
+            mt = masks[key]
+            stored_total += int(mt.sum())
+            assert torch.equal(kob[b, kv, :L][mt], kb[b, kv, :L][mt]), (b, kv)
+            assert torch.equal(vob[b, kv, :L][mt], vb[b, kv, :L][mt]), (b, kv)
+            assert bool((kob[b, kv, :L][~mt] == sentinel).all()), (b, kv)
+            assert bool((vob[b, kv, :L][~mt] == sentinel).all()), (b, kv)
+    assert stored_total == layer.sizes.stored_token_heads
+    return stored_total
+
+
+# Stored token-heads in closed form (sink + window per local head, L per global head; a chunk of C
+# queries adds C - 1 to each local head): Llama-70B-shaped 32K layer and MHA 128K layer.
+FULL_SIZE_STORED = {("llama", "decode"): 721_120, ("llama", "prefill"): 950_440,
+                    ("mha", "decode"): 4_223_872, ("mha", "prefill"): 5_141_152}
+
+
+@pytest.mark.parametrize("name,mode", [("llama", "decode"), ("llama", "prefill"), ("mha", "decode"),
+                                       ("mha", "prefill"), ("ragged", "decode")])
+def test_pack_gather_bit_exact_at_full_size(name, mode):
+    """Every stored row of the bench's 32K layer, the MHA 128K layer and the ragged batch, bit for bit."""
+    wl = W.ALL[name]()
+    prob = wl.decode_problem() if mode == "decode" else wl.prefill_problem()
+    n = check_pack_full_size(prob)
+    if (name, mode) in FULL_SIZE_STORED:
+        assert n == FULL_SIZE_STORED[(name, mode)]
+    else:  # ragged: per sequence 2 global heads of L tokens, 6 local heads of min(L, 4 + 512)
+        assert n == sum(2 * L + 6 * min(L, 4 + 512) for L in prob.ctx_lens)
+
+
 @pytest.mark.parametrize("name", ["tiny", "mistral"])
 @pytest.mark.parametrize("mode", ["decode", "prefill"])
 def test_pack_gather_bit_exact(name, mode):

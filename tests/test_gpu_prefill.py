@@ -92,15 +92,14 @@ def test_prefill_bf16_page_permutation_and_determinism():
     assert torch.equal(out0, out2) and torch.equal(lse0, lse2)
 
 
-@pytest.mark.parametrize("name,seqs,heads", [
-    ("llama", (0, 7), None),
-    ("mha", (0, 3), (0, 1, 7, 8, 9, 31, 32, 56, 63)),
-])
-def test_prefill_bf16_matches_oracle_sampled_at_full_size(name, seqs, heads):
+@pytest.mark.parametrize("name", ["llama", "mha"])
+def test_prefill_bf16_matches_oracle_sampled_at_full_size(name):
     """The bench's layer (and the MHA 128K layer) at full size, in the bench's launch configuration.
 
-    Inputs are generated on the GPU; the oracle checks sampled rows (chunk edges, tile edges at
-    multiples of 512 +- 1, seeded random rows) of the listed sequences and q-heads.
+    Inputs are generated on the GPU.  Every sequence and every q-head is checked on chunk
+    edges, rows at multiples of 512 and one either side, and seeded random rows; for one
+    q-head of a global kv-head and one of a local kv-head of every sequence, also every
+    128-row query-tile edge and the rows either side of it.
     """
     wl = W.ALL[name]()
     prob = wl.prefill_problem()
@@ -111,9 +110,32 @@ def test_prefill_bf16_matches_oracle_sampled_at_full_size(name, seqs, heads):
     out, lse = layer.attention(q)
     torch.cuda.synchronize()
     assert layer.device_status() == 0
-    rows = [sample_rows(c, stride=512, n_random=12, seed=b) if b in seqs else [] for b, c in enumerate(prob.q_counts)]
-    res = compare(prob, q, k, v, out, lse, rows_per_seq=rows, heads=heads, seqs=seqs)
-    assert_close(res, "bf16")
+    rows = [sample_rows(c, stride=512, n_random=12, seed=b) for b, c in enumerate(prob.q_counts)]
+    assert_close(compare(prob, q, k, v, out, lse, rows_per_seq=rows), "bf16")
+    for b, c in enumerate(prob.q_counts):
+        pol = wl.policy[b * wl.num_kv_heads:(b + 1) * wl.num_kv_heads]
+        g_kv = next(kv for kv, p in enumerate(pol) if p[0] == "global")
+        l_kv = next(kv for kv, p in enumerate(pol) if p[0] == "local")
+        edges = [sample_rows(c, stride=128, n_random=4, seed=100 + b) if bb == b else []
+                 for bb in range(wl.batch)]
+        heads = (g_kv * wl.group, l_kv * wl.group + wl.group - 1)
+        assert_close(compare(prob, q, k, v, out, lse, rows_per_seq=edges, heads=heads, seqs=(b,)), "bf16")
+
+
+def test_prefill_bf16_dense_masked_matches_oracle_at_mistral_size():
+    """The dense-plus-mask variant of the bf16 prefill (every head stores its whole context, local heads
+    masked per element over every causal tile) on the Mistral-shaped layer, every sequence and q-head."""
+    wl = W.mistral()
+    prob = wl.prefill_problem()
+    k, v = W.dense_kv(prob, device="cuda")
+    q = W.queries(prob, device="cuda")
+    layer = layer_for(prob, flags=S.SP_FLAG_DENSE_MASKED)
+    layer.build(k, v)
+    out, lse = layer.attention(q)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    rows = [sample_rows(c, stride=128, n_random=16, seed=b) for b, c in enumerate(prob.q_counts)]
+    assert_close(compare(prob, q, k, v, out, lse, rows_per_seq=rows), "bf16")
 
 
 def test_prefill_adaptive_window_matches_oracle():
