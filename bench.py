@@ -260,6 +260,9 @@ def run_ours(args) -> None:
     fp8_ms, fp8_pack_ms = reduce_max([fp8_ms, fp8_pack_ms], world, dev)
     del Ld8
 
+    # ---- retrieval heads: the 32K layer with two retrieval kv-heads per sequence ----
+    retrieval = run_retrieval(wl, dev, flush, world) if wl.name.startswith("llama") else None
+
     # ---- end to end through the public API with host buffers ----
     e2e_dense = run_e2e_dense(args, dev, Ld, k, v, qd, od, lsed, world)
     e2e, append_us = run_e2e_serving(args, dev, wl, dec, k, v, world)
@@ -334,6 +337,7 @@ def run_ours(args) -> None:
                         "what": "decode on FP8 E4M3 pages (1 byte per element), bf16 queries and output"},
         "e2e": e2e,
         "append": {"us": round(append_us, 2), "what": "segpaged_decode_append: one token per sequence, all heads"},
+        "retrieval": retrieval,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "wall_s_timed": round(wall, 3),
@@ -350,6 +354,47 @@ def run_ours(args) -> None:
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def run_retrieval(wl, dev, flush, world) -> dict:
+    """Decode and prefill of the 32K layer with retrieval heads (same shape and batch as `wl`).
+
+    Per sequence: the layer's global kv-head, two retrieval kv-heads (sink 4, window 512,
+    top_p 0.5 of the synthetic per-page importance) and five local ones (sink 4, window 8192).
+    Rates count only the work the heads' visible sets need: stored K+V bytes for decode,
+    4 * head_dim FLOPs per visible pair for prefill.
+    """
+    import torch
+
+    from head_aware_paged_build_b200 import workloads as W
+    from head_aware_paged_build_b200.runtime import layer_for
+
+    wr = W.llama_retrieval(batch=wl.batch)
+    dec, pre = wr.decode_problem(), wr.prefill_problem()
+    k, v = W.dense_kv(dec, device=dev, gen_device=dev)
+    qd = W.queries(dec, device=dev, gen_device=dev)
+    qp = W.queries(pre, device=dev, gen_device=dev)
+    ld, lp = layer_for(dec, device=dev), layer_for(pre, device=dev)
+    ld.build(k, v)
+    lp.build(k, v)
+    od, lsed = torch.empty_like(qd), torch.empty(qd.shape[:2], dtype=torch.float32, device=dev)
+    op, lsep = torch.empty_like(qp), torch.empty(qp.shape[:2], dtype=torch.float32, device=dev)
+    d_ms = median_ms(lambda: ld.attention(qd, od, lsed), flush, 10)
+    p_ms = median_ms(lambda: lp.attention(qp, op, lsep), flush, 3)
+    assert ld.device_status() == 0 and lp.device_status() == 0
+    d_ms, p_ms = reduce_max([d_ms, p_ms], world, dev)
+    pk = peaks()
+    vis = ld.sizes.stored_token_heads * 2 * wr.head_dim * 2
+    flops = 4 * wr.head_dim * lp.sizes.visible_pairs
+    return {"decode_ms": round(d_ms, 5), "decode_visible_kv_bytes": vis,
+            "decode_GB/s": round(weak_rate(vis, world, d_ms) / 1e9, 1),
+            "decode_frac_hbm": round(vis / (d_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+            "prefill_ms": round(p_ms, 4), "prefill_visible_flops": flops,
+            "prefill_TFLOP/s": round(weak_rate(flops, world, p_ms) / 1e12, 1),
+            "prefill_frac_bf16_burst": round(flops / (p_ms * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
+            "kv_saving_decode": round(1 - ld.sizes.stored_token_heads / ld.sizes.dense_token_heads, 4),
+            "what": "32K layer, per sequence 1 global, 2 retrieval (sink 4, window 512, top_p 0.5 of synthetic "
+                    "per-page importance), 5 local kv-heads"}
 
 
 def run_e2e_serving(args, dev, wl, dec, k, v, world) -> tuple[dict, float]:

@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendLaunch a) 
     pg->abs_start = L - slot;
     lo = slot;
   }
-  pg->span = make_span(lo, slot + 1);
+  pg->span = make_span(lo, slot + 1) | (pg->span & kSpanCausal);
   // eviction: position L - window leaves the window [L + 1 - window, L]
   if (local) {
     const int e = L - hd->window;
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendLaunch a) 
       const int se = re % P;
       if (pe->abs_start == e - se) {
         const int elo = max(slot_lo(*pe), se + 1), ehi = slot_hi(*pe);
-        pe->span = elo < ehi ? make_span(elo, ehi) : 0;
+        pe->span = elo < ehi ? (make_span(elo, ehi) | (pe->span & kSpanCausal)) : 0;
       }
     }
   }

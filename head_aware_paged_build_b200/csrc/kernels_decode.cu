@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch
             for (int e = 0; e < 4; ++e) {
               const int tok = tok0 + n * 8 + tq * 2 + (e & 1);
               bool vis = tok >= lo && tok < hi;
-              if (hd.mask_local) vis = vis && sees(1, hd.sink, hd.window, qpos, pg.abs_start + tok);
+              if (hd.mask_local) vis = vis && (page_causal(pg) || sees(1, hd.sink, hd.window, qpos, pg.abs_start + tok));
               sc[n][e] = vis ? sc[n][e] * scale_log2 : -INFINITY;
             }
         }
@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(DecodeLaunch a)
       for (int e = threadIdx.x; e < G * P; e += kF32Threads) {
         const int h = e / P, t = e % P;
         bool vis = t >= slot_lo(pg) && t < slot_hi(pg);
-        if (hd.mask_local) vis = vis && sees(1, hd.sink, hd.window, qpos, pg.abs_start + t);
+        if (hd.mask_local) vis = vis && (page_causal(pg) || sees(1, hd.sink, hd.window, qpos, pg.abs_start + t));
         float s = 0.f;
         for (int i = 0; i < D; ++i) s = fmaf(qs[h * D + i], kp[t * D + i], s);
         sc[e] = vis ? s * a.scale_log2 : -INFINITY;

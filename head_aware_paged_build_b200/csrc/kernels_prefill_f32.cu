@@ -4,7 +4,8 @@
 // single-tile items); thread r owns query row r.  KV
 // tiles of 64 tokens (the head's pages, in its position order) are staged in
 // shared memory; each thread scores the tile's keys for its row, masks them
-// (causal, and sink + window for local heads), and folds them into an online
+// (causal, and sink + window for local heads, except on pages flagged to be
+// seen causally: a retrieval head's sink and kept blocks), and folds them into an online
 // softmax.  Only the tile ranges the planner lists are visited: a local head
 // touches its sink tiles and the tiles of its recent window, never the rest of
 // the context ("SegPagedAttention runtime design", §4).
@@ -18,6 +19,7 @@ namespace {
 
 constexpr int kRows = kPrefillTileTokensF32;  // query rows per CTA = KV tokens per tile
 constexpr float kLn2f = 0.6931471805599453f;
+constexpr int kPosCausal = 1 << 30;  // key flag in pos[]: its page is seen causally (positions stay below 2^30)
 
 template <int D, int P>
 __global__ void __launch_bounds__(kRows) prefill_f32_kernel(PrefillLaunch a) {
@@ -65,7 +67,11 @@ __global__ void __launch_bounds__(kRows) prefill_f32_kernel(PrefillLaunch a) {
           const int ii = e / P, t2 = e % P;
           vs[ii * kRows + j * P + t2] = have ? vpp[e] : 0.f;
         }
-        for (int tt = threadIdx.x; tt < P; tt += kRows) pos[j * P + tt] = (have && tt >= slot_lo(pg) && tt < slot_hi(pg)) ? pg.abs_start + tt : -1;
+        // key position, with kPosCausal set for a page every row sees causally; -1: no key
+        for (int tt = threadIdx.x; tt < P; tt += kRows)
+          pos[j * P + tt] = (have && tt >= slot_lo(pg) && tt < slot_hi(pg))
+                                ? (pg.abs_start + tt) | (page_causal(pg) ? kPosCausal : 0)
+                                : -1;
       }
       __syncthreads();
       if (!active) continue;
@@ -73,9 +79,9 @@ __global__ void __launch_bounds__(kRows) prefill_f32_kernel(PrefillLaunch a) {
       float mx = -INFINITY;
 #pragma unroll 4
       for (int c = 0; c < kRows; ++c) {
-        const int ap = pos[c];
+        const int ap = pos[c] & ~kPosCausal;
         float x = -INFINITY;
-        if (ap >= 0 && sees(hd.kind, hd.sink, hd.window, p, ap)) {
+        if (pos[c] >= 0 && sees((pos[c] & kPosCausal) ? 0 : hd.kind, hd.sink, hd.window, p, ap)) {
           float d = 0.f;
           for (int i = 0; i < D; ++i) d = fmaf(qs[r * (D + 1) + i], ks[c * D + i], d);
           x = d * a.scale_log2;

@@ -9,7 +9,8 @@
 // (query-head, kv-head) pair runs over its own true length, with no mask over
 // invisible KV).  Only tiles that cross a boundary (causal diagonal, window
 // edge, sink page, a segment's partial last page) are masked, per row, by
-// visible column intervals.
+// visible column intervals.  A retrieval head's sink and kept blocks sit on
+// pages flagged to be seen causally; its other pages follow the local rule.
 //
 // Warp roles (576 threads):
 //   warp 0      producer: both Q tiles by TMA (128-byte swizzle); K and V
@@ -82,24 +83,25 @@ struct Bars {
 // Does every row p in [p_first, p_last] see every slot of this page?
 __device__ __forceinline__ bool page_fully_visible(const PageDesc& pg, bool exists, const HeadDesc& hd, int p_first,
                                                    int p_last) {
-  if (!exists || pg.span != make_span(0, 64)) return false;
+  if (!exists || slot_lo(pg) != 0 || slot_hi(pg) != 64) return false;
   const int a0 = pg.abs_start, a1 = pg.abs_start + 63;
   if (a1 > p_first) return false;
-  if (hd.kind == 0) return true;
+  if (hd.kind == 0 || page_causal(pg)) return true;
   return a1 < hd.sink || a0 > p_last - hd.window;
 }
 
 // Slots of a page visible to row p: [0, h1) (sink run) and [l2, h2) (causal
 // part / recent window), inside the page's valid range [lo, hi).  A page with
 // lo > 0 never holds sink positions (sink pages always start at slot 0; only
-// ring pages of decode plans start later), so its sink run is empty.
+// ring pages of decode plans start later), so its sink run is empty.  A page
+// flagged kSpanCausal (a retrieval head's sink or kept block) is seen causally.
 __device__ __forceinline__ void visible_slots(const PageDesc& pg, bool exists, const HeadDesc& hd, int p, int& h1,
                                               int& l2, int& h2) {
   h1 = l2 = h2 = 0;
   if (!exists) return;
   const int lo = slot_lo(pg);
   const int causal = min(slot_hi(pg), p - pg.abs_start + 1);  // valid slots with position <= p
-  if (hd.kind == 0) {
+  if (hd.kind == 0 || page_causal(pg)) {
     l2 = lo, h2 = causal;
   } else {
     h1 = lo > 0 ? 0 : min(causal, hd.sink - pg.abs_start);     // sink run

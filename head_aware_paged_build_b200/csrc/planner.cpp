@@ -5,6 +5,7 @@
 // tables and layout must be built when KV is written and reused, because
 // computing them on every attention call cost a 0.70x slowdown).
 #include <algorithm>
+#include <cmath>
 #include <cstring>
 #include <limits>
 #include <new>
@@ -74,14 +75,50 @@ sp_status validate(const sp_problem& p) {
   if (rows > std::numeric_limits<int32_t>::max()) return fail(SP_ERR_UNSUPPORTED, "too many query rows");
   for (int64_t i = 0; i < int64_t(p.batch) * p.num_kv_heads; ++i) {
     const sp_head_policy& h = p.policy[i];
-    if (h.kind == SP_RETRIEVAL)
-      return fail(SP_ERR_UNSUPPORTED, "RETRIEVAL heads are not implemented (no scoring rule is defined)");
-    if (h.kind != SP_GLOBAL && h.kind != SP_LOCAL && h.kind != SP_DENSE)
-      return fail(SP_ERR_INVALID_ARG, "policy[" + std::to_string(i) + "].kind is not a head kind");
-    if (h.kind == SP_LOCAL && (h.sink < 0 || h.window == 0))
-      return fail(SP_ERR_INVALID_ARG, "policy[" + std::to_string(i) + "]: local heads need sink >= 0, window != 0");
+    const std::string who = "policy[" + std::to_string(i) + "]";
+    if (h.kind != SP_GLOBAL && h.kind != SP_LOCAL && h.kind != SP_DENSE && h.kind != SP_RETRIEVAL)
+      return fail(SP_ERR_INVALID_ARG, who + ".kind is not a head kind");
+    if ((h.kind == SP_LOCAL || h.kind == SP_RETRIEVAL) && (h.sink < 0 || h.window == 0))
+      return fail(SP_ERR_INVALID_ARG, who + ": local and retrieval heads need sink >= 0, window != 0");
+    if (h.kind != SP_RETRIEVAL) continue;
+    if (!std::isfinite(h.top_p)) return fail(SP_ERR_INVALID_ARG, who + ": top_p must be finite");
+    if (p.flags & SP_FLAG_RING) return fail(SP_ERR_UNSUPPORTED, "retrieval heads are not supported in ring plans");
+    if (!p.block_mass || !p.block_mass[i])
+      return fail(SP_ERR_INVALID_ARG, who + ": a retrieval head needs its block_mass entry");
+    const int64_t nb = (int64_t(p.ctx_len[i / p.num_kv_heads]) + p.page_size - 1) / p.page_size;
+    for (int64_t j = 0; j < nb; ++j) {
+      const float m = p.block_mass[i][j];
+      if (!(m >= 0.f) || !std::isfinite(m))
+        return fail(SP_ERR_INVALID_ARG, who + ": block_mass values must be finite and >= 0");
+    }
   }
   return SP_OK;
+}
+
+// Blocks a retrieval head keeps: the candidates (blocks holding a position >=
+// sink) in decreasing importance, ties by lower block, and of those the
+// shortest prefix whose importance reaches top_p of the candidates' total
+// (fp64 sums in that order); top_p >= 1 keeps every candidate, <= 0 none.
+std::vector<uint8_t> kept_blocks(int64_t L, int64_t P, int64_t sink, float top_p, const float* mass) {
+  const int64_t nb = (L + P - 1) / P;
+  std::vector<int64_t> cand;
+  for (int64_t i = 0; i < nb; ++i)
+    if ((i + 1) * P > sink) cand.push_back(i);
+  std::stable_sort(cand.begin(), cand.end(), [&](int64_t a, int64_t b) { return mass[a] > mass[b]; });
+  size_t keep = cand.size();
+  if (top_p <= 0.f) {
+    keep = 0;
+  } else if (top_p < 1.f) {
+    double total = 0.0;
+    for (int64_t i : cand) total += double(mass[i]);
+    const double target = double(top_p) * total;
+    double run = 0.0;
+    keep = 0;
+    while (keep < cand.size() && run < target) run += double(mass[cand[keep++]]);
+  }
+  std::vector<uint8_t> sel(nb, 0);
+  for (size_t k = 0; k < keep; ++k) sel[cand[k]] = 1;
+  return sel;
 }
 
 // Pages of a head (indices into its page list) holding any position of [x, y].
@@ -98,6 +135,37 @@ void pages_touching(const sp_plan& pl, int h, int64_t x, int64_t y, int64_t* v0,
     *v1 = std::max<int64_t>(*v1, g.first_page_index + (hi - g.abs_start) / P + 1);
   }
   if (*v0 > *v1) *v0 = *v1 = 0;
+}
+
+// KV tiles (of `ppt` pages, in the head's page list) that a retrieval head's
+// item must visit for rows at positions [p_first, p_last]: every tile holding
+// a key some row sees, covered by at most two ranges (split at the widest run
+// of tiles no row sees; tiles left inside a range are masked out by the
+// kernel).  A page flagged kSpanCausal is seen by a row at p up to p; any
+// other page by the local rule (sink, or the window of some row).
+void retrieval_tiles(const sp_plan& pl, int h, int64_t p_first, int64_t p_last, int ppt, int64_t* t) {
+  const HeadDesc& hd = pl.heads[h];
+  std::vector<int64_t> tiles;
+  for (int v = 0; v < hd.n_vpages; ++v) {
+    const PageDesc& pg = pl.pages[hd.vpage_begin + v];
+    const int64_t lo = slot_lo(pg), hi = slot_hi(pg);
+    if (hi <= lo) continue;
+    const int64_t a0 = pg.abs_start + lo, a1 = pg.abs_start + hi - 1;
+    const bool seen = a0 <= p_last && (page_causal(pg) || a0 < hd.sink ||
+                                       std::min<int64_t>(a1, p_last) >= p_first - hd.window + 1);
+    if (seen && (tiles.empty() || tiles.back() != v / ppt)) tiles.push_back(v / ppt);
+  }
+  t[0] = t[1] = t[2] = t[3] = 0;
+  if (tiles.empty()) return;
+  size_t cut = 0;  // the widest gap lies after tiles[cut - 1]
+  int64_t gap = 0;
+  for (size_t i = 1; i < tiles.size(); ++i)
+    if (tiles[i] - tiles[i - 1] - 1 > gap) gap = tiles[i] - tiles[i - 1] - 1, cut = i;
+  if (gap == 0) {
+    t[0] = tiles.front(), t[1] = tiles.back() + 1;
+  } else {
+    t[0] = tiles.front(), t[1] = tiles[cut - 1] + 1, t[2] = tiles[cut], t[3] = tiles.back() + 1;
+  }
 }
 
 void align_to(std::vector<uint8_t>& blob, size_t a) { blob.resize((blob.size() + a - 1) / a * a, 0); }
@@ -139,6 +207,7 @@ sp_status plan_build(sp_plan& pl) {
       if (int64_t(pl.ctx_len[b]) + cap > (int64_t(1) << 30)) return fail(SP_ERR_UNSUPPORTED, "ctx_len + capacity above 2^30");
   }
 
+  pl.kept_blocks.assign(nh, {});
   int64_t ctx_row = 0;
   for (int b = 0; b < B; ++b, ctx_row += pl.ctx_len[b - 1]) {
     const int64_t L = pl.ctx_len[b], q0 = pl.q_start[b];
@@ -147,22 +216,58 @@ sp_status plan_build(sp_plan& pl) {
     for (int kv = 0; kv < Hkv; ++kv) {
       const int h = b * Hkv + kv;
       const sp_head_policy& pol = pl.policy[h];
-      const bool local = pol.kind == SP_LOCAL;
+      const bool retrieval = pol.kind == SP_RETRIEVAL;
+      const bool local = pol.kind == SP_LOCAL || retrieval;  // the local rule applies (to unflagged pages)
       const int64_t s = local ? pol.sink : 0;
       // adaptive window (window <= -1): max(1, L / -window) for this sequence
       const int64_t w = !local ? 0 : pol.window > 0 ? pol.window : std::max<int64_t>(1, L / (-int64_t(pol.window)));
-      int64_t firsts[2], lens[2];
-      int ns = 0;
+      // Runs of stored positions (start, length, every query sees them causally).
+      struct Run {
+        int64_t start, len;
+        bool causal;
+      };
+      std::vector<Run> runs;
+      std::vector<uint8_t> sel;
+      if (retrieval) {
+        sel = kept_blocks(L, P, s, pol.top_p, p.block_mass[h]);
+        pl.kept_blocks[h] = sel;
+      }
       if (!local || dense_masked) {
-        firsts[ns] = 0, lens[ns++] = L;
-      } else {
+        runs.push_back({0, L, false});
+      } else if (!retrieval) {
         const int64_t sink_len = std::min<int64_t>(s, L);
         const int64_t rec = std::max<int64_t>(s, q0 - w + 1);
         if (rec <= sink_len) {  // touching: one run [0, L)
-          firsts[ns] = 0, lens[ns++] = L;
+          runs.push_back({0, L, false});
         } else {
-          if (sink_len > 0) firsts[ns] = 0, lens[ns++] = sink_len;
-          if (rec < L) firsts[ns] = rec, lens[ns++] = L - rec;
+          if (sink_len > 0) runs.push_back({0, sink_len, false});
+          if (rec < L) runs.push_back({rec, L - rec, false});
+        }
+      } else {
+        // Retrieval: per block, its sink part and its kept part are seen causally
+        // by every query; an unkept block keeps only its part inside the calls'
+        // windows [max(sink, q0 - w + 1), L).  Touching runs merge when they share
+        // the flag; in decode plans (one query, which sees every stored position)
+        // touching runs always merge.
+        const int64_t rec = std::max<int64_t>(s, q0 - w + 1);
+        const bool decode_head = q0 == L - 1;
+        auto add = [&](int64_t a, int64_t e, bool causal) {
+          if (e <= a) return;
+          if (!runs.empty() && runs.back().start + runs.back().len == a &&
+              (runs.back().causal == causal || decode_head)) {
+            runs.back().len += e - a;
+            runs.back().causal = runs.back().causal && causal;
+          } else {
+            runs.push_back({a, e - a, causal});
+          }
+        };
+        for (int64_t i = 0; i * P < L; ++i) {
+          const int64_t a = i * P, e = std::min<int64_t>(L, a + P), c = std::max<int64_t>(a, s);
+          add(a, std::min<int64_t>(e, s), true);
+          if (sel[i])
+            add(c, e, true);
+          else
+            add(std::max<int64_t>(c, rec), e, false);
         }
       }
       if (ring) {
@@ -170,13 +275,13 @@ sp_status plan_build(sp_plan& pl) {
         // plus pages for `cap` more tokens.  LOCAL: the sink's pages (for all
         // s positions) and a ring of R pages; position a >= s sits in ring slot
         // a mod (R P), so appends never move a token.
-        firsts[0] = 0, lens[0] = L, ns = 1;
+        runs.assign(1, Run{0, L, false});
         if (local) {
           const int64_t sink_len = std::min<int64_t>(s, L);
           const int64_t wlo = std::max<int64_t>(s, L - w), whi = L;
-          ns = 0;
-          if (sink_len > 0) firsts[ns] = 0, lens[ns++] = sink_len;
-          if (whi > wlo) firsts[ns] = wlo, lens[ns++] = whi - wlo;
+          runs.clear();
+          if (sink_len > 0) runs.push_back({0, sink_len, false});
+          if (whi > wlo) runs.push_back({wlo, whi - wlo, false});
         }
       }
       HeadDesc& hd = pl.heads[h];
@@ -225,21 +330,24 @@ sp_status plan_build(sp_plan& pl) {
           if (whi > wlo)
             pl.segments.push_back(sp_segment{int32_t(wlo), int32_t(whi - wlo), int32_t(nsink), int32_t(R)});
         }
-        for (int i = 0; i < ns; ++i) stored += lens[i];
+        for (const Run& r : runs) stored += r.len;
       }
-      for (int i = 0; i < ns && !ring; ++i) {
-        sp_segment g{int32_t(firsts[i]), int32_t(lens[i]), vp, int32_t(ceil_div(lens[i], P))};
+      for (size_t i = 0; i < runs.size() && !ring; ++i) {
+        const Run& r = runs[i];
+        sp_segment g{int32_t(r.start), int32_t(r.len), vp, int32_t(ceil_div(r.len, P))};
         pl.segments.push_back(g);
         for (int k = 0; k < g.num_pages; ++k) {
           PageDesc pd{};
           pd.phys = 0;  // assigned below
           pd.abs_start = g.abs_start + k * P;
           pd.span = make_span(0, int32_t(std::min<int64_t>(P, int64_t(g.abs_start) + g.length - pd.abs_start)));
+          // dense-masked retrieval heads: page k is block k, seen causally when kept
+          if (r.causal || (retrieval && dense_masked && sel[k])) pd.span |= kSpanCausal;
           pd.head = h;
           pl.pages.push_back(pd);
         }
         vp += g.num_pages;
-        stored += lens[i];
+        stored += r.len;
       }
       hd.n_vpages = vp;
       hd.ctx_row0 = int32_t(ctx_row);
@@ -248,8 +356,18 @@ sp_status plan_build(sp_plan& pl) {
         return fail(SP_ERR_UNSUPPORTED, "more than 2^31 pages");
       pl.seg_begin.push_back(int32_t(pl.segments.size()));
       dense_rows += L;
-      // visible (query, key) pairs: global p + 1, local min(p + 1, s + w)
-      for (int64_t q = q0; q < L; ++q) visible += local ? std::min<int64_t>(q + 1, s + w) : q + 1;
+      // visible (query, key) pairs: global p + 1, local min(p + 1, s + w); retrieval:
+      // the sink and kept positions before the window plus the window itself
+      if (retrieval) {
+        std::vector<int64_t> pc(L + 1, 0);  // pc[j]: positions < j seen causally (sink or kept block)
+        for (int64_t j = 0; j < L; ++j) pc[j + 1] = pc[j] + ((j < s || sel[j / P]) ? 1 : 0);
+        for (int64_t q = q0; q < L; ++q) {
+          const int64_t lo = std::max<int64_t>(0, q - w + 1);
+          visible += pc[lo] + (q + 1 - lo);
+        }
+      } else {
+        for (int64_t q = q0; q < L; ++q) visible += local ? std::min<int64_t>(q + 1, s + w) : q + 1;
+      }
     }
   }
   visible *= pl.group;
@@ -379,6 +497,15 @@ sp_status plan_build(sp_plan& pl) {
           p_last = std::max<int64_t>(p_last, it.p0[x] + it.n_rows[x] - 1);
         }
         int64_t v0, v1, v2, v3;
+        if (!pl.kept_blocks[h].empty() && !dense_masked) {
+          int64_t t[4];
+          retrieval_tiles(pl, h, p_first, p_last, ppt, t);
+          it.t0 = int32_t(t[0]), it.t1 = int32_t(t[1]), it.t2 = int32_t(t[2]), it.t3 = int32_t(t[3]);
+          it.work = int32_t((t[1] - t[0]) + (t[3] - t[2]));
+          head_max[h] = std::max(head_max[h], it.work);
+          per_head[h].push_back(it);
+          continue;
+        }
         if (hd.kind == 0 || dense_masked) {
           pages_touching(pl, h, 0, p_last, &v0, &v1);
           v2 = v3 = 0;
@@ -493,6 +620,7 @@ sp_status segpaged_plan_create(const sp_problem* problem, sp_plan** out) {
     pl->prob.ctx_len = pl->prob.q_start = nullptr;
     pl->prob.policy = nullptr;
     pl->prob.page_ids = nullptr;
+    pl->prob.block_mass = nullptr;
     if (st != SP_OK) {
       delete pl;
       return st;

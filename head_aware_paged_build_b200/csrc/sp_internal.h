@@ -38,7 +38,9 @@ enum DeviceCode : int32_t {
 };
 
 // One (sequence, kv-head).  Kinds are resolved: 0 reads the whole causal
-// context, 1 is local (sink + window).
+// context, 1 applies the local rule (sink + window) to every page that is not
+// flagged kSpanCausal.  A retrieval head is kind 1 whose sink pages and kept
+// blocks' pages carry that flag.
 struct alignas(16) HeadDesc {
   int32_t kind;
   int32_t sink;
@@ -56,9 +58,11 @@ struct alignas(16) HeadDesc {
 static_assert(sizeof(HeadDesc) == 48, "HeadDesc layout");
 
 // One page of a head.  Slot t holds position abs_start + t; only slots
-// [lo, hi) hold tokens (lo = span & 0xffff, hi = span >> 16).  Pages of a
-// head are in position order except in ring plans, where the recent window
-// is a ring of pages (see the planner).
+// [lo, hi) hold tokens (lo = span & 0xff, hi = (span >> 16) & 0xff; page sizes
+// are at most 64).  Bit 8 of span (kSpanCausal) marks a page every query sees
+// causally whatever the head's local rule: the sink and kept blocks of a
+// retrieval head.  Pages of a head are in position order except in ring plans,
+// where the recent window is a ring of pages (see the planner).
 struct alignas(16) PageDesc {
   int32_t phys;       // physical page id in the pools
   int32_t abs_start;  // absolute position of slot 0
@@ -66,8 +70,10 @@ struct alignas(16) PageDesc {
   int32_t head;       // owning HeadDesc index
 };
 static_assert(sizeof(PageDesc) == 16, "PageDesc layout");
-SP_HD inline int32_t slot_lo(const PageDesc& p) { return p.span & 0xffff; }
-SP_HD inline int32_t slot_hi(const PageDesc& p) { return p.span >> 16; }
+constexpr int32_t kSpanCausal = 1 << 8;
+SP_HD inline int32_t slot_lo(const PageDesc& p) { return p.span & 0xff; }
+SP_HD inline int32_t slot_hi(const PageDesc& p) { return (p.span >> 16) & 0xff; }
+SP_HD inline bool page_causal(const PageDesc& p) { return (p.span & kSpanCausal) != 0; }
 SP_HD inline int32_t make_span(int32_t lo, int32_t hi) { return lo | (hi << 16); }
 
 // A run of consecutive pages of one head processed by one decode CTA.
@@ -134,8 +140,9 @@ struct sp_plan {
   sp_problem prob{};                      // pointers inside are cleared after copying
   std::vector<int32_t> ctx_len, q_start;
   std::vector<sp_head_policy> policy;
-  std::vector<sp_segment> segments;       // per head: up to two, flattened
+  std::vector<sp_segment> segments;       // per head: its runs of stored positions, flattened
   std::vector<int32_t> seg_begin;         // [n_heads + 1]
+  std::vector<std::vector<uint8_t>> kept_blocks;  // per head: kept blocks of a retrieval head, else empty
   std::vector<sp::HeadDesc> heads;
   std::vector<sp::PageDesc> pages;
   std::vector<sp::DecodeItem> decode_items;

@@ -24,23 +24,26 @@ class SegPagedLayer:
     """Plan + device buffers of one attention layer's batch.
 
     ``policy`` holds ``(kind, sink, window)`` per (sequence, kv-head) with kind
-    in {"global", "local", "dense"}; ``q_start[b]`` is the position of the
-    first query of sequence b (``ctx_len[b] - 1`` for decode).
+    in {"global", "local", "dense"}, or ``("retrieval", sink, window, top_p)``;
+    ``block_mass`` gives each retrieval head's importance per page-size block
+    (None for other heads); ``q_start[b]`` is the position of the first query
+    of sequence b (``ctx_len[b] - 1`` for decode).
     """
 
     def __init__(self, *, batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, page_size: int,
                  dtype: str, ctx_len: Sequence[int], q_start: Sequence[int],
-                 policy: Sequence[tuple[str, int, int]], device="cuda", flags: int = 0,
+                 policy: Sequence[tuple], device="cuda", flags: int = 0,
                  page_ids: Sequence[int] | None = None, first_page: int = 0, target_ctas: int = 0,
                  append_capacity: int = 0, pools: tuple[torch.Tensor, torch.Tensor] | None = None,
-                 kv_dtype: str | None = None, k_scale: float = 1.0, v_scale: float = 1.0):
+                 kv_dtype: str | None = None, k_scale: float = 1.0, v_scale: float = 1.0,
+                 block_mass: Sequence | None = None):
         self.dtype = dtype
         self.torch_dtype = {"f32": torch.float32, "bf16": torch.bfloat16}[dtype]
         self.num_q_heads, self.num_kv_heads, self.head_dim = num_q_heads, num_kv_heads, head_dim
         self.device = torch.device(device)
         self.problem = S.make_problem(batch, num_q_heads, num_kv_heads, head_dim, page_size, dtype, ctx_len,
                                       q_start, policy, first_page, page_ids, target_ctas, flags, append_capacity,
-                                      kv_dtype, k_scale, v_scale)
+                                      kv_dtype, k_scale, v_scale, block_mass)
         self.kv_dtype = kv_dtype or dtype
         self.batch = batch
         self.ctx_len = [int(x) for x in ctx_len]
@@ -162,6 +165,8 @@ class SegPagedLayer:
 def layer_for(prob, device="cuda", flags: int = 0, **kw) -> SegPagedLayer:
     """A SegPagedLayer for a ``workloads.Problem``."""
     wl = prob.wl
+    if "block_mass" not in kw and wl.has_retrieval:
+        kw["block_mass"] = prob.block_masses()
     return SegPagedLayer(batch=wl.batch, num_q_heads=wl.num_q_heads, num_kv_heads=wl.num_kv_heads,
                          head_dim=wl.head_dim, page_size=wl.page_size, dtype=wl.dtype, ctx_len=prob.ctx_lens,
                          q_start=prob.q_starts, policy=wl.policy, device=device, flags=flags, **kw)

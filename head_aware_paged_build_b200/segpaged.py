@@ -43,7 +43,8 @@ class SegPagedError(RuntimeError):
 
 
 class sp_head_policy(ctypes.Structure):
-    _fields_ = [("kind", ctypes.c_int32), ("sink", ctypes.c_int32), ("window", ctypes.c_int32)]
+    _fields_ = [("kind", ctypes.c_int32), ("sink", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("top_p", ctypes.c_float)]
 
 
 class sp_problem(ctypes.Structure):
@@ -53,7 +54,8 @@ class sp_problem(ctypes.Structure):
                 ("policy", ctypes.POINTER(sp_head_policy)), ("first_page", ctypes.c_int64),
                 ("page_ids", ctypes.POINTER(ctypes.c_int32)), ("target_ctas", ctypes.c_int32),
                 ("flags", ctypes.c_uint32), ("append_capacity", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
-                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
+                ("block_mass", ctypes.POINTER(ctypes.POINTER(ctypes.c_float)))]
 
 
 class sp_sizes(ctypes.Structure):
@@ -141,25 +143,46 @@ def _check(st: int, where: str) -> None:
 # ---------------------------------------------------------------------------
 
 def make_problem(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, page_size: int, dtype: str,
-                 ctx_len: Sequence[int], q_start: Sequence[int], policy: Sequence[tuple[str, int, int]],
+                 ctx_len: Sequence[int], q_start: Sequence[int], policy: Sequence[tuple],
                  first_page: int = 0, page_ids: Sequence[int] | None = None, target_ctas: int = 0,
                  flags: int = 0, append_capacity: int = 0, kv_dtype: str | int | None = None,
-                 k_scale: float = 1.0, v_scale: float = 1.0):
-    """Build an ``sp_problem`` plus the host arrays it points to (kept alive in the result)."""
+                 k_scale: float = 1.0, v_scale: float = 1.0, block_mass: Sequence | None = None):
+    """Build an ``sp_problem`` plus the host arrays it points to (kept alive in the result).
+
+    ``policy`` entries are ``(kind, sink, window)`` or, for retrieval heads,
+    ``(kind, sink, window, top_p)``; ``block_mass`` is None or one entry per
+    (sequence, kv-head): the importance of each page-size block (a float
+    sequence) for a retrieval head, None for the others.
+    """
     B = batch
     ctx = (ctypes.c_int32 * B)(*ctx_len)
     q0 = (ctypes.c_int32 * B)(*q_start)
-    pol = (sp_head_policy * len(policy))(*[sp_head_policy(KIND_CODES[k] if isinstance(k, str) else k, s, w)
-                                           for k, s, w in policy])
+    pol = (sp_head_policy * len(policy))(*[
+        sp_head_policy(KIND_CODES[e[0]] if isinstance(e[0], str) else e[0], e[1], e[2],
+                       float(e[3]) if len(e) > 3 else 0.0) for e in policy])
     ids = (ctypes.c_int32 * len(page_ids))(*page_ids) if page_ids is not None else None
+    masses, mass_ptrs = [], None
+    if block_mass is not None:
+        fp = ctypes.POINTER(ctypes.c_float)
+        ptrs = []
+        for m in block_mass:
+            if m is None:
+                ptrs.append(fp())
+            else:
+                arr = (ctypes.c_float * max(1, len(m)))(*[float(x) for x in m])
+                masses.append(arr)
+                ptrs.append(ctypes.cast(arr, fp))
+        mass_ptrs = (fp * len(ptrs))(*ptrs)
     prob = sp_problem(B, num_q_heads, num_kv_heads, head_dim, page_size,
                       DTYPE_CODES[dtype] if isinstance(dtype, str) else dtype,
                       ctx, q0, pol, first_page,
                       ctypes.cast(ids, ctypes.POINTER(ctypes.c_int32)) if ids is not None else None,
                       target_ctas, flags, append_capacity,
                       0 if kv_dtype is None else (DTYPE_CODES[kv_dtype] if isinstance(kv_dtype, str) else kv_dtype),
-                      k_scale, v_scale)
-    prob._keep = (ctx, q0, pol, ids)
+                      k_scale, v_scale,
+                      ctypes.cast(mass_ptrs, ctypes.POINTER(ctypes.POINTER(ctypes.c_float)))
+                      if mass_ptrs is not None else None)
+    prob._keep = (ctx, q0, pol, ids, masses, mass_ptrs)
     return prob
 
 
@@ -188,8 +211,10 @@ def segpaged_plan_sizes(plan: int) -> sp_sizes:
 
 def segpaged_plan_head_segments(plan: int, b: int, kv: int) -> list[tuple[int, int, int, int]]:
     n = ctypes.c_int32()
-    segs = (sp_segment * 4)()
-    _check(load().segpaged_plan_head_segments(plan, b, kv, segs, 4, ctypes.byref(n)), "segpaged_plan_head_segments")
+    _check(load().segpaged_plan_head_segments(plan, b, kv, None, 0, ctypes.byref(n)), "segpaged_plan_head_segments")
+    segs = (sp_segment * max(1, n.value))()
+    _check(load().segpaged_plan_head_segments(plan, b, kv, segs, n.value, ctypes.byref(n)),
+           "segpaged_plan_head_segments")
     return [(s.abs_start, s.length, s.first_page_index, s.num_pages) for s in segs[: n.value]]
 
 

@@ -2,10 +2,13 @@
 
 This module is shared by the CUDA path's tests and benchmark and by the CPU
 oracle's tests.  It holds shapes, head policies and random numbers only: none
-of the method's arithmetic (visible sets, stored sets, page layout, softmax)
-lives here.  Head policies are plain tuples ``(kind, sink, window)`` with
-``kind`` one of the strings ``"global"``, ``"local"`` or ``"dense"``; each side
-maps the strings to its own codes.
+of the method's arithmetic (visible sets, stored sets, page layout, softmax,
+the retrieval heads' block choice) lives here.  Head policies are plain
+tuples ``(kind, sink, window)`` with ``kind`` one of the strings
+``"global"``, ``"local"`` or ``"dense"``, or ``("retrieval", sink, window,
+top_p)``; each side maps the strings to its own codes.  A retrieval head's
+importance per page-size block is a seeded synthetic draw (``block_mass``)
+that both sides receive as an input.
 
 The shapes follow the synthetic layers of the SegPagedAttention write-ups
 (head-aware paged KV cache; "RedKnot SegPagedAttention runtime design", §2 head
@@ -31,7 +34,7 @@ from typing import Sequence
 import torch
 
 BLOCK_ROWS = 1024
-_TENSOR_IDS = {"q": 1, "k": 2, "v": 3}
+_TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "mass": 4}
 _MASK64 = (1 << 64) - 1
 
 
@@ -67,6 +70,20 @@ def normal_rows(cfg_seed: int, tensor: str, b: int, head: int, r0: int, r1: int,
     return torch.cat(out, 0)
 
 
+def block_mass(cfg_seed: int, b: int, kv: int, n_blocks: int) -> list[float]:
+    """Synthetic importance of the first n_blocks page-size blocks of (sequence b, kv-head kv).
+
+    Heavy-tailed and seeded: exp(2 z) with z ~ N(0, 1) i.i.d. per block (a
+    lognormal stand-in for a head's attention mass per page, which is
+    concentrated on a few pages), rounded to float32.  The stream of a head
+    does not depend on n_blocks: a longer context extends it.
+    """
+    if n_blocks <= 0:
+        return []
+    z = normal_rows(cfg_seed, "mass", b, kv, 0, -(-n_blocks // 64), 64).flatten()[:n_blocks]
+    return [float(x) for x in torch.exp(2.0 * z.double()).float()]
+
+
 def torch_dtype(name: str) -> torch.dtype:
     return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
 
@@ -91,7 +108,7 @@ class Workload:
     dtype: str
     page_size: int
     ctx_lens: tuple[int, ...]
-    policy: tuple[tuple[str, int, int], ...]
+    policy: tuple[tuple, ...]
     prefill_chunk: int | None = None
     prefill_ctx_lens: tuple[int, ...] | None = None
     note: str = ""
@@ -99,6 +116,10 @@ class Workload:
     @property
     def group(self) -> int:
         return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def has_retrieval(self) -> bool:
+        return any(p[0] == "retrieval" for p in self.policy)
 
     def decode_problem(self) -> "Problem":
         return Problem(self, tuple(self.ctx_lens), tuple(L - 1 for L in self.ctx_lens))
@@ -131,6 +152,16 @@ class Problem:
     @property
     def total_queries(self) -> int:
         return sum(self.q_counts)
+
+    def block_masses(self) -> list[list[float] | None]:
+        """Per (sequence, kv-head): the importance of each page-size block for a retrieval head, else None."""
+        wl = self.wl
+        out = []
+        for b, L in enumerate(self.ctx_lens):
+            for kv in range(wl.num_kv_heads):
+                pol = wl.policy[b * wl.num_kv_heads + kv]
+                out.append(block_mass(wl.seed, b, kv, -(-L // wl.page_size)) if pol[0] == "retrieval" else None)
+        return out
 
 
 # --------------------------------------------------------------------------
@@ -240,12 +271,33 @@ def mha() -> Workload:
                     prefill_chunk=4096)
 
 
+def llama_retrieval(batch: int = 8, top_p: float = 0.5) -> Workload:
+    """The Llama-70B-shaped 32K layer with retrieval heads: per sequence the layer's global
+    kv-head, two retrieval kv-heads (sink 4, window 512, top_p) and five local ones (sink 4,
+    window 8192).  The pages give no retrieval share for this model; two of eight is this
+    workload's choice.  Block importance: ``block_mass`` draws."""
+    g = llama_layer_globals()[0]
+    rest = [h for h in range(8) if h != g]
+    retr = set(rest[:2])
+    row = tuple(GLOBAL if h == g else ("retrieval", 4, 512, top_p) if h in retr else _local(4, 8192)
+                for h in range(8))
+    name = "llama_retrieval" if batch == 8 else f"llama_retrieval_b{batch}"
+    return Workload(name, 5, batch, 64, 8, 128, "bf16", 64, (32768,) * batch, row * batch, prefill_chunk=4096)
+
+
+def tiny_retrieval() -> Workload:
+    """The tiny layer (fp32, page 16) with kv-head 1 a retrieval head (sink 4, window 32, top_p 0.6)."""
+    return Workload("tiny_retrieval", 6, 1, 4, 2, 64, "f32", 16, (257,),
+                    (GLOBAL, ("retrieval", 4, 32, 0.6)), prefill_chunk=256, prefill_ctx_lens=(256,))
+
+
 ALL = {"tiny": tiny, "mistral": mistral, "llama": llama, "ragged": ragged, "mha": mha,
-       "llama_b1": lambda: llama(batch=1)}
+       "llama_b1": lambda: llama(batch=1), "llama_retrieval": llama_retrieval,
+       "tiny_retrieval": tiny_retrieval}
 
 
 def custom(name: str, seed: int, batch: int, hq: int, hkv: int, d: int, dtype: str, page: int,
-           ctx_lens: Sequence[int], policy: Sequence[tuple[str, int, int]],
+           ctx_lens: Sequence[int], policy: Sequence[tuple],
            chunk: int | None = None) -> Workload:
     """A hand-made workload for edge-case tests."""
     assert len(policy) == batch * hkv

@@ -46,7 +46,7 @@ extern "C" {
 #define SP_API
 #endif
 
-#define SEGPAGED_ABI_VERSION 1
+#define SEGPAGED_ABI_VERSION 2
 
 /* stride_seq value selecting sequences packed back to back (varlen). */
 #define SP_VARLEN (-1)
@@ -62,9 +62,19 @@ typedef enum {
 
 /* Head kinds ("RedKnot head classification", four-kind table).  DENSE reads
  * the full causal context like GLOBAL (its RoPE re-alignment belongs to KV
- * reuse, outside attention).  RETRIEVAL (pages fetched on demand) is not
- * implemented: the pages give no rule for choosing the pages; it returns
- * SP_ERR_UNSUPPORTED. */
+ * reuse, outside attention).  RETRIEVAL has the whole context as candidates
+ * but keeps only its top-p important tokens, fetched page by page (same
+ * table; "SegPagedAttention runtime design", closing summary: retrieval heads
+ * fetch pages on demand).  The pages give no scoring rule; this library's
+ * reading: the caller gives an importance per block of page_size positions
+ * (sp_problem.block_mass, e.g. the head's attention mass per page); the head
+ * keeps its first `sink` tokens and its `window` most recent tokens, like a
+ * LOCAL head, plus the fewest blocks that, taken in decreasing importance
+ * (ties: the lower block first), reach the fraction top_p of the total
+ * importance of the candidate blocks (those holding a position >= sink); sums
+ * run in fp64 in that order.  top_p >= 1 keeps every block (the head is then
+ * GLOBAL), top_p <= 0 none (LOCAL).  A query at position p sees the kept
+ * blocks' positions up to p, the sink and its window. */
 typedef enum { SP_GLOBAL = 0, SP_LOCAL = 1, SP_DENSE = 2, SP_RETRIEVAL = 3 } sp_kind;
 
 /* SP_E4M3 is a page type only (sp_problem.kv_dtype): FP8 E4M3 codes, 1 byte. */
@@ -90,14 +100,15 @@ enum {
 };
 
 /* Policy of one (sequence, kv-head).  `sink` >= 0 and `window` are read for
- * SP_LOCAL only.  window >= 1 is a fixed window; window <= -1 is an adaptive
- * window of max(1, ctx_len / -window) tokens for that sequence ("RedKnot head
- * classification", adaptive window: e.g. -2 gives ctx_len // 2).  window == 0
- * is invalid. */
+ * SP_LOCAL and SP_RETRIEVAL.  window >= 1 is a fixed window; window <= -1 is
+ * an adaptive window of max(1, ctx_len / -window) tokens for that sequence
+ * ("RedKnot head classification", adaptive window: e.g. -2 gives ctx_len // 2).
+ * window == 0 is invalid.  `top_p` (finite) is read for SP_RETRIEVAL only. */
 typedef struct {
   int32_t kind;
   int32_t sink;
   int32_t window;
+  float top_p;
 } sp_head_policy;
 
 /* One attention layer's batch.  All arrays are host memory, copied by
@@ -127,6 +138,13 @@ typedef struct {
  *               halves the bytes decode reads.  The pages say the system works
  *               with FP8 quantisation ("RedKnot overview (aipuzi)", FAQ Q5); the
  *               per-layer scale is this library's reading.
+ *   block_mass  NULL when no head is SP_RETRIEVAL; else [batch * num_kv_heads]
+ *               host pointers, (b, kv) order: the entry of a retrieval head
+ *               points to ceil(ctx_len[b] / page_size) finite, non-negative
+ *               floats, the importance of positions [i * page_size,
+ *               (i + 1) * page_size); other entries are ignored.  Copied (as
+ *               the kept-block choice) by segpaged_plan_create.  Retrieval
+ *               heads are not supported in ring plans (SP_ERR_UNSUPPORTED).
  */
 typedef struct {
   int32_t batch;
@@ -145,6 +163,7 @@ typedef struct {
   int32_t append_capacity; /* ring plans: tokens every sequence may still gain */
   int32_t kv_dtype;        /* page type: 0 = dtype, or SP_E4M3 (bf16 decode plans) */
   float k_scale, v_scale;  /* SP_E4M3 pages: stored code = E4M3(x * (1 / scale)) */
+  const float* const* block_mass; /* SP_RETRIEVAL heads: importance per page-size block */
 } sp_problem;
 
 typedef struct {
@@ -178,8 +197,11 @@ typedef struct sp_plan sp_plan;
  * §3 SegmentPageTable: page ids per head segment plus per-head policy).  Host
  * only, no CUDA call.  For each (b, kv): GLOBAL/DENSE keep one segment
  * [0, L); LOCAL keeps [0, min(sink, L)) and [max(sink, q0 - window + 1), L),
- * the union of what the call's queries see (merged when they touch).  Each
- * segment starts on a fresh page.  The plan also holds the decode split list
+ * the union of what the call's queries see (merged when they touch);
+ * RETRIEVAL keeps the LOCAL runs plus its kept blocks (in prefill plans a
+ * run that every query sees causally, sink or kept blocks, is a segment of
+ * its own, apart from the window's runs).  Each segment starts on a fresh
+ * page.  The plan also holds the decode split list
  * and the prefill tile list, so that no layout work happens per attention
  * call (same page, §5: layout computed on every call cost a 0.70x slowdown).
  * The plan is immutable and may be shared by several streams. */

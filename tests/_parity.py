@@ -7,6 +7,7 @@ import numpy as np
 import torch
 
 import oracle
+from _retrieval import oracle_head
 
 # Tolerances of the attention outputs against the fp64 oracle: per-head
 # cosine >= 0.99998 ("SegPagedAttention runtime design", §4 verify_against_dense)
@@ -22,7 +23,7 @@ def oracle_rows(prob, q_host, k_host, v_host, b, h, rows=None):
     """Oracle output for (sequence b, q-head h) at varlen rows `rows` (indices within the sequence)."""
     wl = prob.wl
     kv = h // wl.group
-    kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+    kind, s, w, extra = oracle_head(prob, b, kv)
     L, q0 = prob.ctx_lens[b], prob.q_starts[b]
     C = L - q0
     rows = np.arange(C) if rows is None else np.asarray(rows)
@@ -31,7 +32,7 @@ def oracle_rows(prob, q_host, k_host, v_host, b, h, rows=None):
     q = q_host[torch.as_tensor(off + rows, device=q_host.device), h].cpu().double().numpy()
     k = k_host[b, kv, :L].cpu().double().numpy()
     v = v_host[b, kv, :L].cpu().double().numpy()
-    return oracle.attention_rows(q, q0 + rows, k, v, kind, s, w)
+    return oracle.attention_rows(q, q0 + rows, k, v, kind, s, w, **extra)
 
 
 def compare(prob, q_host, k_host, v_host, out, lse, rows_per_seq=None, heads=None, seqs=None):
@@ -65,8 +66,10 @@ def compare(prob, q_host, k_host, v_host, out, lse, rows_per_seq=None, heads=Non
             used += 16 * prob.ctx_lens[keys[i][0]] * wl.head_dim
             i += 1
         groups, meta = [], []
+        masses = prob.block_masses() if wl.has_retrieval else None
         for b, kv in chunk:
-            kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
+            kind, s, w, extra = oracle_head(prob, b, kv, masses)
+            ext = (extra["sel"], extra["block"]) if extra else ()
             L, q0 = prob.ctx_lens[b], prob.q_starts[b]
             off = prob.q_offsets[b]
             k = k_host[b, kv, :L].cpu().double().numpy()
@@ -74,7 +77,7 @@ def compare(prob, q_host, k_host, v_host, out, lse, rows_per_seq=None, heads=Non
             for h, ridx in tasks[(b, kv)]:
                 # inputs may live on the GPU (large layers are generated there): copy the slices
                 q = q_host[torch.as_tensor(off + ridx, device=q_host.device), h].cpu().double().numpy()
-                groups.append((q, q0 + ridx, k, v, kind, s, w))
+                groups.append((q, q0 + ridx, k, v, kind, s, w) + ext)
                 meta.append((b, h, off + ridx))
         res = oracle.attention_batch(groups)
         for (b, h, idx), (o_ref, l_ref) in zip(meta, res):

@@ -33,7 +33,7 @@ def test_library_exports_every_header_symbol():
     lib = S.load()
     for n in names:
         assert getattr(lib, n) is not None
-    assert S.segpaged_abi_version() == 1
+    assert S.segpaged_abi_version() == 2
     assert S.status_name(S.SP_ERR_WORKSPACE) == "SP_ERR_WORKSPACE"
 
 
@@ -162,7 +162,7 @@ BASE = dict(batch=1, num_q_heads=4, num_kv_heads=2, head_dim=64, page_size=16, d
     (dict(policy=[("global", 0, 0), ("local", -1, -2)]), S.SP_ERR_INVALID_ARG),
     (dict(policy=[("global", 0, 0), ("local", -1, 8)]), S.SP_ERR_INVALID_ARG),
     (dict(policy=[("global", 0, 0), (7, 0, 8)]), S.SP_ERR_INVALID_ARG),
-    (dict(policy=[("global", 0, 0), ("retrieval", 0, 0)]), S.SP_ERR_UNSUPPORTED),
+    (dict(policy=[("global", 0, 0), ("retrieval", 4, 8, 0.5)]), S.SP_ERR_INVALID_ARG),  # no block_mass
     (dict(head_dim=96), S.SP_ERR_UNSUPPORTED),
     (dict(dtype=5), S.SP_ERR_UNSUPPORTED),
     (dict(dtype="bf16"), S.SP_ERR_UNSUPPORTED),  # bf16 needs page 64

@@ -96,19 +96,25 @@ def test_clock_sampler_takes_median_max_and_active_reasons():
     assert cs.stop() is None
 
 
-def test_kernel_traffic_only_while_the_source_is_unchanged(tmp_path):
+def test_kernel_traffic_only_while_the_source_is_unchanged(tmp_path, monkeypatch):
     """DRAM bytes come from profiles/traffic.json only for the captured workload and kernel source."""
+    import hashlib
     import json
-    rec = json.loads((bench.ROOT / "profiles" / "traffic.json").read_text())
-    csrc = bench.ROOT / "head_aware_paged_build_b200" / "csrc"
-    for kernel, src in (("decode_mma_kernel", "kernels_decode.cu"), ("prefill_tc_kernel", "kernels_prefill_tc.cu")):
-        key = rec[kernel]["workload_key"]
-        assert bench.kernel_traffic(kernel, csrc / src, key) == rec[kernel]["bytes_per_launch"]
-        assert bench.kernel_traffic(kernel, csrc / src, key + "_other") is None
-        changed = tmp_path / src
-        changed.write_bytes((csrc / src).read_bytes() + b"\n// changed\n")
-        assert bench.kernel_traffic(kernel, changed, key) is None
-    assert bench.kernel_traffic("no_such_kernel", csrc / "kernels_decode.cu", "llama_l0") is None
+    src = tmp_path / "kernel.cu"
+    src.write_text("// a kernel\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"k": {"bytes_per_launch": 123, "source_sha16": sha, "workload_key": "llama_l0"}}))
+    monkeypatch.setattr(bench, "ROOT", tmp_path)
+    assert bench.kernel_traffic("k", src, "llama_l0") == 123
+    assert bench.kernel_traffic("k", src, "llama_l0_other") is None
+    assert bench.kernel_traffic("no_such_kernel", src, "llama_l0") is None
+    src.write_text("// a kernel, changed\n")
+    assert bench.kernel_traffic("k", src, "llama_l0") is None
+    # the committed record names the bench's kernels and workload
+    rec = json.loads((Path(__file__).resolve().parent.parent / "profiles" / "traffic.json").read_text())
+    assert {"prefill_tc_kernel", "decode_mma_kernel"} <= set(rec)
 
 
 def test_weak_rate_and_config():

@@ -9,6 +9,7 @@ import oracle
 from head_aware_paged_build_b200 import segpaged as S
 from head_aware_paged_build_b200 import workloads as W
 from head_aware_paged_build_b200.runtime import layer_for
+from _retrieval import oracle_head
 
 pytestmark = pytest.mark.gpu
 
@@ -41,8 +42,8 @@ def check_pack(prob, flags=0, **kw):
     for b in range(wl.batch):
         L, q0 = prob.ctx_lens[b], prob.q_starts[b]
         for kv in range(wl.num_kv_heads):
-            kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
-            m = oracle.stored_mask("global" if dense_masked else kind, s, w, L, q0)
+            kind, s, w, extra = oracle_head(prob, b, kv)
+            m = oracle.stored_mask("global" if dense_masked else kind, s, w, L, q0, **extra)
             mt = torch.from_numpy(m)
             stored_total += int(m.sum())
             assert torch.equal(kob[b, kv, :L][mt], kb[b, kv, :L][mt]), (b, kv)
@@ -74,10 +75,10 @@ def check_pack_full_size(prob):
     for b in range(wl.batch):
         L, q0 = prob.ctx_lens[b], prob.q_starts[b]
         for kv in range(wl.num_kv_heads):
-            kind, s, w = wl.policy[b * wl.num_kv_heads + kv]
-            key = (kind, s, w, L, q0)
+            kind, s, w, extra = oracle_head(prob, b, kv)
+            key = (kind, s, w, L, q0) if not extra else (b, kv)
             if key not in masks:
-                masks[key] = torch.from_numpy(oracle.stored_mask(kind, s, w, L, q0)).cuda()
+                masks[key] = torch.from_numpy(oracle.stored_mask(kind, s, w, L, q0, **extra)).cuda()
             mt = masks[key]
             stored_total += int(mt.sum())
             assert torch.equal(kob[b, kv, :L][mt], kb[b, kv, :L][mt]), (b, kv)
