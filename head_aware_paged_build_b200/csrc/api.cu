@@ -269,6 +269,40 @@ sp_status segpaged_decode_append(const sp_plan* plan, void* d_table, const void*
   return e == cudaSuccess ? SP_OK : cuda_fail(e, "segpaged_decode_append launch");
 }
 
+sp_status segpaged_decode_step(const sp_plan* plan, void* d_table, const void* k_new, const void* v_new,
+                               int64_t stride_seq, int64_t stride_head, void* k_pool, void* v_pool, const void* q,
+                               void* out, float* lse, float softmax_scale, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  using namespace sp;
+  sp_status st = check_attention_args(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale);
+  if (st != SP_OK) return st;
+  if (!(plan->prob.flags & SP_FLAG_RING)) return fail(SP_ERR_INVALID_ARG, "segpaged_decode_step needs a ring plan");
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16))
+    return fail(SP_ERR_INVALID_ARG, "k_new and v_new must be non-NULL and 16-byte aligned");
+  const int64_t eb = plan->elem_bytes;
+  if (stride_seq < 0 || stride_head < 0 || (stride_seq * eb) % 16 || (stride_head * eb) % 16)
+    return fail(SP_ERR_INVALID_ARG, "strides must be >= 0 and give 16-byte aligned rows");
+  if (!workspace || !aligned(workspace, 256)) return fail(SP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (int64_t(workspace_bytes) < plan->sizes.workspace_bytes)
+    return fail(SP_ERR_WORKSPACE, "workspace smaller than workspace_bytes");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (plan->prob.dtype != SP_BF16) {  // fp32 pages: the append kernel, then the decode kernels
+    st = segpaged_decode_append(plan, d_table, k_new, v_new, stride_seq, stride_head, k_pool, v_pool, workspace,
+                                stream);
+    if (st != SP_OK) return st;
+    return segpaged_attention(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale, workspace,
+                              workspace_bytes, stream);
+  }
+  DecodeLaunch L = decode_launch_of(plan, d_table, k_pool, v_pool, q, out, lse, softmax_scale, workspace,
+                                    static_cast<int32_t*>(workspace));
+  L.append = true;
+  L.k_new = k_new, L.v_new = v_new;
+  L.new_stride_seq = stride_seq, L.new_stride_head = stride_head;
+  L.k_inv = 1.0f / plan->k_scale, L.v_inv = 1.0f / plan->v_scale;
+  const cudaError_t e = launch_decode(L, s);
+  return e == cudaSuccess ? SP_OK : cuda_fail(e, "segpaged_decode_step launch");
+}
+
 sp_status segpaged_read_device_status(const void* workspace, int32_t* code, void* stream) {
   if (!workspace || !code) return sp::fail(SP_ERR_INVALID_ARG, "workspace and code must be non-NULL");
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -128,6 +128,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Order this thread's earlier generic-proxy global writes before later
+// async-proxy accesses (bulk copies) of the same memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // --------------------------------------------------------------------------
 // Bulk (non-tensor) asynchronous copy global -> shared, completing on an mbarrier.
 // Both addresses 16-byte aligned, size a multiple of 16.

@@ -65,6 +65,14 @@ struct DecodeLaunch {
   float* partial;    // workspace partial slots
   int32_t* counters; // workspace arrival counters of split heads (zero between calls)
   int32_t* status;
+  // Fused decode step of a ring plan (bf16 / E4M3 pages): before attending, each
+  // CTA appends the new token of the heads whose target or evicted page lies in
+  // its page range, and the CTA that finishes a head advances its context.
+  bool append;
+  const void* k_new;   // [B, Hkv, D] bf16 rows, strides in elements
+  const void* v_new;
+  int64_t new_stride_seq, new_stride_head;
+  float k_inv, v_inv;  // E4M3 pages: 1 / k_scale, 1 / v_scale
 };
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t s);
 

@@ -27,6 +27,7 @@
 // separate combine pass for split heads.
 #include <cmath>
 
+#include "append_common.cuh"
 #include "device_common.cuh"
 #include "kernels.h"
 
@@ -155,8 +156,71 @@ __device__ __forceinline__ void merge_split_head(const DecodeLaunch& a, const He
         (row_m[threadIdx.x] + log2f(row_l[threadIdx.x])) * kLn2;
 }
 
-template <int D, int NST, bool FP8>
-__global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch a) {
+// Fused decode step: the new token of head `hd` has been written by the CTA
+// that owns its target page; the CTA finishing the head (its single item, or
+// the final merge of a split head) advances the context, exactly as the
+// standalone append does after writing (or reports a ring without room).
+template <int P>
+__device__ __noinline__ void finish_append(const DecodeLaunch& a, int head) {
+  // re-read from the table (not kept in registers through the page loop); no
+  // thread writes this head's descriptor before this point of the launch
+  const HeadDesc hd = a.heads[head];
+  int vp, slot;
+  append_target<P>(hd, vp, slot);
+  if (vp >= hd.n_vpages) {
+    record_error(a.status, kDevAppendFull);
+    return;
+  }
+  const int64_t phys = a.pages[hd.vpage_begin + vp].phys;
+  if (phys < 0 || phys >= a.pool_pages) return;  // reported where the page was met
+  HeadDesc* w = const_cast<HeadDesc*>(a.heads) + head;
+  w->ctx_len = hd.ctx_len + 1;
+  w->q_start = hd.ctx_len;
+}
+
+// Producer-warp prologue of the fused decode step: for each item of this CTA,
+// append the head's new token if its target page lies in the item's page range,
+// and evict the token that leaves the window if that token's page does.  The
+// writes are ordered before the warp's bulk copies of the same pages.
+template <int D, bool FP8>
+__device__ __forceinline__ void append_prologue(const DecodeLaunch& a, int ib, int ie, int lane) {
+  constexpr int P = 64;
+  PageDesc* pages = const_cast<PageDesc*>(a.pages);
+  for (int it = ib; it < ie; ++it) {
+    const DecodeItem item = a.items[it];
+    const HeadDesc hd = a.heads[item.head];
+    int vp, slot;
+    append_target<P>(hd, vp, slot);
+    if (vp >= hd.n_vpages) continue;  // no room: the head's finisher reports it
+    PageDesc* pg = pages + hd.vpage_begin + vp;
+    const int64_t phys = pg->phys;
+    if (phys < 0 || phys >= a.pool_pages) continue;  // corrupted table: the producer reports the page
+    const int g = hd.vpage_begin + vp;
+    if (g >= item.vp_begin && g < item.vp_end) {
+      const __nv_bfloat16* kn = static_cast<const __nv_bfloat16*>(a.k_new) + int64_t(hd.b) * a.new_stride_seq +
+                                int64_t(hd.kv) * a.new_stride_head;
+      const __nv_bfloat16* vn = static_cast<const __nv_bfloat16*>(a.v_new) + int64_t(hd.b) * a.new_stride_seq +
+                                int64_t(hd.kv) * a.new_stride_head;
+      append_write_token<__nv_bfloat16, D, P, FP8>(
+          kn, vn, static_cast<uint8_t*>(const_cast<void*>(a.kpool)) + phys * a.page_bytes,
+          static_cast<uint8_t*>(const_cast<void*>(a.vpool)) + phys * a.page_bytes, slot, a.k_inv, a.v_inv, lane, 32);
+      if (lane == 0) append_update_target(pg, hd.ctx_len, slot);
+    }
+    int evp, eslot, epos;
+    append_eviction<P>(hd, evp, eslot, epos);
+    if (evp >= 0 && lane == 0) {
+      const int ge = hd.vpage_begin + evp;
+      if (ge >= item.vp_begin && ge < item.vp_end) append_update_eviction(pages + ge, epos, eslot);
+    }
+    __syncwarp();
+  }
+  fence_proxy_async_global();  // the token's bytes before this warp's bulk copies of its page
+  __threadfence_block();
+  __syncwarp();
+}
+
+template <int D, int NST, bool FP8, bool APPEND>
+__device__ __forceinline__ void decode_mma_body(const DecodeLaunch& a) {
   using S = DecodeSmem<D, NST, FP8>;
   constexpr int P = 64;
   constexpr int PB = S::kPageBytes;
@@ -196,8 +260,11 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch
     // the stage's full barrier), start the copies.
     int k = 0;
     bool ok = true;
+    if constexpr (APPEND) append_prologue<D, FP8>(a, ib, ie, lane);
     for (int base = gb; base < ge && ok; base += 32) {
-      const int4 mine = base + lane < ge ? __ldg(reinterpret_cast<const int4*>(a.pages + base + lane))
+      // page records this launch may have changed (fused append) are read through L2
+      const int4 mine = base + lane < ge ? (APPEND ? __ldcg(reinterpret_cast<const int4*>(a.pages + base + lane))
+                                                   : __ldg(reinterpret_cast<const int4*>(a.pages + base + lane)))
                                          : make_int4(0, 0, 0, 0);
       const int n = min(32, ge - base);
       for (int i = 0; i < n; ++i, ++k) {
@@ -448,6 +515,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch
         if (col == 0) slot[G * D + row * 2] = M, slot[G * D + row * 2 + 1] = L;
       }
     }
+    if constexpr (APPEND) {
+      if (item.slot < 0 && threadIdx.x == 0) finish_append<64>(a, item.head);
+    }
     if (item.slot >= 0) {
       // Split head: publish this partial, take a ticket; the last CTA to arrive
       // merges in slot order (fixed order: bitwise reproducible) and returns
@@ -483,7 +553,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch
             else
               merge_split_head<D, 4, 4, false>(a, hd, qh0, G, n_src, src, part, mbuf, mlbuf, warp, lane);
             if (part == nullptr) {
-              if (threadIdx.x == 0) a.counters[item.comb] = 0;
+              if (threadIdx.x == 0) {
+                a.counters[item.comb] = 0;
+                if constexpr (APPEND) finish_append<64>(a, item.head);
+              }
               break;
             }
             // group merged: reset its counter, publish the group slot, ticket on the head
@@ -545,12 +618,27 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch
           if (threadIdx.x < G && a.lse)
             a.lse[int64_t(hd.q_row0) * a.num_q_heads + qh0 + threadIdx.x] =
                 (row_m[threadIdx.x] + log2f(row_l[threadIdx.x])) * kLn2;
-          if (threadIdx.x == 0) a.counters[item.comb] = 0;
+          if (threadIdx.x == 0) {
+            a.counters[item.comb] = 0;
+            if constexpr (APPEND) finish_append<64>(a, item.head);
+          }
         }
       }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
   }
+}
+
+// The decode kernel, and the fused decode step (append + decode), which must
+// keep two CTAs on every SM: its prologue would otherwise raise the register
+// count past the 168 that two 5-warp CTAs leave each thread.
+template <int D, int NST, bool FP8>
+__global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch a) {
+  decode_mma_body<D, NST, FP8, false>(a);
+}
+template <int D, int NST, bool FP8>
+__global__ void __launch_bounds__(kDecodeThreads, 2) decode_step_kernel(DecodeLaunch a) {
+  decode_mma_body<D, NST, FP8, true>(a);
 }
 
 // ---------------------------------------------------------------------------
@@ -697,7 +785,7 @@ template <int D, bool FP8>
 cudaError_t launch_mma(const DecodeLaunch& a, cudaStream_t s) {
   constexpr int NST = FP8 ? kStagesFp8 : kStagesBf16;
   using Sm = DecodeSmem<D, NST, FP8>;
-  auto kern = decode_mma_kernel<D, NST, FP8>;
+  auto kern = a.append ? decode_step_kernel<D, NST, FP8> : decode_mma_kernel<D, NST, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kBytes);
   if (e != cudaSuccess) return e;
   kern<<<a.n_ctas, kDecodeThreads, Sm::kBytes, s>>>(a);  // split heads are merged in-kernel

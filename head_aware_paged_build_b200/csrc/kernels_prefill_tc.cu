@@ -27,10 +27,16 @@
 //   warps 2-9   softmax of tile A, warps 10-17 softmax of tile B: two threads
 //               per row, each owning one of the KV tile's two pages (64
 //               columns); S read with tcgen05.ld, online softmax in the log2
-//               domain with the row maximum exchanged between the two halves
-//               through shared memory, a lazy rescale of O (only when the row
-//               maximum grows by more than 2^8), P written back as bf16 over
-//               the half's own first 32 S columns; then the epilogue (O / l, LSE).
+//               domain against a running reference kept per row, a lazy
+//               rescale of O (only when the row maximum grows by more than
+//               2^8), P written back as bf16 over the half's own first 32 S
+//               columns; then the epilogue (O / l, LSE).  Usually one pass:
+//               each 32-column chunk is exponentiated against the reference as
+//               soon as it is read, and the halves only vote; a tile whose
+//               scores outgrow some row's reference takes the two-pass step
+//               (row maxima exchanged between the halves through shared
+//               memory, held-back chunks recomputed from S, stored chunks of
+//               rows whose reference moved rescaled in TMEM).
 // The commit that signals S_x(j) also covers P_x(j-1) V, so a softmax thread
 // holding S_x(j) may rescale O_x and overwrite P_x with no further wait.
 // Every wait is bounded; a wait that runs out records a status code, and the
@@ -45,6 +51,8 @@
 
 namespace sp {
 namespace {
+
+
 
 constexpr int kTile = kPrefillTileTokensBf16;  // 128 query rows, 128 KV tokens
 constexpr int kThreads = 576;
@@ -93,8 +101,7 @@ __device__ __forceinline__ bool page_fully_visible(const PageDesc& pg, bool exis
 // Slots of a page visible to row p: [0, h1) (sink run) and [l2, h2) (causal
 // part / recent window), inside the page's valid range [lo, hi).  A page with
 // lo > 0 never holds sink positions (sink pages always start at slot 0; only
-// ring pages of decode plans start later), so its sink run is empty.  A page
-// flagged kSpanCausal (a retrieval head's sink or kept block) is seen causally.
+// ring pages of decode plans start later), so its sink run is empty.
 __device__ __forceinline__ void visible_slots(const PageDesc& pg, bool exists, const HeadDesc& hd, int p, int& h1,
                                               int& l2, int& h2) {
   h1 = l2 = h2 = 0;
@@ -301,7 +308,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // tcgen05.ld / st are warp-collective: the wait outcome is voted per warp,
         // then across the tile's eight warps at the exchange barrier below.
         const bool got = __all_sync(kFull, mbar_wait(&bars->s_full[x], j & 1));
-        // pass 1: this half's row maximum (S stays in TMEM), one 32-column chunk at a time
         int h1 = 64, l2 = 0, h2 = 0;
         if (!full) visible_slots(pg, have, hd, p, h1, l2, h2);
         auto mask32 = [&](float (&w)[32], int c) {  // chunk c: page slots [32 c, 32 c + 32)
@@ -311,9 +317,40 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if (!(t < h1 || (t >= l2 && t < h2))) w[e] = -INFINITY;
           }
         };
+        auto exp_chunk = [&](const float (&w)[32], uint64_t nbase2, uint32_t (&pk)[16]) -> uint64_t {
+          const uint64_t scale2 = f2_pack(sl2, sl2);
+          uint64_t s2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t x2 = f2_fma(f2_pack(w[2 * e], w[2 * e + 1]), scale2, nbase2);
+            float e0, e1;
+            if (kPolyPeriod > 0 && (e % (kPolyPeriod > 0 ? kPolyPeriod : 1)) == kPolyPeriod - 1) {
+              exp2_poly_pair(x2, e0, e1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              e0 = fast_exp2(x0), e1 = fast_exp2(x1);
+            }
+            s2[e & 1] = f2_add(s2[e & 1], f2_pack(e0, e1));
+            pk[e] = pack_bf16x2(e0, e1);
+          }
+          return f2_add(s2[0], s2[1]);
+        };
+        // One pass: each 32-column chunk's maximum, then P = 2^(s - m_run)
+        // against the row's running reference.  A warp stores a chunk's P only
+        // when all its rows stay within 2^8 of their reference (the weights the
+        // lazy rescale keeps); once a warp holds back a chunk it stores no
+        // more, so that chunk's scores stay in TMEM.  If any row of the tile
+        // outgrew its reference, the tile takes the two-pass step: maxima
+        // exchanged, held-back chunks recomputed from S, stored chunks of rows
+        // whose reference moved rescaled in TMEM.
         float mx = -INFINITY;
+        uint64_t csum[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        int stored = 0;  // chunks of this warp already in TMEM (warp-uniform)
         if (got) {
           tc::fence_after_sync();
+          const float base = m_run == -INFINITY ? 0.f : m_run;
+          const uint64_t nbase2 = f2_pack(-base, -base);
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             float w[32];
@@ -328,70 +365,82 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
               for (int i = 0; i < 4; ++i) m4[i] = fmax3(m4[i], w[e + i], w[e + 4 + i]);
             mx = fmax3(fmax3(m4[0], m4[1], m4[2]), m4[3], mx);
+            const bool fit = m_run != -INFINITY && !(mx * sl2 > m_run + kRescaleLog2);
+            if (stored == c && __all_sync(kFull, fit)) {
+              uint32_t pk[16];
+              csum[c] = exp_chunk(w, nbase2, pk);
+              tc::tmem_st16(t_s(x) + lane_off + 64 * h + 16 * c, pk);
+              stored = c + 1;
+            }
           }
         }
         xch[(j & 1) * 2 * kTile + h * kTile + r] = mx;
-        if (!bar_red_and(bar_id, 8 * 32, got)) {
-          fail(kDevTimeoutMma);
-          ok = false;
-          break;
-        }
-        const float mt = fmaxf(mx, xch[(j & 1) * 2 * kTile + (1 - h) * kTile + r]);
-        const float mts = mt * sl2;
-        float alpha = 1.f;
-        bool need = false;
-        if (mts > m_run + kRescaleLog2) {
-          alpha = fast_exp2(m_run - mts);
-          need = m_run != -INFINITY;
-          m_run = mts;
-        }
-        // pass 2: P = 2^(s - m) in bf16.  This half's page (columns [64 h, 64 h + 64))
-        // becomes P columns [64 h, 64 h + 32), over its own scores already read; one
-        // pair in kPolyPeriod takes its 2^x on the FMA pipe.
-        const float base = m_run == -INFINITY ? 0.f : m_run;
-        const uint64_t scale2 = f2_pack(sl2, sl2), nbase2 = f2_pack(-base, -base);
-        uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float w[32];
-          tc::tmem_ld32(t_s(x) + lane_off + 64 * h + 32 * c, w);
-          tc::tmem_wait_ld();
-          if (!full) mask32(w, c);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint64_t x2 = f2_fma(f2_pack(w[2 * e], w[2 * e + 1]), scale2, nbase2);
-            float e0, e1;
-            if (kPolyPeriod > 0 && (e % (kPolyPeriod > 0 ? kPolyPeriod : 1)) == kPolyPeriod - 1) {
-              exp2_poly_pair(x2, e0, e1);
-            } else {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              e0 = fast_exp2(x0), e1 = fast_exp2(x1);
-            }
-            sum2[e & 1] = f2_add(sum2[e & 1], f2_pack(e0, e1));
-            pk[e] = pack_bf16x2(e0, e1);
+        if (bar_red_and(bar_id, 8 * 32, got && stored == 2)) {
+          float s0, s1, s2, s3;
+          f2_unpack(csum[0], s0, s1);
+          f2_unpack(csum[1], s2, s3);
+          l_run = l_run + ((s0 + s1) + (s2 + s3));
+        } else {
+          if (!bar_red_and(bar_id, 8 * 32, got)) {
+            fail(kDevTimeoutMma);
+            ok = false;
+            break;
           }
-          tc::tmem_st16(t_s(x) + lane_off + 64 * h + 16 * c, pk);
-        }
-        float s0, s1, s2, s3;
-        f2_unpack(sum2[0], s0, s1);
-        f2_unpack(sum2[1], s2, s3);
-        l_run = l_run * alpha + ((s0 + s1) + (s2 + s3));
-        // O_x is stable here: the commit behind s_full also covered P_x(j-1) V, and
-        // P_x(j) V is issued only after this thread arrives on p_full.  This half
-        // rescales its half of the row's O columns (after P, when the scores'
-        // registers are free).
-        if (__any_sync(kFull, need)) {
-          const float f = need ? alpha : 1.f;
+          tc::tmem_wait_st();  // P chunks stored above are read back below
+          const float mt = fmaxf(mx, xch[(j & 1) * 2 * kTile + (1 - h) * kTile + r]);
+          const float mts = mt * sl2;
+          float alpha = 1.f;
+          bool need = false;
+          if (mts > m_run + kRescaleLog2) {
+            alpha = fast_exp2(m_run - mts);
+            need = m_run != -INFINITY;
+            m_run = mts;
+          }
+          const float base = m_run == -INFINITY ? 0.f : m_run;
+          const uint64_t nbase2 = f2_pack(-base, -base);
+          float lsum = 0.f;
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            float o[32];
-            tc::tmem_ld32(t_o(x) + lane_off + h * (D / 2) + c * 32, o);
-            tc::tmem_wait_ld();
+          for (int c = 0; c < 2; ++c) {
+            if (c < stored) {
+              // stored against the old reference: scale by alpha where it moved
+              float s0, s1;
+              f2_unpack(csum[c], s0, s1);
+              lsum += (s0 + s1) * alpha;
+              if (__any_sync(kFull, need)) {
+                uint32_t pk[16];
+                tc::tmem_ld16(t_s(x) + lane_off + 64 * h + 16 * c, pk);
+                tc::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= f;
-            tc::tmem_st32(t_o(x) + lane_off + h * (D / 2) + c * 32, o);
+                for (int e = 0; e < 16; ++e) {
+                  const float lo = __uint_as_float(pk[e] << 16), hi = __uint_as_float(pk[e] & 0xffff0000u);
+                  pk[e] = pack_bf16x2(lo * alpha, hi * alpha);
+                }
+                tc::tmem_st16(t_s(x) + lane_off + 64 * h + 16 * c, pk);
+              }
+            } else {
+              float w[32];
+              tc::tmem_ld32(t_s(x) + lane_off + 64 * h + 32 * c, w);
+              tc::tmem_wait_ld();
+              if (!full) mask32(w, c);
+              uint32_t pk[16];
+              float s0, s1;
+              f2_unpack(exp_chunk(w, nbase2, pk), s0, s1);
+              lsum += s0 + s1;
+              tc::tmem_st16(t_s(x) + lane_off + 64 * h + 16 * c, pk);
+            }
+          }
+          l_run = l_run * alpha + lsum;
+          if (__any_sync(kFull, need)) {
+            const float f = need ? alpha : 1.f;
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+              float o[32];
+              tc::tmem_ld32(t_o(x) + lane_off + h * (D / 2) + c * 32, o);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] *= f;
+              tc::tmem_st32(t_o(x) + lane_off + h * (D / 2) + c * 32, o);
+            }
           }
         }
         tc::tmem_wait_st();

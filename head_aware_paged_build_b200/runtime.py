@@ -134,8 +134,7 @@ class SegPagedLayer:
                              self.workspace.data_ptr(), self.workspace.numel(), _stream(stream))
         return out, lse
 
-    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
-        """Ring plans: add one token per sequence (k_new, v_new: [B, Hkv, d])."""
+    def _check_new_rows(self, k_new: torch.Tensor, v_new: torch.Tensor) -> None:
         self._check_tensor(k_new, "k_new", self.torch_dtype)
         self._check_tensor(v_new, "v_new", self.torch_dtype)
         if (k_new.dim() != 3 or k_new.shape != v_new.shape or k_new.stride() != v_new.stride() or
@@ -143,9 +142,36 @@ class SegPagedLayer:
                 k_new.shape[2] != self.head_dim):
             raise ValueError(f"k_new / v_new must be [{self.batch}, {self.num_kv_heads}, {self.head_dim}] "
                              f"with the same strides, head_dim contiguous; got {tuple(k_new.shape)}")
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
+        """Ring plans: add one token per sequence (k_new, v_new: [B, Hkv, d])."""
+        self._check_new_rows(k_new, v_new)
         S.segpaged_decode_append(self.plan, self.table.data_ptr(), k_new.data_ptr(), v_new.data_ptr(),
                                  k_new.stride(0), k_new.stride(1), self.k_pool.data_ptr(), self.v_pool.data_ptr(),
                                  self.workspace.data_ptr(), _stream(stream))
+
+    def decode_step(self, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor, out: torch.Tensor | None = None,
+                    lse: torch.Tensor | None = None, scale: float = 0.0, stream=None):
+        """Ring plans: append one token per sequence and attend with its queries (q: [B, Hq, d]) in one call;
+        the same results as ``append`` followed by ``attention``.  Returns (out, lse)."""
+        self._check_new_rows(k_new, v_new)
+        rows = (self.sizes.num_queries, self.num_q_heads)
+        self._check_tensor(q, "q", self.torch_dtype)
+        if tuple(q.shape) != rows + (self.head_dim,) or not q.is_contiguous():
+            raise ValueError(f"q must be contiguous {rows + (self.head_dim,)}, got {tuple(q.shape)}")
+        out = torch.empty_like(q) if out is None else out
+        self._check_tensor(out, "out", self.torch_dtype)
+        if out.shape != q.shape or not out.is_contiguous():
+            raise ValueError(f"out must be contiguous {tuple(q.shape)}, got {tuple(out.shape)}")
+        lse = torch.empty(rows, dtype=torch.float32, device=q.device) if lse is None else lse
+        self._check_tensor(lse, "lse", torch.float32)
+        if tuple(lse.shape) != rows or not lse.is_contiguous():
+            raise ValueError(f"lse must be contiguous {rows}, got {tuple(lse.shape)}")
+        S.segpaged_decode_step(self.plan, self.table.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_new.stride(0),
+                               k_new.stride(1), self.k_pool.data_ptr(), self.v_pool.data_ptr(), q.data_ptr(),
+                               out.data_ptr(), lse.data_ptr(), scale, self.workspace.data_ptr(),
+                               self.workspace.numel(), _stream(stream))
+        return out, lse
 
     def device_status(self, stream=None) -> int:
         return S.segpaged_read_device_status(self.workspace.data_ptr(), _stream(stream))
@@ -203,15 +229,16 @@ class DecodeStepGraph:
 
     A step copies the new token's K and V rows ([B, Hkv, d]) and its queries
     ([B, Hq, d]) from the pinned host buffers ``k_in``, ``v_in``, ``q_in``,
-    appends the token (``segpaged_decode_append``), runs decode attention and
-    copies O and LSE into the pinned host buffers ``out`` and ``lse``.  The
-    caller refills the inputs, then calls ``replay()``; every replay appends
-    one more token (the device table advances in place).  The graph holds the
-    same library calls an eager step makes; it removes the per-call launch
-    gaps between them.
+    appends the token and runs decode attention (``segpaged_decode_step``: one
+    launch on bf16 pages; with ``fused=False`` the two calls
+    ``segpaged_decode_append`` and ``segpaged_attention``) and copies O and
+    LSE into the pinned host buffers ``out`` and ``lse``.  The caller refills
+    the inputs, then calls ``replay()``; every replay appends one more token
+    (the device table advances in place).  The graph holds the same library
+    calls an eager step makes; it removes the per-call launch gaps between them.
     """
 
-    def __init__(self, layer: SegPagedLayer, stream: torch.cuda.Stream | None = None):
+    def __init__(self, layer: SegPagedLayer, stream: torch.cuda.Stream | None = None, fused: bool = True):
         if layer.problem.flags & S.SP_FLAG_RING == 0:
             raise ValueError("DecodeStepGraph needs a ring plan (flags=SP_FLAG_RING)")
         if not layer.sizes.is_decode:
@@ -245,8 +272,11 @@ class DecodeStepGraph:
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph, stream=stream):
             self._dev_in.copy_(self._host_in, non_blocking=True)
-            layer.append(self._k, self._v)
-            layer.attention(self._q, self._o, self._lse)
+            if fused:
+                layer.decode_step(self._k, self._v, self._q, self._o, self._lse)
+            else:
+                layer.append(self._k, self._v)
+                layer.attention(self._q, self._o, self._lse)
             self._host_out.copy_(self._dev_out, non_blocking=True)
 
     def replay(self) -> None:

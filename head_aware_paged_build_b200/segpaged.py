@@ -31,7 +31,8 @@ EXPORTED = ("segpaged_plan_create", "segpaged_plan_destroy", "segpaged_plan_size
             "segpaged_plan_head_segments", "segpaged_plan_head_pages", "segpaged_plan_decode_items",
             "segpaged_plan_prefill_items", "segpaged_table_write",
             "build_segpaged_cache", "build_segpaged_cache_layers", "segpaged_gather", "segpaged_attention",
-            "segpaged_attention_decode_noalloc", "segpaged_decode_append", "segpaged_read_device_status",
+            "segpaged_attention_decode_noalloc", "segpaged_decode_append", "segpaged_decode_step",
+            "segpaged_read_device_status",
             "segpaged_clear_device_status", "segpaged_eval_exp2_fma", "segpaged_status_string",
             "segpaged_last_error", "segpaged_abi_version")
 
@@ -109,6 +110,7 @@ def load(path: Path | str | None = None) -> ctypes.CDLL:
         "segpaged_attention": ([vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp], i32),
         "segpaged_attention_decode_noalloc": ([vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp], i32),
         "segpaged_decode_append": ([vp, vp, vp, vp, i64, i64, vp, vp, vp, vp], i32),
+        "segpaged_decode_step": ([vp, vp, vp, vp, i64, i64, vp, vp, vp, vp, vp, ctypes.c_float, vp, sz, vp], i32),
         "segpaged_read_device_status": ([vp, ctypes.POINTER(i32), vp], i32),
         "segpaged_clear_device_status": ([vp, vp], i32),
         "segpaged_eval_exp2_fma": ([vp, vp, i64, vp], i32),
@@ -303,6 +305,14 @@ def segpaged_decode_append(plan: int, d_table: int, k_new: int, v_new: int, stri
     """Append one token per sequence to a ring plan's cache, in place (device table updated)."""
     _check(load().segpaged_decode_append(plan, d_table, k_new, v_new, stride_seq, stride_head, k_pool, v_pool,
                                          workspace, stream), "segpaged_decode_append")
+
+
+def segpaged_decode_step(plan: int, d_table: int, k_new: int, v_new: int, stride_seq: int, stride_head: int,
+                         k_pool: int, v_pool: int, q: int, out: int, lse: int | None, softmax_scale: float,
+                         workspace: int, workspace_bytes: int, stream: int = 0) -> None:
+    """Append one token per sequence to a ring plan's cache and attend with it (one launch on bf16 pages)."""
+    _check(load().segpaged_decode_step(plan, d_table, k_new, v_new, stride_seq, stride_head, k_pool, v_pool, q, out,
+                                       lse, softmax_scale, workspace, workspace_bytes, stream), "segpaged_decode_step")
 
 
 def segpaged_attention_status(*args) -> int:

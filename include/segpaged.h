@@ -398,6 +398,27 @@ SP_API sp_status segpaged_decode_append(const sp_plan* plan, void* d_table, cons
                                         int64_t stride_seq, int64_t stride_head, void* k_pool, void* v_pool,
                                         void* workspace, void* stream);
 
+/* segpaged_decode_step: one serving decode step of a ring plan, the same as
+ * segpaged_decode_append followed by segpaged_attention on the same table,
+ * with bit for bit the same outputs, pool and table ("SegPagedAttention
+ * runtime design", §3: a LOCAL head's window moves without moving tokens; §5:
+ * no layout work per call).  On bf16 and E4M3 pages it is one launch: each
+ * decode CTA appends the new token of the heads whose target page lies in its
+ * page range before streaming those pages, and evicts the token that leaves a
+ * LOCAL window when that token's page is in its range; the CTA that finishes
+ * a head advances its context length.  fp32 pages run the two calls.
+ *   k_new, v_new, stride_seq, stride_head  as segpaged_decode_append
+ *   q    device [batch, num_q_heads, head_dim]: the queries at the new
+ *        positions (each sequence's current context length before the call)
+ *   out, lse, softmax_scale, workspace, workspace_bytes  as segpaged_attention
+ * Errors: as the two calls (a ring without room records device code 6 and
+ * attends over the unchanged context; SP_ERR_INVALID_ARG for a plan that is
+ * not a ring plan). */
+SP_API sp_status segpaged_decode_step(const sp_plan* plan, void* d_table, const void* k_new, const void* v_new,
+                                      int64_t stride_seq, int64_t stride_head, void* k_pool, void* v_pool,
+                                      const void* q, void* out, float* lse, float softmax_scale, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
 /* Device status word.  The pages have no counterpart: this is the failure
  * detection of this library's kernels.  Kernels never trap; a failed
  * device-side check or a bounded wait that ran out records a non-zero code in
