@@ -118,7 +118,10 @@ sp_status pack_common(const sp_plan* plan, const void* d_table, const void* k_in
     L.kdense_in = k_in, L.vdense_in = v_in, L.kpool_out = k_out, L.vpool_out = v_out;
   }
   launch_pack(L, static_cast<cudaStream_t>(stream));
-  const cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && !inverse && plan->hdr.n_spare > 0)  // the spare pool starts zero-filled
+    e = launch_zero_pages(section<int32_t>(d_table, plan->hdr.off_free) + kFreeIdsOffset, plan->hdr.n_spare,
+                          plan->sizes.page_bytes, k_out, v_out, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SP_OK : cuda_fail(e, inverse ? "segpaged_gather launch" : "build_segpaged_cache launch");
 }
 
@@ -172,6 +175,8 @@ sp_status build_segpaged_cache_layers(int32_t n_layers, const sp_plan* const* pl
     if (p->prob.dtype != p0->prob.dtype || p->prob.head_dim != p0->prob.head_dim ||
         p->prob.page_size != p0->prob.page_size || p->fp8 != p0->fp8)
       return fail(SP_ERR_INVALID_ARG, "every layer needs the same dtype, head_dim, page_size and page type");
+    if (p->hdr.n_spare > 0)
+      return fail(SP_ERR_UNSUPPORTED, "plans with a spare pool are packed by build_segpaged_cache");
     if (!k_dense[i] || !v_dense[i] || !aligned(k_dense[i], 16) || !aligned(v_dense[i], 16))
       return fail(SP_ERR_INVALID_ARG, "dense K/V pointers must be non-NULL and 16-byte aligned");
     la.page_begin[i] = int32_t(total);
@@ -265,6 +270,7 @@ sp_status segpaged_decode_append(const sp_plan* plan, void* d_table, const void*
   L.pool_pages = plan->sizes.pool_pages;
   L.k_new = k_new, L.v_new = v_new, L.kpool = k_pool, L.vpool = v_pool;
   L.status = static_cast<int32_t*>(workspace);
+  L.free_pool = const_cast<int32_t*>(section<int32_t>(d_table, plan->hdr.off_free));
   const cudaError_t e = launch_append(L, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SP_OK : cuda_fail(e, "segpaged_decode_append launch");
 }
@@ -299,6 +305,7 @@ sp_status segpaged_decode_step(const sp_plan* plan, void* d_table, const void* k
   L.k_new = k_new, L.v_new = v_new;
   L.new_stride_seq = stride_seq, L.new_stride_head = stride_head;
   L.k_inv = 1.0f / plan->k_scale, L.v_inv = 1.0f / plan->v_scale;
+  L.free_pool = const_cast<int32_t*>(section<int32_t>(d_table, plan->hdr.off_free));
   const cudaError_t e = launch_decode(L, s);
   return e == cudaSuccess ? SP_OK : cuda_fail(e, "segpaged_decode_step launch");
 }

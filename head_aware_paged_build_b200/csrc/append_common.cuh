@@ -42,6 +42,28 @@ __device__ __forceinline__ void append_eviction(const HeadDesc& hd, int& vp, int
   vp = nsink + re / P, slot = re % P;
 }
 
+// The physical page of the target record, taken from the ring plan's shared
+// spare pool when the record has none yet (a GLOBAL head growing into a page
+// it reserved as a record only).  Returns kNoPage, and records device code 7,
+// when the pool is empty.  The pool only hands pages out during a table's
+// life (segpaged_table_write refills it), so one atomic decrement per page is
+// enough.  One thread.
+__device__ __forceinline__ int32_t append_take_page(PageDesc* pg, int32_t* free_pool, int32_t* status) {
+  int32_t phys = pg->phys;
+  if (phys != kNoPage) return phys;
+  if (free_pool) {
+    const int32_t idx = atomicSub(free_pool, 1) - 1;
+    if (idx >= 0) {
+      phys = free_pool[kFreeIdsOffset + idx];
+      pg->phys = phys;
+      return phys;
+    }
+    atomicAdd(free_pool, 1);
+  }
+  record_error(status, kDevPoolEmpty);
+  return kNoPage;
+}
+
 // The target page's new valid range (one thread).
 __device__ __forceinline__ void append_update_target(PageDesc* pg, int L, int slot) {
   int lo = slot_lo(*pg);

@@ -27,6 +27,9 @@ struct PackLaunch {
   void* vdense_out;
 };
 void launch_pack(const PackLaunch& L, cudaStream_t s);
+// Zero-fill the pages ids[0 .. n) of both pools (a ring plan's spare pool, at build).
+cudaError_t launch_zero_pages(const int32_t* ids, int32_t n, int64_t page_bytes, void* kpool, void* vpool,
+                              cudaStream_t s);
 
 // Pack of several layers in one launch (kernel parameter, passed by value).
 constexpr int kMaxPackLayers = 128;
@@ -73,6 +76,7 @@ struct DecodeLaunch {
   const void* v_new;
   int64_t new_stride_seq, new_stride_head;
   float k_inv, v_inv;  // E4M3 pages: 1 / k_scale, 1 / v_scale
+  int32_t* free_pool;  // table's spare pool section (count, then ids)
 };
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t s);
 
@@ -122,6 +126,7 @@ struct AppendLaunch {
   void* kpool;
   void* vpool;
   int32_t* status;
+  int32_t* free_pool;  // table's spare pool section (count, then ids)
 };
 cudaError_t launch_append(const AppendLaunch& a, cudaStream_t s);
 

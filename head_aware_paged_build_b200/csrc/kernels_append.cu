@@ -26,7 +26,11 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendLaunch a) 
     return;
   }
   PageDesc* pg = a.pages + h.vpage_begin + vp;
-  const int64_t phys = pg->phys;
+  __shared__ int32_t s_phys;
+  if (threadIdx.x == 0) s_phys = append_take_page(pg, a.free_pool, a.status);
+  __syncthreads();
+  const int64_t phys = s_phys;
+  if (phys == kNoPage) return;  // the spare pool is empty: the append is skipped (reported)
   if (phys < 0 || phys >= a.pool_pages) {  // corrupted table: report, write nothing
     if (threadIdx.x == 0) record_error(a.status, kDevBadPage);
     return;

@@ -193,10 +193,18 @@ __device__ __forceinline__ void append_prologue(const DecodeLaunch& a, int ib, i
     append_target<P>(hd, vp, slot);
     if (vp >= hd.n_vpages) continue;  // no room: the head's finisher reports it
     PageDesc* pg = pages + hd.vpage_begin + vp;
-    const int64_t phys = pg->phys;
-    if (phys < 0 || phys >= a.pool_pages) continue;  // corrupted table: the producer reports the page
     const int g = hd.vpage_begin + vp;
-    if (g >= item.vp_begin && g < item.vp_end) {
+    const bool owner = g >= item.vp_begin && g < item.vp_end;
+    int64_t phys = pg->phys;
+    if (owner && phys == kNoPage) {  // a GLOBAL head's reserved record: take a page from the spare pool
+      int32_t taken = 0;
+      if (lane == 0) taken = append_take_page(pg, a.free_pool, a.status);
+      phys = __shfl_sync(0xffffffffu, taken, 0);
+      if (phys == kNoPage) continue;  // pool empty: the append is skipped (reported)
+    }
+    // only LOCAL heads evict, and their target pages always have a page
+    if (phys < 0 || phys >= a.pool_pages) continue;  // corrupted table: the producer reports the page
+    if (owner) {
       const __nv_bfloat16* kn = static_cast<const __nv_bfloat16*>(a.k_new) + int64_t(hd.b) * a.new_stride_seq +
                                 int64_t(hd.kv) * a.new_stride_head;
       const __nv_bfloat16* vn = static_cast<const __nv_bfloat16*>(a.v_new) + int64_t(hd.b) * a.new_stride_seq +
@@ -215,7 +223,7 @@ __device__ __forceinline__ void append_prologue(const DecodeLaunch& a, int ib, i
     __syncwarp();
   }
   fence_proxy_async_global();  // the token's bytes before this warp's bulk copies of its page
-  __threadfence_block();
+  __threadfence();             // page records taken from the pool, before the head's finisher reads them
   __syncwarp();
 }
 
@@ -280,8 +288,8 @@ __device__ __forceinline__ void decode_mma_body(const DecodeLaunch& a) {
             record_error(a.status, kDevTimeoutEmpty);
             good = 0;
           } else {
-            if (pgd.phys < 0 || pgd.phys >= a.pool_pages) {  // corrupted table: report, read nothing
-              record_error(a.status, kDevBadPage);
+            if (slot_hi(pgd) > slot_lo(pgd) && (pgd.phys < 0 || pgd.phys >= a.pool_pages)) {
+              record_error(a.status, kDevBadPage);  // corrupted table: report, read nothing
               pgd.span = 0;
             }
             sdesc[s] = pgd;
@@ -675,6 +683,7 @@ __global__ void __launch_bounds__(kF32Threads) decode_f32_kernel(DecodeLaunch a)
     for (int j = 0; j < ACC; ++j) acc[j] = 0.f;
     for (int g = item.vp_begin; g < item.vp_end; ++g) {
       const PageDesc pg = a.pages[g];
+      if (slot_hi(pg) <= slot_lo(pg)) continue;  // no token (a ring page or a reserved record)
       if (pg.phys < 0 || pg.phys >= a.pool_pages) {  // corrupted table: report, read nothing
         if (threadIdx.x == 0) record_error(a.status, kDevBadPage);
         continue;

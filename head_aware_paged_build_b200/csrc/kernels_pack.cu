@@ -58,6 +58,7 @@ __device__ __forceinline__ void pack_page(const PackArgs& a, int page, const T* 
   __shared__ uint32_t stage[P * PW];
 
   const PageDesc pg = a.pages[page];
+  if (pg.phys < 0) return;  // a record waiting for a page from the spare pool holds nothing
   const HeadDesc hd = a.heads[pg.head];
   const int64_t base = (a.stride_seq >= 0 ? int64_t(hd.b) * a.stride_seq : int64_t(hd.ctx_row0) * a.stride_tok) +
                        int64_t(hd.kv) * a.stride_head;
@@ -106,6 +107,7 @@ __global__ void __launch_bounds__(kPackThreads) gather_kernel(PackArgs a, const 
   __shared__ uint32_t stage[P * PW];
 
   const PageDesc pg = a.pages[blockIdx.x];
+  if (pg.phys < 0) return;  // a record waiting for a page from the spare pool holds nothing
   const HeadDesc hd = a.heads[pg.head];
   const int64_t base = (a.stride_seq >= 0 ? int64_t(hd.b) * a.stride_seq : int64_t(hd.ctx_row0) * a.stride_tok) +
                        int64_t(hd.kv) * a.stride_head;
@@ -156,6 +158,7 @@ __device__ __forceinline__ void pack_fp8_page(const PackArgs& a, int page, float
   constexpr int PW = vstage_pitch_words<__nv_bfloat16>(D);  // staging pitch (32-bit words)
   __shared__ uint32_t stage[P * PW];
   const PageDesc pg = a.pages[page];
+  if (pg.phys < 0) return;  // a record waiting for a page from the spare pool holds nothing
   const HeadDesc hd = a.heads[pg.head];
   const int64_t base = (a.stride_seq >= 0 ? int64_t(hd.b) * a.stride_seq : int64_t(hd.ctx_row0) * a.stride_tok) +
                        int64_t(hd.kv) * a.stride_head;
@@ -227,6 +230,7 @@ __global__ void __launch_bounds__(kPackThreads) gather_fp8_kernel(PackArgs a, co
   constexpr int SP = P + 4;  // staging pitch (bytes) of the V codes [D][tokens]
   __shared__ uint8_t stage[D * SP];
   const PageDesc pg = a.pages[blockIdx.x];
+  if (pg.phys < 0) return;  // a record waiting for a page from the spare pool holds nothing
   const HeadDesc hd = a.heads[pg.head];
   const int64_t base = (a.stride_seq >= 0 ? int64_t(hd.b) * a.stride_seq : int64_t(hd.ctx_row0) * a.stride_tok) +
                        int64_t(hd.kv) * a.stride_head;
@@ -283,7 +287,29 @@ void launch_pack_t(const PackLaunch& L, cudaStream_t s) {
                                                             static_cast<uint8_t*>(L.vpool_out));
 }
 
+// Zero one page of each pool per block: the spare pool's pages, so that an
+// append that takes one leaves only finite values in the slots it masks out.
+__global__ void __launch_bounds__(kPackThreads) zero_pages_kernel(const int32_t* __restrict__ ids,
+                                                                  int64_t page_bytes, uint8_t* __restrict__ kpool,
+                                                                  uint8_t* __restrict__ vpool) {
+  const int64_t phys = ids[blockIdx.x];
+  uint4* k = reinterpret_cast<uint4*>(kpool + phys * page_bytes);
+  uint4* v = reinterpret_cast<uint4*>(vpool + phys * page_bytes);
+  for (int64_t i = threadIdx.x; i < page_bytes / 16; i += kPackThreads) {
+    k[i] = make_uint4(0, 0, 0, 0);
+    v[i] = make_uint4(0, 0, 0, 0);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_zero_pages(const int32_t* ids, int32_t n, int64_t page_bytes, void* kpool, void* vpool,
+                              cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  zero_pages_kernel<<<n, kPackThreads, 0, s>>>(ids, page_bytes, static_cast<uint8_t*>(kpool),
+                                               static_cast<uint8_t*>(vpool));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pack_layers(const PackLayersArgs& la, bool bf16, bool fp8, int D, int P, void* kpool, void* vpool,
                                cudaStream_t s) {

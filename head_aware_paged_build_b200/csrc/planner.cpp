@@ -43,6 +43,9 @@ sp_status validate(const sp_problem& p) {
   if (p.append_capacity < 0) return fail(SP_ERR_INVALID_ARG, "append_capacity must be >= 0");
   if (p.append_capacity > 0 && !(p.flags & SP_FLAG_RING))
     return fail(SP_ERR_INVALID_ARG, "append_capacity needs SP_FLAG_RING");
+  if (p.spare_pages < 0) return fail(SP_ERR_INVALID_ARG, "spare_pages must be >= 0");
+  if (p.spare_pages > 0 && !(p.flags & SP_FLAG_RING))
+    return fail(SP_ERR_INVALID_ARG, "spare_pages needs SP_FLAG_RING");
   if ((p.flags & SP_FLAG_RING) && (p.flags & SP_FLAG_DENSE_MASKED))
     return fail(SP_ERR_UNSUPPORTED, "ring plans are SegPaged plans (no dense-masked variant)");
   if (p.first_page < 0) return fail(SP_ERR_INVALID_ARG, "first_page must be >= 0");
@@ -310,7 +313,11 @@ sp_status plan_build(sp_plan& pl) {
         };
         if (!local) {
           const int64_t np = ceil_div(L + cap, P);
-          for (int64_t k = 0; k < np; ++k) add_page(k * P, 0, std::clamp<int64_t>(L - k * P, 0, P));
+          for (int64_t k = 0; k < np; ++k) {
+            add_page(k * P, 0, std::clamp<int64_t>(L - k * P, 0, P));
+            // with a shared spare pool, pages reserved for growth are records only
+            if (p.spare_pages > 0 && k * P >= L) pl.pages.back().phys = kNoPage;
+          }
           pl.segments.push_back(sp_segment{0, int32_t(L), 0, int32_t(np)});
         } else {
           const int64_t nsink = ceil_div(s, P);
@@ -373,20 +380,32 @@ sp_status plan_build(sp_plan& pl) {
   visible *= pl.group;
 
   // --- physical page ids -----------------------------------------------------
-  int64_t max_id = n_pages - 1;
+  // The plan owns one page per page record with a page, then the spare pool;
+  // logical page k (records in order, then the pool) is physical page
+  // first_page + (page_ids ? page_ids[k] : k).
+  int64_t n_assigned = 0;
+  for (const PageDesc& pd : pl.pages) n_assigned += pd.phys != kNoPage;
+  const int64_t n_owned = n_assigned + p.spare_pages;
+  if (n_owned > std::numeric_limits<int32_t>::max()) return fail(SP_ERR_UNSUPPORTED, "more than 2^31 pages");
+  int64_t max_id = n_owned - 1;
   if (p.page_ids) {
-    std::vector<int32_t> ids(p.page_ids, p.page_ids + n_pages);
+    std::vector<int32_t> ids(p.page_ids, p.page_ids + n_owned);
     for (int32_t id : ids)
       if (id < 0) return fail(SP_ERR_INVALID_ARG, "page_ids must be non-negative");
     std::sort(ids.begin(), ids.end());
     if (std::adjacent_find(ids.begin(), ids.end()) != ids.end())
       return fail(SP_ERR_INVALID_ARG, "page_ids must be distinct");
-    max_id = n_pages ? ids.back() : -1;
+    max_id = n_owned ? ids.back() : -1;
   }
   if (p.first_page + max_id + 1 > std::numeric_limits<int32_t>::max())
     return fail(SP_ERR_UNSUPPORTED, "pool above 2^31 pages");
+  auto phys_of = [&](int64_t k) { return int32_t(p.first_page + (p.page_ids ? p.page_ids[k] : k)); };
+  int64_t logical = 0;
   for (int64_t i = 0; i < n_pages; ++i)
-    pl.pages[i].phys = int32_t(p.first_page + (p.page_ids ? p.page_ids[i] : i));
+    if (pl.pages[i].phys != kNoPage) pl.pages[i].phys = phys_of(logical++);
+  std::vector<int32_t> free_stack(kFreeIdsOffset + p.spare_pages, 0);
+  free_stack[0] = p.spare_pages;
+  for (int64_t k = 0; k < p.spare_pages; ++k) free_stack[kFreeIdsOffset + k] = phys_of(n_assigned + k);
 
   // --- decode: balanced page ranges per CTA, cut at head boundaries ---------
   int n_slots = 0;
@@ -555,12 +574,14 @@ sp_status plan_build(sp_plan& pl) {
   H.off_decode_cta = append(pl.blob, pl.decode_cta_begin);
   H.off_combine = append(pl.blob, pl.combine);
   H.off_prefill = append(pl.blob, pl.prefill);
+  H.off_free = append(pl.blob, free_stack);
+  H.n_spare = p.spare_pages;
   align_to(pl.blob, 256);
   std::memcpy(pl.blob.data(), &H, sizeof(H));
 
   sp_sizes& z = pl.sizes;
   z = sp_sizes{};
-  z.num_pages = n_pages;
+  z.num_pages = n_owned;
   z.pool_pages = p.first_page + max_id + 1;
   z.page_bytes = int64_t(P) * D * (pl.fp8 ? 1 : pl.elem_bytes);
   z.table_bytes = int64_t(pl.blob.size());

@@ -18,7 +18,8 @@ namespace sp {
 
 constexpr int32_t kTableMagic = 0x53504731;  // "SPG1"
 constexpr int kStatusBytes = 256;            // workspace prefix holding the status word
-constexpr int kPrefillTileTokensBf16 = 128;  // KV / query tile of the tcgen05 prefill kernel
+constexpr int kPrefillTileTokensBf16 = 128;  // query tile of the tcgen05 prefill kernel
+constexpr int kPrefillKvTileBf16 = 64;       // KV tokens (one page) per step of the tcgen05 prefill kernel
 constexpr int kPrefillTileTokensF32 = 64;    // KV / query tile of the fp32 prefill kernel
 constexpr int kMaxGroup = 16;                // q-heads per kv-head handled by one decode CTA
 
@@ -35,7 +36,15 @@ enum DeviceCode : int32_t {
   kDevTimeoutSoftmax = 4,  // the MMA issuer gave up waiting for P
   kDevBadPage = 5,         // a table page id outside [0, pool_pages): nothing read or written there
   kDevAppendFull = 6,      // an append found no reserved page left (ring plans)
+  kDevPoolEmpty = 7,       // an append found the shared spare pool empty (ring plans with spare pages)
 };
+
+// Shared spare pool of a ring plan (table section): word 0 holds how many of
+// the page ids at words kFreeIdsOffset ... are still free; appends take the
+// last free one with an atomic decrement.  A page record waiting for a page
+// from the pool has phys == kNoPage.
+constexpr int kFreeIdsOffset = 4;
+constexpr int32_t kNoPage = -1;
 
 // One (sequence, kv-head).  Kinds are resolved: 0 reads the whole causal
 // context, 1 applies the local rule (sink + window) to every page that is not
@@ -131,6 +140,9 @@ struct alignas(16) TableHeader {
   int32_t n_combine;
   int32_t n_prefill_items;
   int64_t off_heads, off_pages, off_decode_items, off_decode_cta, off_combine, off_prefill;
+  int64_t off_free;  // spare pool section (count, then page ids)
+  int32_t n_spare;
+  int32_t pad;
 };
 
 }  // namespace sp

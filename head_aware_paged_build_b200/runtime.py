@@ -36,14 +36,14 @@ class SegPagedLayer:
                  page_ids: Sequence[int] | None = None, first_page: int = 0, target_ctas: int = 0,
                  append_capacity: int = 0, pools: tuple[torch.Tensor, torch.Tensor] | None = None,
                  kv_dtype: str | None = None, k_scale: float = 1.0, v_scale: float = 1.0,
-                 block_mass: Sequence | None = None):
+                 block_mass: Sequence | None = None, spare_pages: int = 0):
         self.dtype = dtype
         self.torch_dtype = {"f32": torch.float32, "bf16": torch.bfloat16}[dtype]
         self.num_q_heads, self.num_kv_heads, self.head_dim = num_q_heads, num_kv_heads, head_dim
         self.device = torch.device(device)
         self.problem = S.make_problem(batch, num_q_heads, num_kv_heads, head_dim, page_size, dtype, ctx_len,
                                       q_start, policy, first_page, page_ids, target_ctas, flags, append_capacity,
-                                      kv_dtype, k_scale, v_scale, block_mass)
+                                      kv_dtype, k_scale, v_scale, block_mass, spare_pages)
         self.kv_dtype = kv_dtype or dtype
         self.batch = batch
         self.ctx_len = [int(x) for x in ctx_len]

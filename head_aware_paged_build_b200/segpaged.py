@@ -56,7 +56,7 @@ class sp_problem(ctypes.Structure):
                 ("page_ids", ctypes.POINTER(ctypes.c_int32)), ("target_ctas", ctypes.c_int32),
                 ("flags", ctypes.c_uint32), ("append_capacity", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
                 ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
-                ("block_mass", ctypes.POINTER(ctypes.POINTER(ctypes.c_float)))]
+                ("block_mass", ctypes.POINTER(ctypes.POINTER(ctypes.c_float))), ("spare_pages", ctypes.c_int32)]
 
 
 class sp_sizes(ctypes.Structure):
@@ -148,7 +148,8 @@ def make_problem(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
                  ctx_len: Sequence[int], q_start: Sequence[int], policy: Sequence[tuple],
                  first_page: int = 0, page_ids: Sequence[int] | None = None, target_ctas: int = 0,
                  flags: int = 0, append_capacity: int = 0, kv_dtype: str | int | None = None,
-                 k_scale: float = 1.0, v_scale: float = 1.0, block_mass: Sequence | None = None):
+                 k_scale: float = 1.0, v_scale: float = 1.0, block_mass: Sequence | None = None,
+                 spare_pages: int = 0):
     """Build an ``sp_problem`` plus the host arrays it points to (kept alive in the result).
 
     ``policy`` entries are ``(kind, sink, window)`` or, for retrieval heads,
@@ -183,7 +184,7 @@ def make_problem(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
                       0 if kv_dtype is None else (DTYPE_CODES[kv_dtype] if isinstance(kv_dtype, str) else kv_dtype),
                       k_scale, v_scale,
                       ctypes.cast(mass_ptrs, ctypes.POINTER(ctypes.POINTER(ctypes.c_float)))
-                      if mass_ptrs is not None else None)
+                      if mass_ptrs is not None else None, spare_pages)
     prob._keep = (ctx, q0, pol, ids, masses, mass_ptrs)
     return prob
 

@@ -145,6 +145,15 @@ typedef struct {
  *               (i + 1) * page_size); other entries are ignored.  Copied (as
  *               the kept-block choice) by segpaged_plan_create.  Retrieval
  *               heads are not supported in ring plans (SP_ERR_UNSUPPORTED).
+ *   spare_pages SP_FLAG_RING plans: a pool of this many pages shared by the
+ *               plan's GLOBAL heads ("RedKnot overview (aipuzi)", §3.2: per-head
+ *               pools that hand out pages as heads grow).  With spare_pages > 0
+ *               the pages a GLOBAL head reserves for append_capacity are page
+ *               records only, with no physical page: an append that reaches
+ *               such a record takes a page from the shared pool, so the pool is
+ *               sized for the growth of all heads together rather than each
+ *               head's worst case.  build_segpaged_cache zero-fills the spare
+ *               pages.  0 keeps one physical page per reserved record.
  */
 typedef struct {
   int32_t batch;
@@ -164,10 +173,11 @@ typedef struct {
   int32_t kv_dtype;        /* page type: 0 = dtype, or SP_E4M3 (bf16 decode plans) */
   float k_scale, v_scale;  /* SP_E4M3 pages: stored code = E4M3(x * (1 / scale)) */
   const float* const* block_mass; /* SP_RETRIEVAL heads: importance per page-size block */
+  int32_t spare_pages;            /* ring plans: size of the shared spare pool (0: none) */
 } sp_problem;
 
 typedef struct {
-  int64_t num_pages;          /* pages the plan owns in each of the K and V pools */
+  int64_t num_pages;          /* pages the plan owns in each of the K and V pools (spare pool included) */
   int64_t pool_pages;         /* pages each pool must hold: first_page + max id + 1 */
   int64_t page_bytes;         /* bytes of one page = page_size * head_dim * element size */
   int64_t table_bytes;        /* size of the device table blob */
@@ -428,6 +438,7 @@ SP_API sp_status segpaged_decode_step(const sp_plan* plan, void* d_table, const 
  *   5     a page id in the device table lies outside [0, pool_pages): the
  *         kernel read or wrote nothing there (a corrupted table)
  *   6     a ring append found no reserved page left (the append was skipped)
+ *   7     a ring append found the shared spare pool empty (the append was skipped)
  * read synchronises `stream`, copies the word to *code (host) and returns
  * SP_OK for 0, SP_ERR_DEVICE_CHECK for a recorded code (SP_ERR_CUDA if the
  * synchronisation or the copy fails); clear zeroes the word's 256-byte block

@@ -322,3 +322,43 @@ def test_multi_layer_build_checks_before_launch():
     assert "same dtype" in S.last_error()
     S.segpaged_plan_destroy(a)
     S.segpaged_plan_destroy(b)
+
+
+def test_ring_plan_spare_pool_ids_and_checks():
+    """With a shared spare pool, a GLOBAL head's reserved records have no page (-1) and the plan owns
+    its assigned pages plus the pool; page_ids permute both; the pool needs a ring plan."""
+    L0 = (70, 200, 5)
+    pol = [("local", 4, 40), ("global", 0, 0)] * 3
+    base = S.make_problem(3, 4, 2, 128, 64, "bf16", L0, [L - 1 for L in L0], pol, flags=S.SP_FLAG_RING,
+                          append_capacity=150)
+    plan = S.segpaged_plan_create(base)
+    z0 = S.segpaged_plan_sizes(plan)
+    full = [S.segpaged_plan_head_pages(plan, b, 1) for b in range(3)]
+    S.segpaged_plan_destroy(plan)
+    spare = 3
+    p = S.make_problem(3, 4, 2, 128, 64, "bf16", L0, [L - 1 for L in L0], pol, flags=S.SP_FLAG_RING,
+                       append_capacity=150, spare_pages=spare)
+    plan = S.segpaged_plan_create(p)
+    z = S.segpaged_plan_sizes(plan)
+    heads = [S.segpaged_plan_head_pages(plan, b, 1) for b in range(3)]
+    local = [S.segpaged_plan_head_pages(plan, b, 0) for b in range(3)]
+    S.segpaged_plan_destroy(plan)
+    for L, ids, ids_full in zip(L0, heads, full):
+        held = -(-L // 64)
+        assert len(ids) == len(ids_full) and all(i >= 0 for i in ids[:held]) and all(i == -1 for i in ids[held:])
+    reserved = sum(len(f) - -(-L // 64) for L, f in zip(L0, full))
+    assert z.num_pages == z0.num_pages - reserved + spare == z.pool_pages
+    owned = sorted(i for ids in heads + local for i in ids if i >= 0)
+    assert owned == list(range(z.num_pages - spare))  # records first, the pool's pages after them
+    perm = list(np.random.default_rng(4).permutation(z.num_pages) + 2)
+    p2 = S.make_problem(3, 4, 2, 128, 64, "bf16", L0, [L - 1 for L in L0], pol, flags=S.SP_FLAG_RING,
+                        append_capacity=150, spare_pages=spare, page_ids=perm)
+    plan = S.segpaged_plan_create(p2)
+    got = sorted(i for b in range(3) for kv in range(2) for i in S.segpaged_plan_head_pages(plan, b, kv) if i >= 0)
+    assert got == sorted(perm[:z.num_pages - spare]) and S.segpaged_plan_sizes(plan).pool_pages == max(perm) + 1
+    S.segpaged_plan_destroy(plan)
+    for bad, code in ((dict(spare_pages=-1, flags=S.SP_FLAG_RING), S.SP_ERR_INVALID_ARG),
+                      (dict(spare_pages=2), S.SP_ERR_INVALID_ARG)):
+        q = S.make_problem(3, 4, 2, 128, 64, "bf16", L0, [L - 1 for L in L0], pol, **bad)
+        st, pl = S.segpaged_plan_create_status(q)
+        assert st == code and not pl
