@@ -222,21 +222,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D);
       const uint32_t q_addr = smem_u32(q_s), st_addr = smem_u32(stage_s);
       auto issue_s = [&](int x, int st) {
-        const uint32_t qa = q_addr + x * Sm::kQ, ka = st_addr + st * Sm::kStage;
+        // a descriptor's start-address field is address >> 4, so each k-step's
+        // descriptor is the tile's base descriptor plus a fixed offset
+        const uint64_t qd = tc::smem_desc_sw128(q_addr + x * Sm::kQ);
+        const uint64_t kd = tc::smem_desc_sw128(st_addr + st * Sm::kStage);
+        const uint32_t ts = t_s(x);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc::mma_bf16_ss(t_s(x), tc::smem_desc_sw128(qa + off), tc::smem_desc_sw128(ka + off), idesc_s, kk > 0);
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          tc::mma_bf16_ss(ts, qd + off, kd + off, idesc_s, kk > 0);
         }
         tc::commit(&bars->s_full[x]);
       };
       auto issue_pv = [&](int x, int st, bool acc) {
-        const uint32_t va = st_addr + st * Sm::kStage + Sm::kK;
+        const uint64_t vd = tc::smem_desc_sw128(st_addr + st * Sm::kStage + Sm::kK);
+        const uint32_t to = t_o(x), ts = t_s(x);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)  // P of page h sits at columns [64 h, 64 h + 32)
-          tc::mma_bf16_ts(t_o(x), t_s(x) + (kk >> 2) * 64 + (kk & 3) * 8,
-                          tc::smem_desc_sw128(va + (kk >> 2) * (D * 128) + (kk & 3) * 32), idesc_o,
-                          (acc || kk > 0) ? 1u : 0u);
+          tc::mma_bf16_ts(to, ts + (kk >> 2) * 64 + (kk & 3) * 8, vd + (((kk >> 2) * (D * 128) + (kk & 3) * 32) >> 4),
+                          idesc_o, (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(&bars->q, 0) && mbar_wait(&kv_full[0], 0);
       if (!ok) fail(kDevTimeoutFull);

@@ -19,7 +19,6 @@ namespace sp {
 constexpr int32_t kTableMagic = 0x53504731;  // "SPG1"
 constexpr int kStatusBytes = 256;            // workspace prefix holding the status word
 constexpr int kPrefillTileTokensBf16 = 128;  // query tile of the tcgen05 prefill kernel
-constexpr int kPrefillKvTileBf16 = 64;       // KV tokens (one page) per step of the tcgen05 prefill kernel
 constexpr int kPrefillTileTokensF32 = 64;    // KV / query tile of the fp32 prefill kernel
 constexpr int kMaxGroup = 16;                // q-heads per kv-head handled by one decode CTA
 
