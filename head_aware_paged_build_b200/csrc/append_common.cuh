@@ -86,9 +86,11 @@ __device__ __forceinline__ void append_update_eviction(PageDesc* pe, int pos, in
 // t = first, first + stride, ... of the caller cooperate).  bf16 pages use the
 // swizzled operand layouts, fp32 pages row-major K and transposed V, E4M3
 // pages the codes of the bf16 values times 1 / scale (nearest even,
-// saturating), as the pack writes them.
+// saturating), as the pack writes them.  The new row never overlaps the page,
+// so the loads need not wait for the stores.
 template <typename T, int D, int P, bool FP8>
-__device__ __forceinline__ void append_write_token(const T* kn, const T* vn, uint8_t* kdst, uint8_t* vdst, int slot,
+__device__ __forceinline__ void append_write_token(const T* __restrict__ kn, const T* __restrict__ vn,
+                                                   uint8_t* __restrict__ kdst, uint8_t* __restrict__ vdst, int slot,
                                                    float k_inv, float v_inv, int first, int stride) {
   constexpr int CR = D * int(sizeof(T)) / 16;
   if constexpr (FP8) {

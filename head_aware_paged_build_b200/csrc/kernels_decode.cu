@@ -48,7 +48,8 @@ struct DecodeSmem {
   static constexpr int kMlOff = kMergeOff + kConsumerWarps * kMaxGroup * kMergePitch * 4;
   static constexpr int kBarOff = kMlOff + kConsumerWarps * kMaxGroup * 2 * 4;
   static constexpr int kDescOff = kBarOff + 2 * NST * 8;  // PageDesc of each stage (16-byte aligned)
-  static constexpr int kBytes = kDescOff + NST * 16;
+  static constexpr int kPatchOff = kDescOff + NST * 16;  // fused step: slot of the stage's new token, or -1
+  static constexpr int kBytes = kPatchOff + ((NST * 4 + 15) / 16) * 16;
 };
 
 // Final merge of a split head, run by its last CTA over the n_slots partials
@@ -161,9 +162,10 @@ __device__ __forceinline__ void merge_split_head(const DecodeLaunch& a, const He
 // the final merge of a split head) advances the context, exactly as the
 // standalone append does after writing (or reports a ring without room).
 template <int P>
-__device__ __noinline__ void finish_append(const DecodeLaunch& a, int head) {
+__device__ __forceinline__ void finish_append(const DecodeLaunch& a, int head) {
   // re-read from the table (not kept in registers through the page loop); no
-  // thread writes this head's descriptor before this point of the launch
+  // thread writes this head's descriptor before this point of the launch.
+  // Inlined: an out-of-line call here cost ~9 us per launch on the 32K layer.
   const HeadDesc hd = a.heads[head];
   int vp, slot;
   append_target<P>(hd, vp, slot);
@@ -178,53 +180,36 @@ __device__ __noinline__ void finish_append(const DecodeLaunch& a, int head) {
   w->q_start = hd.ctx_len;
 }
 
-// Producer-warp prologue of the fused decode step: for each item of this CTA,
-// append the head's new token if its target page lies in the item's page range,
-// and evict the token that leaves the window if that token's page does.  The
-// writes are ordered before the warp's bulk copies of the same pages.
-template <int D, bool FP8>
-__device__ __forceinline__ void append_prologue(const DecodeLaunch& a, int ib, int ie, int lane) {
+// Fused decode step, producer side.  Lane i holds the append of item
+// `first + i` of this CTA: the head's target page (index in the table's page
+// list, or -1 when the head has no room left) and slot, and the page and slot
+// of the token that leaves a LOCAL head's window (-1: none).  The producer
+// meets each page of its items once, in order; at the target or eviction page
+// it applies the append's record changes to its copy of the record before it
+// publishes it, writes the record back, and marks the stage so that the warp
+// whose tokens hold the new slot writes the new token into the staged page
+// (and the pool page) itself: the page's bulk copy never waits for the append.
+struct AppendInfo {
+  int vend = 0;  // item's page range end
+  int tg = -1, slot = 0, len = 0;
+  int eg = -1, eslot = 0, epos = 0;
+};
+
+__device__ __forceinline__ AppendInfo append_info(const DecodeLaunch& a, int it, int ie) {
   constexpr int P = 64;
-  PageDesc* pages = const_cast<PageDesc*>(a.pages);
-  for (int it = ib; it < ie; ++it) {
-    const DecodeItem item = a.items[it];
-    const HeadDesc hd = a.heads[item.head];
-    int vp, slot;
-    append_target<P>(hd, vp, slot);
-    if (vp >= hd.n_vpages) continue;  // no room: the head's finisher reports it
-    PageDesc* pg = pages + hd.vpage_begin + vp;
-    const int g = hd.vpage_begin + vp;
-    const bool owner = g >= item.vp_begin && g < item.vp_end;
-    int64_t phys = pg->phys;
-    if (owner && phys == kNoPage) {  // a GLOBAL head's reserved record: take a page from the spare pool
-      int32_t taken = 0;
-      if (lane == 0) taken = append_take_page(pg, a.free_pool, a.status);
-      phys = __shfl_sync(0xffffffffu, taken, 0);
-      if (phys == kNoPage) continue;  // pool empty: the append is skipped (reported)
-    }
-    // only LOCAL heads evict, and their target pages always have a page
-    if (phys < 0 || phys >= a.pool_pages) continue;  // corrupted table: the producer reports the page
-    if (owner) {
-      const __nv_bfloat16* kn = static_cast<const __nv_bfloat16*>(a.k_new) + int64_t(hd.b) * a.new_stride_seq +
-                                int64_t(hd.kv) * a.new_stride_head;
-      const __nv_bfloat16* vn = static_cast<const __nv_bfloat16*>(a.v_new) + int64_t(hd.b) * a.new_stride_seq +
-                                int64_t(hd.kv) * a.new_stride_head;
-      append_write_token<__nv_bfloat16, D, P, FP8>(
-          kn, vn, static_cast<uint8_t*>(const_cast<void*>(a.kpool)) + phys * a.page_bytes,
-          static_cast<uint8_t*>(const_cast<void*>(a.vpool)) + phys * a.page_bytes, slot, a.k_inv, a.v_inv, lane, 32);
-      if (lane == 0) append_update_target(pg, hd.ctx_len, slot);
-    }
-    int evp, eslot, epos;
-    append_eviction<P>(hd, evp, eslot, epos);
-    if (evp >= 0 && lane == 0) {
-      const int ge = hd.vpage_begin + evp;
-      if (ge >= item.vp_begin && ge < item.vp_end) append_update_eviction(pages + ge, epos, eslot);
-    }
-    __syncwarp();
-  }
-  fence_proxy_async_global();  // the token's bytes before this warp's bulk copies of its page
-  __threadfence();             // page records taken from the pool, before the head's finisher reads them
-  __syncwarp();
+  AppendInfo r;
+  if (it >= ie) return r;
+  const DecodeItem item = a.items[it];
+  const HeadDesc hd = a.heads[item.head];
+  r.vend = item.vp_end;
+  int vp, slot;
+  append_target<P>(hd, vp, slot);
+  if (vp >= hd.n_vpages) return r;  // no room: nothing changes (the head's finisher reports it)
+  r.tg = hd.vpage_begin + vp, r.slot = slot, r.len = hd.ctx_len;
+  int evp, eslot, epos;
+  append_eviction<P>(hd, evp, eslot, epos);
+  if (evp >= 0) r.eg = hd.vpage_begin + evp, r.eslot = eslot, r.epos = epos;
+  return r;
 }
 
 template <int D, int NST, bool FP8, bool APPEND>
@@ -268,12 +253,18 @@ __device__ __forceinline__ void decode_mma_body(const DecodeLaunch& a) {
     // the stage's full barrier), start the copies.
     int k = 0;
     bool ok = true;
-    if constexpr (APPEND) append_prologue<D, FP8>(a, ib, ie, lane);
+    int32_t* spatch = reinterpret_cast<int32_t*>(smem + S::kPatchOff);
+    // page records this launch may change (fused append) are read through L2
+    auto records = [&](int base) {
+      const int4* r = reinterpret_cast<const int4*>(a.pages + base + lane);
+      return base + lane < ge ? (APPEND ? __ldcg(r) : __ldg(r)) : make_int4(0, 0, 0, 0);
+    };
+    int4 mine = records(gb);  // issued before the append bookkeeping's loads, so their latencies overlap
+    AppendInfo ai;
+    int ai_first = ib, cur = ib;  // lane i holds item ai_first + i; cur: the item of the current page
+    if constexpr (APPEND) ai = append_info(a, ib + lane, ie);
     for (int base = gb; base < ge && ok; base += 32) {
-      // page records this launch may have changed (fused append) are read through L2
-      const int4 mine = base + lane < ge ? (APPEND ? __ldcg(reinterpret_cast<const int4*>(a.pages + base + lane))
-                                                   : __ldg(reinterpret_cast<const int4*>(a.pages + base + lane)))
-                                         : make_int4(0, 0, 0, 0);
+      if (base != gb) mine = records(base);
       const int n = min(32, ge - base);
       for (int i = 0; i < n; ++i, ++k) {
         PageDesc pgd;
@@ -282,6 +273,36 @@ __device__ __forceinline__ void decode_mma_body(const DecodeLaunch& a) {
         pgd.span = __shfl_sync(0xffffffffu, mine.z, i);
         pgd.head = __shfl_sync(0xffffffffu, mine.w, i);
         const int s = k % NST;
+        int patch = -1;
+        if constexpr (APPEND) {
+          const int g = base + i;
+          while (g >= __shfl_sync(0xffffffffu, ai.vend, cur - ai_first)) {
+            if (++cur - ai_first == 32) ai_first = cur, ai = append_info(a, cur + lane, ie);
+          }
+          const int c = cur - ai_first;
+          const int tg = __shfl_sync(0xffffffffu, ai.tg, c), eg = __shfl_sync(0xffffffffu, ai.eg, c);
+          if (g == tg || g == eg) {
+            PageDesc* rec = const_cast<PageDesc*>(a.pages) + g;
+            if (g == tg) {
+              if (pgd.phys == kNoPage) {  // a GLOBAL head's reserved record: take a page from the spare pool
+                int32_t taken = 0;
+                if (lane == 0) {
+                  taken = append_take_page(rec, a.free_pool, a.status);
+                  __threadfence();  // the record's page before the head's finisher reads it
+                }
+                pgd.phys = __shfl_sync(0xffffffffu, taken, 0);
+              }
+              if (pgd.phys >= 0 && pgd.phys < a.pool_pages) {  // else: pool empty (reported) or a corrupted table
+                patch = __shfl_sync(0xffffffffu, ai.slot, c);
+                append_update_target(&pgd, __shfl_sync(0xffffffffu, ai.len, c), patch);
+              }
+            }
+            if (g == eg)
+              append_update_eviction(&pgd, __shfl_sync(0xffffffffu, ai.epos, c),
+                                     __shfl_sync(0xffffffffu, ai.eslot, c));
+            if (lane == 0) *rec = pgd;
+          }
+        }
         int good = 1;
         if (lane == 0) {
           if (k >= NST && !mbar_wait(&empty[s], ((k / NST) & 1) ^ 1)) {
@@ -293,6 +314,7 @@ __device__ __forceinline__ void decode_mma_body(const DecodeLaunch& a) {
               pgd.span = 0;
             }
             sdesc[s] = pgd;
+            if constexpr (APPEND) spatch[s] = patch;
             uint8_t* kd = stage + s * 2 * PB;
             if (slot_hi(pgd) > slot_lo(pgd)) {
               mbar_arrive_expect_tx(&full[s], 2 * PB);
@@ -370,6 +392,26 @@ __device__ __forceinline__ void decode_mma_body(const DecodeLaunch& a) {
       const PageDesc pg = sdesc[s];
       const int tok0 = warp * 16;
       const int lo = slot_lo(pg), hi = slot_hi(pg);
+      if constexpr (APPEND) {
+        const int patch = reinterpret_cast<const int32_t*>(smem + S::kPatchOff)[s];
+        if (ok && patch >= tok0 && patch < tok0 + 16) {
+          // this warp's tokens hold the new one: write it into the staged page
+          // (the bytes the page will hold) and into the pool page
+          const __nv_bfloat16* kn = static_cast<const __nv_bfloat16*>(a.k_new) + int64_t(hd.b) * a.new_stride_seq +
+                                    int64_t(hd.kv) * a.new_stride_head;
+          const __nv_bfloat16* vn = static_cast<const __nv_bfloat16*>(a.v_new) + int64_t(hd.b) * a.new_stride_seq +
+                                    int64_t(hd.kv) * a.new_stride_head;
+          uint8_t* ks = stage + s * 2 * PB;
+          append_write_token<__nv_bfloat16, D, P, FP8>(kn, vn, ks, ks + PB, patch, a.k_inv, a.v_inv, lane, 32);
+          append_write_token<__nv_bfloat16, D, P, FP8>(
+              kn, vn, static_cast<uint8_t*>(const_cast<void*>(a.kpool)) + int64_t(pg.phys) * a.page_bytes,
+              static_cast<uint8_t*>(const_cast<void*>(a.vpool)) + int64_t(pg.phys) * a.page_bytes, patch, a.k_inv,
+              a.v_inv, lane, 32);
+          // generic writes to the stage before the next bulk copy into it (async proxy)
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+        }
+      }
       if (ok && tok0 < hi && tok0 + 16 > lo) {
         const uint32_t kst = smem_u32(stage + s * 2 * PB);
         const uint32_t vst = kst + PB;
@@ -638,8 +680,8 @@ __device__ __forceinline__ void decode_mma_body(const DecodeLaunch& a) {
 }
 
 // The decode kernel, and the fused decode step (append + decode), which must
-// keep two CTAs on every SM: its prologue would otherwise raise the register
-// count past the 168 that two 5-warp CTAs leave each thread.
+// keep two CTAs on every SM: its append bookkeeping would otherwise raise the
+// register count past the 168 that two 5-warp CTAs leave each thread.
 template <int D, int NST, bool FP8>
 __global__ void __launch_bounds__(kDecodeThreads) decode_mma_kernel(DecodeLaunch a) {
   decode_mma_body<D, NST, FP8, false>(a);

@@ -412,11 +412,14 @@ SP_API sp_status segpaged_decode_append(const sp_plan* plan, void* d_table, cons
  * segpaged_decode_append followed by segpaged_attention on the same table,
  * with bit for bit the same outputs, pool and table ("SegPagedAttention
  * runtime design", §3: a LOCAL head's window moves without moving tokens; §5:
- * no layout work per call).  On bf16 and E4M3 pages it is one launch: each
- * decode CTA appends the new token of the heads whose target page lies in its
- * page range before streaming those pages, and evicts the token that leaves a
- * LOCAL window when that token's page is in its range; the CTA that finishes
- * a head advances its context length.  fp32 pages run the two calls.
+ * no layout work per call).  On bf16 and E4M3 pages it is one launch: the
+ * decode CTA whose page range holds a head's target page changes that page's
+ * record as it streams the page, and the warp whose tokens hold the new slot
+ * writes the new token into the staged copy of the page and into the pool
+ * page, so no page copy waits for the append; the CTA whose range holds the
+ * page of the token that leaves a LOCAL window changes that record the same
+ * way; the CTA that finishes a head advances its context length.  fp32 pages
+ * run the two calls.
  *   k_new, v_new, stride_seq, stride_head  as segpaged_decode_append
  *   q    device [batch, num_q_heads, head_dim]: the queries at the new
  *        positions (each sequence's current context length before the call)
