@@ -96,13 +96,14 @@ def test_decode_step_ring_without_room_reports_like_the_append():
 
 
 def test_decode_step_graph_fused_equals_unfused():
-    """The serving step captured in a CUDA graph, fused and unfused, on the 32K layer (batch 2)."""
-    wl = W.llama(batch=2)
+    """The serving step captured in a CUDA graph, fused and unfused, on the 32K layer at the bench's
+    batch of 8: outputs every step, and pools and tables at the end, bit for bit."""
+    wl = W.llama()
     n = 6
     dec = wl.decode_problem()
     start = W.Problem(wl, tuple(L - n for L in dec.ctx_lens), tuple(L - n - 1 for L in dec.ctx_lens))
     k, v = W.dense_kv(dec, device="cuda", gen_device="cuda")
-    steps = []
+    steps, layers = [], []
     for fused in (True, False):
         layer = layer_for(start, flags=S.SP_FLAG_RING, append_capacity=n)
         layer.build(k, v)
@@ -117,6 +118,11 @@ def test_decode_step_graph_fused_equals_unfused():
             torch.cuda.synchronize()
             outs.append((g.out.clone(), g.lse.clone()))
         assert layer.device_status() == 0
+        del g
         steps.append(outs)
+        layers.append(layer)
     for (oa, la), (ob, lb) in zip(*steps):
         assert torch.equal(oa, ob) and torch.equal(la, lb)
+    a, b = layers
+    assert torch.equal(a.k_pool, b.k_pool) and torch.equal(a.v_pool, b.v_pool)
+    assert torch.equal(a.table, b.table)
