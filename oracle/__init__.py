@@ -61,6 +61,8 @@ def _bind(lib):
     lib.oracle_e4m3_encode.restype = None
     lib.oracle_e4m3_decode.argtypes = [i64, p, dbl, p]
     lib.oracle_e4m3_decode.restype = None
+    lib.oracle_block_mass.argtypes = [i64, i64, p, i64, p, dbl, i64, p]
+    lib.oracle_block_mass.restype = ctypes.c_int
     return lib
 
 
@@ -248,4 +250,25 @@ def e4m3_decode(codes, scale: float, lib=None) -> np.ndarray:
     c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
     out = np.empty(c.shape, np.float64)
     lib.oracle_e4m3_decode(c.size, _ptr(c), float(scale), _ptr(out))
+    return out
+
+
+def block_mass(q, k, block: int, scale: float | None = None, lib=None) -> np.ndarray:
+    """Attention mass per block of ``block`` positions (fp64, [ceil(L / block)]).
+
+    ``q [g, d]``: the g queries of one kv-head's group at the last position of the
+    context; ``k [L, d]``: the context's keys.  Each query's softmax over all L
+    positions, summed per block and averaged over the g queries (the importance a
+    retrieval head's top-p selection reads).  ``scale`` defaults to 1/sqrt(d).
+    """
+    lib = lib or load()
+    q = np.ascontiguousarray(np.atleast_2d(q), dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    g, d = q.shape
+    L = k.shape[0]
+    if scale is None:
+        scale = 1.0 / np.sqrt(np.float64(d))
+    out = np.empty(-(-L // int(block)), np.float64)
+    if lib.oracle_block_mass(g, d, _ptr(q), L, _ptr(k), float(scale), int(block), _ptr(out)) != 0:
+        raise ValueError("oracle: block_mass needs g, d, L, block >= 1")
     return out

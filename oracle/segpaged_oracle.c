@@ -321,3 +321,43 @@ void oracle_e4m3_encode(int64_t n, const float* x, float inv_scale, uint8_t* cod
 void oracle_e4m3_decode(int64_t n, const uint8_t* codes, double scale, double* values) {
   for (int64_t i = 0; i < n; ++i) values[i] = oracle_e4m3_value(codes[i]) * scale;
 }
+
+/*
+ * Attention mass per block: the scoring pass that gives a RETRIEVAL head its
+ * importance.  The pages leave the scoring rule open; the reading taken is
+ * the head's own attention mass per page (four-kind table, retrieval row:
+ * the important tokens are the ones the head attends to).  For the query at
+ * the last position p = L - 1 of a sequence, over its whole causal context
+ * [0, L), in fp64:
+ *   s_hj = scale * q_h . k_j,  a_hj = exp(s_hj - max_j s_hj) / sum_j exp(s_hj - max_j s_hj)
+ *   mass_i = (1 / g) * sum_h sum_{j in [i*block, min((i+1)*block, L))} a_hj
+ * i.e. the softmax probability each of the kv-head's g q-heads puts on block
+ * i, averaged over the group.  q [g][d], k [L][d]; mass [ceil(L / block)] out.
+ * Returns 0, or -1 for sizes < 1.
+ */
+int oracle_block_mass(int64_t g, int64_t d, const double* q, int64_t L, const double* k, double scale,
+                      int64_t block, double* mass) {
+  if (g < 1 || d < 1 || L < 1 || block < 1) return -1;
+  const int64_t nb = (L + block - 1) / block;
+  for (int64_t i = 0; i < nb; ++i) mass[i] = 0.0;
+  double* a = (double*)malloc((size_t)L * sizeof(double));
+  if (!a) return -1;
+  for (int64_t h = 0; h < g; ++h) {
+    const double* qh = q + h * d;
+    double m = -INFINITY;
+    for (int64_t j = 0; j < L; ++j) {
+      double acc = 0.0;
+      for (int64_t t = 0; t < d; ++t) acc += qh[t] * k[j * d + t];
+      a[j] = scale * acc;
+      if (a[j] > m) m = a[j];
+    }
+    double z = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+      a[j] = exp(a[j] - m);
+      z += a[j];
+    }
+    for (int64_t j = 0; j < L; ++j) mass[j / block] += a[j] / z / (double)g;
+  }
+  free(a);
+  return 0;
+}

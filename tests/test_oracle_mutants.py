@@ -39,6 +39,12 @@ MUTANTS = {
     "retrieval_sink_blocks_are_candidates": ("if (taken[i] || (i + 1) * block <= sink) continue;",
                                              "if (taken[i]) continue;"),
     "retrieval_top_p_one_drops_empty_blocks": ("} else if (top_p < 1.0f) {", "} else if (top_p <= 1.0f) {"),
+    # attention mass per block (retrieval importance scoring pass)
+    "block_mass_not_averaged": ("mass[j / block] += a[j] / z / (double)g;", "mass[j / block] += a[j] / z;"),
+    "block_mass_shifted_block": ("mass[j / block] += a[j] / z / (double)g;",
+                                 "mass[(j > 0 ? j - 1 : 0) / block] += a[j] / z / (double)g;"),
+    "block_mass_scale_dropped": ("a[j] = scale * acc;", "a[j] = acc;"),
+    "block_mass_rotated_dims": ("acc += qh[t] * k[j * d + t];", "acc += qh[t] * k[j * d + (t + 1) % d];"),
     # FP8 E4M3 encoder / decoder
     "e4m3_bias_8": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
     "e4m3_subnormal_step": ("ldexp((double)m, -9)", "ldexp((double)m, -10)"),

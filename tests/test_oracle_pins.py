@@ -419,3 +419,66 @@ def test_retrieval_equal_keys_average_the_kept_values():
         np.testing.assert_allclose(out[p], v[vis].mean(0), rtol=0, atol=1e-12)
         s0 = float(q[p] @ k[0]) / math.sqrt(d)
         assert abs(lse[p] - (s0 + math.log(len(vis)))) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# Attention mass per block (the scoring pass behind a retrieval head's importance)
+# --------------------------------------------------------------------------
+
+def _mass_by_hand(q, k, block, scale):
+    """The definition with Python floats: each query's softmax over all positions, summed per block,
+    averaged over the queries."""
+    g, L = len(q), len(k)
+    nb = -(-L // block)
+    out = [0.0] * nb
+    for h in range(g):
+        s = [scale * math.fsum(a * b for a, b in zip(q[h], k[j])) for j in range(L)]
+        m = max(s)
+        e = [math.exp(x - m) for x in s]
+        z = math.fsum(e)
+        for i in range(nb):
+            out[i] += math.fsum(e[i * block:(i + 1) * block]) / z / g
+    return out
+
+
+@pytest.mark.parametrize("g,d,L,block", [(1, 4, 9, 4), (2, 8, 37, 8), (4, 16, 64, 16), (3, 5, 1, 4)])
+def test_block_mass_matches_brute_force(g, d, L, block):
+    rng = np.random.default_rng(g * 100 + L)
+    q, k = _rand(rng, g, d), _rand(rng, L, d)
+    scale = 1.0 / math.sqrt(d)
+    got = oracle.block_mass(q, k, block)
+    ref = _mass_by_hand(q.tolist(), k.tolist(), block, scale)
+    assert np.allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_block_mass_is_a_distribution():
+    rng = np.random.default_rng(5)
+    for L, block in ((1000, 64), (999, 64), (65, 64), (64, 64)):
+        m = oracle.block_mass(_rand(rng, 8, 32), 3.0 * _rand(rng, L, 32), block)
+        assert len(m) == -(-L // block) and (m >= 0).all() and abs(m.sum() - 1.0) < 1e-12
+
+
+def test_block_mass_equal_keys_is_proportional_to_block_length():
+    """Equal keys give every position the same weight: block i's mass is its length over L
+    (the ragged last block included)."""
+    rng = np.random.default_rng(6)
+    L, block = 200, 64
+    k = np.tile(_rand(rng, 1, 16), (L, 1))
+    m = oracle.block_mass(_rand(rng, 4, 16), k, block)
+    lens = np.array([min(block, L - i * block) for i in range(-(-L // block))], np.float64)
+    assert np.allclose(m, lens / L, rtol=0, atol=1e-14)
+
+
+def test_block_mass_dominant_key_and_group_average():
+    """One key aligned with the query at 40 sigma takes essentially all of that query's mass; a second
+    query of the group that attends uniformly (zero query) spreads its half evenly."""
+    rng = np.random.default_rng(7)
+    L, d, block = 300, 16, 64
+    k = 0.1 * _rand(rng, L, d)
+    q0 = _rand(rng, d)
+    k[170] = 40.0 * math.sqrt(d) * q0 / (q0 @ q0)  # q0 . k_170 * scale = 40
+    m1 = oracle.block_mass(q0[None], k, block)
+    assert m1[170 // block] > 1 - 1e-12
+    m2 = oracle.block_mass(np.stack([q0, np.zeros(d)]), k, block)  # the zero query weighs every key 1 / L
+    lens = np.array([min(block, L - i * block) for i in range(-(-L // block))], np.float64)
+    assert np.allclose(m2, (m1 + lens / L) / 2, rtol=0, atol=1e-14)
