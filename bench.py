@@ -362,10 +362,13 @@ def run_retrieval(wl, dev, flush, world) -> dict:
     Per sequence: the layer's global kv-head, two retrieval kv-heads (sink 4, window 512,
     top_p 0.5 of the synthetic per-page importance) and five local ones (sink 4, window 8192).
     Rates count only the work the heads' visible sets need: stored K+V bytes for decode,
-    4 * head_dim FLOPs per visible pair for prefill.
+    4 * head_dim FLOPs per visible pair for prefill.  The scoring pass that computes a
+    retrieval head's importance (attention mass per page, segpaged_block_mass) is timed on
+    the same layer: it reads every key once.
     """
     import torch
 
+    from head_aware_paged_build_b200 import segpaged as S
     from head_aware_paged_build_b200 import workloads as W
     from head_aware_paged_build_b200.runtime import layer_for
 
@@ -382,11 +385,27 @@ def run_retrieval(wl, dev, flush, world) -> dict:
     d_ms = median_ms(lambda: ld.attention(qd, od, lsed), flush, 10)
     p_ms = median_ms(lambda: lp.attention(qp, op, lsep), flush, 3)
     assert ld.device_status() == 0 and lp.device_status() == 0
-    d_ms, p_ms = reduce_max([d_ms, p_ms], world, dev)
+    # the scoring pass that gives retrieval heads their importance (segpaged_block_mass):
+    # every key of every (sequence, kv-head) read once, with the queries at the last position
+    B, hkv, L, d = k.shape
+    mprob = S.make_problem(B, wr.num_q_heads, hkv, d, wr.page_size, "bf16", dec.ctx_lens,
+                           [x - 1 for x in dec.ctx_lens], [("global", 0, 0)] * (B * hkv))
+    nb = -(-L // wr.page_size)
+    mass = torch.empty(B, hkv, nb, dtype=torch.float32, device=dev)
+    mws = torch.empty(S.segpaged_block_mass_workspace(mprob), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream().cuda_stream
+    m_ms = median_ms(lambda: S.segpaged_block_mass(mprob, k.data_ptr(), k.stride(0), k.stride(1), k.stride(2),
+                                                   qd.data_ptr(), 0.0, mass.data_ptr(), nb, mws.data_ptr(),
+                                                   mws.numel(), stream), flush, 10)
+    d_ms, p_ms, m_ms = reduce_max([d_ms, p_ms, m_ms], world, dev)
     pk = peaks()
     vis = ld.sizes.stored_token_heads * 2 * wr.head_dim * 2
     flops = 4 * wr.head_dim * lp.sizes.visible_pairs
-    return {"decode_ms": round(d_ms, 5), "decode_visible_kv_bytes": vis,
+    key_bytes = sum(dec.ctx_lens) * hkv * d * 2
+    return {"block_mass_ms": round(m_ms, 5), "block_mass_key_bytes": key_bytes,
+            "block_mass_GB/s": round(weak_rate(key_bytes, world, m_ms) / 1e9, 1),
+            "block_mass_frac_hbm": round(key_bytes / (m_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+            "decode_ms": round(d_ms, 5), "decode_visible_kv_bytes": vis,
             "decode_GB/s": round(weak_rate(vis, world, d_ms) / 1e9, 1),
             "decode_frac_hbm": round(vis / (d_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
             "prefill_ms": round(p_ms, 4), "prefill_visible_flops": flops,

@@ -130,4 +130,25 @@ struct AppendLaunch {
 };
 cudaError_t launch_append(const AppendLaunch& a, cudaStream_t s);
 
+// Attention mass per page-size block (segpaged_block_mass): the importance a
+// retrieval head's top-p selection reads.  Passed by value (__grid_constant__),
+// the per-sequence context lengths included.
+constexpr int kMassMaxBatch = 2048;
+constexpr int kMassBlock = 64;  // positions per block (the bf16 page size)
+struct BlockMassLaunch {
+  const void* k;  // dense bf16 keys, element strides below, head_dim contiguous
+  int64_t stride_seq, stride_head, stride_tok;
+  const void* q;  // [B, Hq, D] bf16: each sequence's query at its last position
+  float scale_log2;
+  int32_t B, Hq, Hkv, G, D;
+  int32_t nb_max;          // blocks of the longest sequence: the workspace's row pitch
+  int32_t blocks_per_cta;  // grid.x = ceil(nb_max / blocks_per_cta), grid.y = B * Hkv
+  float* ws_m;             // [B * Hq][nb_max]: a block's score maximum (log2 units)
+  float* ws_s;             // [B * Hq][nb_max]: its sum of 2^(score - maximum)
+  float* mass;             // [B * Hkv][mass_stride]
+  int64_t mass_stride;
+  int32_t L[kMassMaxBatch];
+};
+cudaError_t launch_block_mass(const BlockMassLaunch& a, cudaStream_t s);
+
 }  // namespace sp

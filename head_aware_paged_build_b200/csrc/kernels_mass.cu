@@ -1,0 +1,256 @@
+// Attention mass per page-size block: the scoring pass behind a retrieval
+// head's importance.  The pages leave the scoring rule open ("RedKnot head
+// classification", four-kind table: a retrieval head fetches only the pages
+// that matter); the reading taken is the head's own attention mass per page.
+// For each sequence b and kv-head kv, the query of each q-head h of the GQA
+// group at the last position L_b - 1 attends over the whole context [0, L_b):
+//   mass[b][kv][i] = (1 / g) * sum_h sum_{j in block i} softmax_j(scale * q_h . k_j)
+// with blocks of 64 positions (the bf16 page size).
+//
+// Pass 1 (block_mass_kernel): one warp per block.  The GQA group's g query
+// rows are the 16 rows of mma.sync.m16n8k16 (bf16, fp32 accumulate) and each
+// lane loads its tokens' keys straight from the dense cache, 16 bytes at a
+// time: lane tq of a quad owns dimensions 32 j + 8 tq .. +7 of its token, and
+// the query fragments use the same permutation of the 32 dimensions of each
+// group, so the dot products are unchanged.  Per (q-head, block) it writes the
+// block's score maximum m and sum 2^(s - m) (log2 units).
+// Pass 2 (block_mass_combine_kernel): one CTA per (sequence, kv-head): per
+// q-head M = max over blocks, Z = sum_blocks s_i 2^(m_i - M); mass_i =
+// (1 / g) sum_h s_hi 2^(m_hi - M_h) / Z_h.  Every sum runs in a fixed order,
+// so results are bitwise reproducible.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+#include <string>
+
+#include "device_common.cuh"
+#include "kernels.h"
+
+namespace sp {
+namespace {
+
+constexpr uint32_t kFull = 0xffffffffu;
+constexpr int kMassThreads = 128;     // pass 1: 4 warps, one block each per step
+constexpr int kCombineThreads = 256;  // pass 2
+
+template <int D>
+__global__ void __launch_bounds__(kMassThreads) block_mass_kernel(const __grid_constant__ BlockMassLaunch a) {
+  const int bk = blockIdx.y, b = bk / a.Hkv, kv = bk % a.Hkv;
+  const int L = a.L[b], nb = (L + kMassBlock - 1) / kMassBlock;
+  const int blk0 = blockIdx.x * a.blocks_per_cta, blk1 = min(nb, blk0 + a.blocks_per_cta);
+  if (blk0 >= blk1) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = lane >> 2, tq = lane & 3;
+  const int G = a.G, r0 = grp, r1 = grp + 8;
+
+  // query fragments: k-steps 2j, 2j+1 cover dimensions 32 j .. 32 j + 31, lane tq
+  // holds dimensions 32 j + 8 tq .. +7 (pairs {0,1},{2,3} -> k-step 2j, {4,5},{6,7} -> 2j+1)
+  uint32_t qa[D / 16][4];
+  const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(a.q) + (int64_t(b) * a.Hq + kv * G) * D;
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j) {
+    const int c0 = 32 * j + 8 * tq;
+    const uint4 x0 = r0 < G ? *reinterpret_cast<const uint4*>(qrow + r0 * D + c0) : make_uint4(0, 0, 0, 0);
+    const uint4 x1 = r1 < G ? *reinterpret_cast<const uint4*>(qrow + r1 * D + c0) : make_uint4(0, 0, 0, 0);
+    qa[2 * j][0] = x0.x, qa[2 * j][2] = x0.y, qa[2 * j + 1][0] = x0.z, qa[2 * j + 1][2] = x0.w;
+    qa[2 * j][1] = x1.x, qa[2 * j][3] = x1.y, qa[2 * j + 1][1] = x1.z, qa[2 * j + 1][3] = x1.w;
+  }
+  const __nv_bfloat16* kb =
+      static_cast<const __nv_bfloat16*>(a.k) + int64_t(b) * a.stride_seq + int64_t(kv) * a.stride_head;
+  const float sl2 = a.scale_log2;
+  const int64_t row0 = (int64_t(b) * a.Hq + kv * G + r0) * a.nb_max;
+  const int64_t row1 = (int64_t(b) * a.Hq + kv * G + r1) * a.nb_max;
+
+  for (int blk = blk0 + warp; blk < blk1; blk += kMassThreads / 32) {
+    const int t0 = blk * kMassBlock;
+    float sc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {  // 8 tiles of 8 tokens; this lane's B-fragment token is t0 + 8 nt + grp
+      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      const int tok = t0 + nt * 8 + grp;
+      const __nv_bfloat16* kr = kb + int64_t(tok) * a.stride_tok + 8 * tq;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        const uint4 u = tok < L ? __ldg(reinterpret_cast<const uint4*>(kr + 32 * j)) : make_uint4(0, 0, 0, 0);
+        mma_bf16_16816(sc[nt], qa[2 * j], u.x, u.y);
+        mma_bf16_16816(sc[nt], qa[2 * j + 1], u.z, u.w);
+      }
+    }
+    // scores in log2 units, positions past the context masked; c0, c1: row r0, c2, c3: row r1
+    float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = t0 + nt * 8 + 2 * tq + (e & 1);
+        const float x = tok < L ? sc[nt][e] * sl2 : -INFINITY;
+        sc[nt][e] = x;
+        if (e < 2) m0 = fmaxf(m0, x); else m1 = fmaxf(m1, x);
+      }
+    m0 = fmaxf(m0, __shfl_xor_sync(kFull, m0, 1));
+    m0 = fmaxf(m0, __shfl_xor_sync(kFull, m0, 2));
+    m1 = fmaxf(m1, __shfl_xor_sync(kFull, m1, 1));
+    m1 = fmaxf(m1, __shfl_xor_sync(kFull, m1, 2));
+    float s0 = 0.f, s1 = 0.f;  // every block holds a valid position, so m0, m1 are finite
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      s0 += fast_exp2(sc[nt][0] - m0) + fast_exp2(sc[nt][1] - m0);
+      s1 += fast_exp2(sc[nt][2] - m1) + fast_exp2(sc[nt][3] - m1);
+    }
+    s0 += __shfl_xor_sync(kFull, s0, 1);
+    s0 += __shfl_xor_sync(kFull, s0, 2);
+    s1 += __shfl_xor_sync(kFull, s1, 1);
+    s1 += __shfl_xor_sync(kFull, s1, 2);
+    if (tq == 0) {
+      if (r0 < G) a.ws_m[row0 + blk] = m0, a.ws_s[row0 + blk] = s0;
+      if (r1 < G) a.ws_m[row1 + blk] = m1, a.ws_s[row1 + blk] = s1;
+    }
+  }
+}
+
+// Block-wide reduction in a fixed order (warp butterfly, then the warps' results in order).
+template <bool MAX>
+__device__ __forceinline__ float block_reduce(float v, float* scratch) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float w = __shfl_xor_sync(kFull, v, o);
+    v = MAX ? fmaxf(v, w) : v + w;
+  }
+  const int warp = threadIdx.x >> 5;
+  __syncthreads();  // scratch free from the previous reduction
+  if ((threadIdx.x & 31) == 0) scratch[warp] = v;
+  __syncthreads();
+  float r = scratch[0];
+  for (int w = 1; w < kCombineThreads / 32; ++w) r = MAX ? fmaxf(r, scratch[w]) : r + scratch[w];
+  return r;
+}
+
+__global__ void __launch_bounds__(kCombineThreads) block_mass_combine_kernel(const __grid_constant__ BlockMassLaunch a) {
+  __shared__ float scratch[kCombineThreads / 32];
+  __shared__ float s_max[16], s_inv[16];
+  const int bk = blockIdx.x, b = bk / a.Hkv, kv = bk % a.Hkv;
+  const int L = a.L[b], nb = (L + kMassBlock - 1) / kMassBlock;
+  const int G = a.G;
+  for (int h = 0; h < G; ++h) {
+    const int64_t row = (int64_t(b) * a.Hq + kv * G + h) * a.nb_max;
+    float m = -INFINITY;
+    for (int i = threadIdx.x; i < nb; i += kCombineThreads) m = fmaxf(m, a.ws_m[row + i]);
+    const float M = block_reduce<true>(m, scratch);
+    float z = 0.f;
+    for (int i = threadIdx.x; i < nb; i += kCombineThreads) z += a.ws_s[row + i] * exp2f(a.ws_m[row + i] - M);
+    const float Z = block_reduce<false>(z, scratch);
+    if (threadIdx.x == 0) s_max[h] = M, s_inv[h] = 1.f / Z;
+  }
+  __syncthreads();
+  float* out = a.mass + int64_t(bk) * a.mass_stride;
+  const float inv_g = 1.f / float(G);
+  for (int i = threadIdx.x; i < nb; i += kCombineThreads) {
+    float acc = 0.f;
+    for (int h = 0; h < G; ++h) {
+      const int64_t idx = (int64_t(b) * a.Hq + kv * G + h) * a.nb_max + i;
+      acc += a.ws_s[idx] * exp2f(a.ws_m[idx] - s_max[h]) * s_inv[h];
+    }
+    out[i] = acc * inv_g;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_block_mass(const BlockMassLaunch& a, cudaStream_t s) {
+  const dim3 grid((a.nb_max + a.blocks_per_cta - 1) / a.blocks_per_cta, a.B * a.Hkv);
+  if (a.D == 128)
+    block_mass_kernel<128><<<grid, kMassThreads, 0, s>>>(a);
+  else
+    block_mass_kernel<64><<<grid, kMassThreads, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  block_mass_combine_kernel<<<a.B * a.Hkv, kCombineThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace sp
+
+// ---------------------------------------------------------------------------
+// C ABI
+// ---------------------------------------------------------------------------
+namespace sp {
+namespace {
+
+sp_status mass_shape(const sp_problem* p, int32_t& G, int32_t& nb_max) {
+  if (!p) return fail(SP_ERR_INVALID_ARG, "problem is NULL");
+  if (p->batch < 1 || p->num_q_heads < 1 || p->num_kv_heads < 1)
+    return fail(SP_ERR_INVALID_ARG, "batch and head counts must be >= 1");
+  if (p->batch > kMassMaxBatch) return fail(SP_ERR_UNSUPPORTED, "segpaged_block_mass: at most 2048 sequences");
+  if (p->dtype != SP_BF16) return fail(SP_ERR_UNSUPPORTED, "segpaged_block_mass: bf16 keys and queries only");
+  if (p->head_dim != 64 && p->head_dim != 128) return fail(SP_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (p->page_size != kMassBlock) return fail(SP_ERR_UNSUPPORTED, "segpaged_block_mass: page_size must be 64");
+  if (p->num_q_heads % p->num_kv_heads != 0 || p->num_q_heads / p->num_kv_heads > 16)
+    return fail(SP_ERR_UNSUPPORTED, "num_q_heads must be a multiple of num_kv_heads, at most 16 times it");
+  if (!p->ctx_len) return fail(SP_ERR_INVALID_ARG, "ctx_len is NULL");
+  int64_t lmax = 0;
+  for (int b = 0; b < p->batch; ++b) {
+    if (p->ctx_len[b] < 1) return fail(SP_ERR_INVALID_ARG, "ctx_len must be >= 1");
+    lmax = std::max<int64_t>(lmax, p->ctx_len[b]);
+  }
+  G = p->num_q_heads / p->num_kv_heads;
+  nb_max = int32_t((lmax + kMassBlock - 1) / kMassBlock);
+  return SP_OK;
+}
+
+int64_t mass_workspace_bytes(const sp_problem* p, int32_t nb_max) {
+  const int64_t raw = 2 * int64_t(p->batch) * p->num_q_heads * nb_max * int64_t(sizeof(float));
+  return (raw + 255) / 256 * 256;
+}
+
+}  // namespace
+}  // namespace sp
+
+extern "C" sp_status segpaged_block_mass_workspace(const sp_problem* problem, size_t* bytes) {
+  using namespace sp;
+  int32_t G, nb_max;
+  const sp_status st = mass_shape(problem, G, nb_max);
+  if (st != SP_OK) return st;
+  if (!bytes) return fail(SP_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = size_t(mass_workspace_bytes(problem, nb_max));
+  return SP_OK;
+}
+
+extern "C" sp_status segpaged_block_mass(const sp_problem* problem, const void* k_dense, int64_t stride_seq,
+                                         int64_t stride_head, int64_t stride_tok, const void* q, float softmax_scale,
+                                         float* mass, int64_t mass_stride, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  using namespace sp;
+  int32_t G, nb_max;
+  sp_status st = mass_shape(problem, G, nb_max);
+  if (st != SP_OK) return st;
+  auto al = [](const void* ptr, uintptr_t n) { return (reinterpret_cast<uintptr_t>(ptr) % n) == 0; };
+  if (!k_dense || !q || !mass || !workspace) return fail(SP_ERR_INVALID_ARG, "k_dense, q, mass and workspace must be non-NULL");
+  if (!al(k_dense, 16) || !al(q, 16) || !al(mass, 4) || !al(workspace, 256))
+    return fail(SP_ERR_INVALID_ARG, "k_dense and q must be 16-byte aligned, mass 4-byte, workspace 256-byte");
+  if (stride_seq < 0 || stride_head < 0 || stride_tok < 0 || stride_seq % 8 || stride_head % 8 || stride_tok % 8)
+    return fail(SP_ERR_INVALID_ARG, "strides must be >= 0 and multiples of 8 elements (16-byte rows)");
+  if (mass_stride < nb_max) return fail(SP_ERR_INVALID_ARG, "mass_stride below ceil(max ctx_len / page_size)");
+  if (int64_t(workspace_bytes) < mass_workspace_bytes(problem, nb_max))
+    return fail(SP_ERR_WORKSPACE, "workspace smaller than segpaged_block_mass_workspace");
+  if (!std::isfinite(softmax_scale)) return fail(SP_ERR_INVALID_ARG, "softmax_scale must be finite");
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(problem->head_dim));
+  static BlockMassLaunch a;  // 8 KB of lengths: kept off the caller's stack
+  static std::mutex mu;      // the launch copies it; one call fills it at a time
+  std::lock_guard<std::mutex> lock(mu);
+  a = BlockMassLaunch{};
+  a.k = k_dense, a.q = q;
+  a.stride_seq = stride_seq, a.stride_head = stride_head, a.stride_tok = stride_tok;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.B = problem->batch, a.Hq = problem->num_q_heads, a.Hkv = problem->num_kv_heads, a.G = G;
+  a.D = problem->head_dim;
+  a.nb_max = nb_max;
+  a.blocks_per_cta = 16;
+  float* ws = static_cast<float*>(workspace);
+  a.ws_m = ws;
+  a.ws_s = ws + int64_t(a.B) * a.Hq * nb_max;
+  a.mass = mass, a.mass_stride = mass_stride;
+  for (int b = 0; b < a.B; ++b) a.L[b] = problem->ctx_len[b];
+  const cudaError_t e = launch_block_mass(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SP_OK : fail(SP_ERR_CUDA, std::string("segpaged_block_mass launch: ") + cudaGetErrorString(e));
+}

@@ -198,6 +198,35 @@ def layer_for(prob, device="cuda", flags: int = 0, **kw) -> SegPagedLayer:
                          q_start=prob.q_starts, policy=wl.policy, device=device, flags=flags, **kw)
 
 
+def block_mass(k_dense: torch.Tensor, q: torch.Tensor, ctx_len: Sequence[int], page_size: int = 64,
+               scale: float = 0.0, stream=None) -> torch.Tensor:
+    """The attention mass per page-size block of each (sequence, kv-head): the importance a retrieval
+    head's top-p selection reads (``segpaged_block_mass``).
+
+    ``k_dense``: bf16 [B, Hkv, Lmax, d] (d contiguous, rows 16-byte aligned); ``q``: bf16 [B, Hq, d]
+    contiguous, each sequence's queries at its last position ``ctx_len[b] - 1``.  Returns fp32
+    [B, Hkv, ceil(Lmax / page_size)] on k's device; row (b, kv) holds ceil(ctx_len[b] / page_size)
+    masses summing to 1, zeros after them.  ``[m[b, kv, :n].tolist() ...]`` are the ``block_mass``
+    entries a plan takes.
+    """
+    B, hkv, lmax, d = k_dense.shape
+    if k_dense.dtype != torch.bfloat16 or q.dtype != torch.bfloat16:
+        raise ValueError("block_mass: bf16 keys and queries")
+    if k_dense.stride(-1) != 1 or not q.is_contiguous() or tuple(q.shape[::2]) != (B, d) or q.shape[1] % hkv:
+        raise ValueError(f"block_mass: q must be contiguous [{B}, Hq, {d}] with Hq a multiple of {hkv}")
+    if len(ctx_len) != B or max(ctx_len) > lmax or min(ctx_len) < 1:
+        raise ValueError("block_mass: one ctx_len in [1, Lmax] per sequence")
+    hq = q.shape[1]
+    prob = S.make_problem(B, hq, hkv, d, page_size, "bf16", ctx_len, [L - 1 for L in ctx_len],
+                          [("global", 0, 0)] * (B * hkv))
+    nb = -(-lmax // page_size)
+    out = torch.zeros(B, hkv, nb, dtype=torch.float32, device=k_dense.device)
+    ws = torch.empty(S.segpaged_block_mass_workspace(prob), dtype=torch.uint8, device=k_dense.device)
+    S.segpaged_block_mass(prob, k_dense.data_ptr(), k_dense.stride(0), k_dense.stride(1), k_dense.stride(2),
+                          q.data_ptr(), scale, out.data_ptr(), nb, ws.data_ptr(), ws.numel(), _stream(stream))
+    return out
+
+
 def build_layers(layers: Sequence[SegPagedLayer], k_dense: Sequence[torch.Tensor], v_dense: Sequence[torch.Tensor],
                  varlen: bool = False, stream=None) -> None:
     """Pack several layers that share one pair of pools with a single launch.

@@ -33,8 +33,8 @@ EXPORTED = ("segpaged_plan_create", "segpaged_plan_destroy", "segpaged_plan_size
             "build_segpaged_cache", "build_segpaged_cache_layers", "segpaged_gather", "segpaged_attention",
             "segpaged_attention_decode_noalloc", "segpaged_decode_append", "segpaged_decode_step",
             "segpaged_read_device_status",
-            "segpaged_clear_device_status", "segpaged_eval_exp2_fma", "segpaged_status_string",
-            "segpaged_last_error", "segpaged_abi_version")
+            "segpaged_clear_device_status", "segpaged_eval_exp2_fma", "segpaged_block_mass_workspace",
+            "segpaged_block_mass", "segpaged_status_string", "segpaged_last_error", "segpaged_abi_version")
 
 
 class SegPagedError(RuntimeError):
@@ -114,6 +114,9 @@ def load(path: Path | str | None = None) -> ctypes.CDLL:
         "segpaged_read_device_status": ([vp, ctypes.POINTER(i32), vp], i32),
         "segpaged_clear_device_status": ([vp, vp], i32),
         "segpaged_eval_exp2_fma": ([vp, vp, i64, vp], i32),
+        "segpaged_block_mass_workspace": ([ctypes.POINTER(sp_problem), ctypes.POINTER(sz)], i32),
+        "segpaged_block_mass": ([ctypes.POINTER(sp_problem), vp, i64, i64, i64, vp, ctypes.c_float, vp, i64, vp,
+                                 sz, vp], i32),
         "segpaged_status_string": ([i32], ctypes.c_char_p),
         "segpaged_last_error": ([], ctypes.c_char_p),
         "segpaged_abi_version": ([], i32),
@@ -336,6 +339,28 @@ def segpaged_clear_device_status(workspace: int, stream: int = 0) -> None:
 def segpaged_eval_exp2_fma(d_x: int, d_y: int, n: int, stream: int = 0) -> None:
     """y = the prefill kernel's FMA-pipe 2^x of x (device float arrays of n elements)."""
     _check(load().segpaged_eval_exp2_fma(d_x, d_y, n, stream), "segpaged_eval_exp2_fma")
+
+
+def segpaged_block_mass_workspace(problem: sp_problem) -> int:
+    """Workspace bytes segpaged_block_mass needs for ``problem``."""
+    n = ctypes.c_size_t()
+    _check(load().segpaged_block_mass_workspace(ctypes.byref(problem), ctypes.byref(n)),
+           "segpaged_block_mass_workspace")
+    return n.value
+
+
+def segpaged_block_mass(problem: sp_problem, k_dense: int, stride_seq: int, stride_head: int, stride_tok: int,
+                        q: int, softmax_scale: float, mass: int, mass_stride: int, workspace: int,
+                        workspace_bytes: int, stream: int = 0) -> None:
+    """The attention mass per page-size block of each (sequence, kv-head): a retrieval head's importance."""
+    _check(load().segpaged_block_mass(ctypes.byref(problem), k_dense, stride_seq, stride_head, stride_tok, q,
+                                      softmax_scale, mass, mass_stride, workspace, workspace_bytes, stream),
+           "segpaged_block_mass")
+
+
+def segpaged_block_mass_status(problem: sp_problem, *args) -> int:
+    """Like segpaged_block_mass but returns the status code instead of raising."""
+    return load().segpaged_block_mass(ctypes.byref(problem), *args)
 
 
 def segpaged_abi_version() -> int:

@@ -449,6 +449,42 @@ SP_API sp_status segpaged_decode_step(const sp_plan* plan, void* d_table, const 
 SP_API sp_status segpaged_read_device_status(const void* workspace, int32_t* code, void* stream);
 SP_API sp_status segpaged_clear_device_status(void* workspace, void* stream);
 
+/* segpaged_block_mass: the importance a RETRIEVAL head's top-p selection
+ * reads, computed on the device from the dense cache: the head's own
+ * attention mass per page-size block.  The pages leave the scoring rule open
+ * ("RedKnot head classification", four-kind table, retrieval row: the head
+ * fetches only the important tokens, page by page); the reading taken: for
+ * sequence b and kv-head kv, each q-head h of the GQA group attends with its
+ * query at the last position L_b - 1 over the whole context [0, L_b), and
+ *   mass[b * num_kv_heads + kv][i] = (1 / g) sum_h sum_{j in block i} softmax_j(scale q_h . k_j)
+ * for blocks i of page_size positions [i P, (i + 1) P), the last one ragged;
+ * every row sums to 1.  Its rows are the block_mass entries a plan takes.
+ *   problem   host; only batch, num_q_heads, num_kv_heads, head_dim,
+ *             page_size, dtype and ctx_len are read.  bf16 only, page_size 64,
+ *             head_dim 64 or 128, g = num_q_heads / num_kv_heads <= 16,
+ *             batch <= 2048 (else SP_ERR_UNSUPPORTED); ctx_len[b] >= 1.
+ *   k_dense   device bf16 keys, element strides stride_seq, stride_head,
+ *             stride_tok (multiples of 8, head_dim contiguous), 16-byte aligned
+ *             (the layout build_segpaged_cache reads)
+ *   q         device bf16 [batch, num_q_heads, head_dim], 16-byte aligned:
+ *             each sequence's queries at its last position
+ *   softmax_scale  <= 0 selects 1 / sqrt(head_dim)
+ *   mass      device fp32 [batch * num_kv_heads][mass_stride], mass_stride >=
+ *             ceil(max ctx_len / page_size); entries i < ceil(ctx_len[b] /
+ *             page_size) of each row are written, the rest left as they are
+ *   workspace device, 256-byte aligned, at least the bytes
+ *             segpaged_block_mass_workspace gives (SP_ERR_WORKSPACE if smaller);
+ *             fully overwritten, no zeroing needed
+ * Two launches on `stream` (a pass over the keys, one warp per block, then a
+ * per (sequence, kv-head) normalisation); fixed summation orders, so the
+ * result is bitwise reproducible.  Argument errors are reported before any
+ * launch.  Calls from several host threads are serialised on the host. */
+SP_API sp_status segpaged_block_mass_workspace(const sp_problem* problem, size_t* bytes);
+SP_API sp_status segpaged_block_mass(const sp_problem* problem, const void* k_dense, int64_t stride_seq,
+                                     int64_t stride_head, int64_t stride_tok, const void* q, float softmax_scale,
+                                     float* mass, int64_t mass_stride, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
 /* segpaged_eval_exp2_fma: y[i] = 2^x[i] as the bf16 prefill kernel computes
  * it on the FMA pipe for one exponent pair in sixteen (the pages have no
  * counterpart: it is this library's own 2^x, a cubic on [-1/2, 1/2] fitted by

@@ -362,3 +362,36 @@ def test_ring_plan_spare_pool_ids_and_checks():
         q = S.make_problem(3, 4, 2, 128, 64, "bf16", L0, [L - 1 for L in L0], pol, **bad)
         st, pl = S.segpaged_plan_create_status(q)
         assert st == code and not pl
+
+
+def test_block_mass_argument_checks():
+    """segpaged_block_mass reports every argument error on the host, before any launch."""
+    import ctypes
+
+    def prob(**kw):
+        base = dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=128, page_size=64, dtype="bf16",
+                    ctx_len=[700, 1300], q_start=[699, 1299], policy=[("global", 0, 0)] * 4)
+        base.update(kw)
+        return S.make_problem(**base)
+
+    n = ctypes.c_size_t()
+    for kw, code in ((dict(page_size=16), S.SP_ERR_UNSUPPORTED), (dict(dtype="f32"), S.SP_ERR_UNSUPPORTED),
+                     (dict(head_dim=96), S.SP_ERR_UNSUPPORTED),
+                     (dict(num_q_heads=34, num_kv_heads=2, policy=[("global", 0, 0)] * 4), S.SP_ERR_UNSUPPORTED),
+                     (dict(num_q_heads=7), S.SP_ERR_UNSUPPORTED),
+                     (dict(ctx_len=[700, 0]), S.SP_ERR_INVALID_ARG)):
+        assert S.load().segpaged_block_mass_workspace(ctypes.byref(prob(**kw)), ctypes.byref(n)) == code, kw
+    p = prob()
+    ws = S.segpaged_block_mass_workspace(p)
+    assert ws == -(-2 * 2 * 8 * 21 * 4 // 256) * 256  # 2 floats per (q-head, block), 21 blocks of the longest
+    good = (1 << 20, 128 * 2048 * 2, 2048 * 128, 128, 2 << 20, 0.0, 4 << 20, 21, 8 << 20, ws, None)
+    for i, bad, code in ((0, 0, S.SP_ERR_INVALID_ARG), (0, 8, S.SP_ERR_INVALID_ARG),  # NULL, misaligned keys
+                         (3, 12, S.SP_ERR_INVALID_ARG),                                 # stride not a multiple of 8
+                         (4, 0, S.SP_ERR_INVALID_ARG), (6, 0, S.SP_ERR_INVALID_ARG),    # NULL q, NULL mass
+                         (5, float("nan"), S.SP_ERR_INVALID_ARG),                      # scale
+                         (7, 20, S.SP_ERR_INVALID_ARG),                                 # mass_stride < 21 blocks
+                         (8, 64, S.SP_ERR_INVALID_ARG),                                 # workspace not 256-aligned
+                         (9, ws - 256, S.SP_ERR_WORKSPACE)):
+        args = list(good)
+        args[i] = bad
+        assert S.segpaged_block_mass_status(p, *args) == code, (i, bad, S.last_error())

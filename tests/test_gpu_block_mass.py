@@ -1,0 +1,71 @@
+"""segpaged_block_mass: the attention mass per page-size block (a retrieval head's importance).
+
+Each (sequence, kv-head) row is compared with the fp64 oracle's block mass of
+the same keys and queries: every entry within 2e-4 relative + 1e-7 absolute
+(fp32 scores of bf16 products, fp32 sums), rows summing to 1, zeros after a
+row's blocks.  Shapes: the Llama-70B-shaped 32K layer at batch 8, head_dim 64
+with 16 q-heads per kv-head, one q-head per kv-head, ragged lengths (1, one
+block, one position past a block, a partial last block), keys read through
+a [B, L, Hkv, d] layout; repeated calls are bitwise equal.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from head_aware_paged_build_b200 import workloads as W
+from head_aware_paged_build_b200.runtime import block_mass
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _inputs(name, seed, B, hq, hkv, d, lens):
+    wl = W.custom(name, seed, B, hq, hkv, d, "bf16", 64, lens, [("global", 0, 0)] * (B * hkv))
+    prob = wl.decode_problem()  # one query per sequence, at its last position
+    k, _ = W.dense_kv(prob, device="cuda", gen_device="cuda")
+    q = W.queries(prob, device="cuda", gen_device="cuda")
+    return wl, k, q
+
+
+def _check(m, k, q, lens, hkv):
+    mh, kh, qh = m.cpu().double().numpy(), k.cpu(), q.cpu()
+    g = q.shape[1] // hkv
+    for b, L in enumerate(lens):
+        nb = -(-L // 64)
+        for kv in range(hkv):
+            ref = oracle.block_mass(qh[b, kv * g:(kv + 1) * g].double().numpy(), kh[b, kv, :L].double().numpy(), 64)
+            got = mh[b, kv]
+            assert np.all(np.abs(got[:nb] - ref) <= 2e-4 * ref + 1e-7), (b, kv, np.abs(got[:nb] - ref).max())
+            assert abs(got[:nb].sum() - 1.0) < 1e-5 and not got[nb:].any(), (b, kv)
+
+
+@pytest.mark.parametrize("name,B,hq,hkv,d,lens", [
+    ("mass_llama", 8, 64, 8, 128, (32768,) * 8),
+    ("mass_d64_g16", 2, 32, 2, 64, (4000, 1500)),
+    ("mass_mha", 2, 4, 4, 128, (3000, 700)),
+    ("mass_ragged", 5, 16, 4, 128, (1, 64, 65, 130, 1999)),
+])
+def test_block_mass_matches_oracle(name, B, hq, hkv, d, lens):
+    wl, k, q = _inputs(name, 11, B, hq, hkv, d, lens)
+    m = block_mass(k, q, lens)
+    torch.cuda.synchronize()
+    _check(m, k, q, lens, hkv)
+    assert torch.equal(m, block_mass(k, q, lens))  # fixed summation orders: bitwise repeatable
+
+
+def test_block_mass_reads_any_key_layout():
+    """Keys laid out [B, L, Hkv, d] (token-major), read through the strides, give the same masses bit for bit."""
+    lens = (777, 1290)
+    wl, k, q = _inputs("mass_layout", 12, 2, 8, 2, 128, lens)
+    tok_major = k.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)  # same values, strides (L Hkv d, d, Hkv d)
+    assert tok_major.stride(1) == 128 and tok_major.stride(2) == 2 * 128
+    m = block_mass(tok_major, q, lens)
+    assert torch.equal(m, block_mass(k, q, lens))
+    _check(m, k, q, lens, 2)
