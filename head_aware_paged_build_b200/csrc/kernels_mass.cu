@@ -16,8 +16,8 @@
 // block's score maximum m and sum 2^(s - m) (log2 units).
 // Pass 2 (block_mass_combine_kernel): one CTA per (sequence, kv-head): per
 // q-head M = max over blocks, Z = sum_blocks s_i 2^(m_i - M); mass_i =
-// (1 / g) sum_h s_hi 2^(m_hi - M_h) / Z_h.  Every sum runs in a fixed order,
-// so results are bitwise reproducible.
+// (1 / g) sum_h s_hi 2^(m_hi - M_h) / Z_h, one warp per q-head for M and Z.
+// Every sum runs in a fixed order, so results are bitwise reproducible.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -109,38 +109,25 @@ __global__ void __launch_bounds__(kMassThreads) block_mass_kernel(const __grid_c
   }
 }
 
-// Block-wide reduction in a fixed order (warp butterfly, then the warps' results in order).
-template <bool MAX>
-__device__ __forceinline__ float block_reduce(float v, float* scratch) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float w = __shfl_xor_sync(kFull, v, o);
-    v = MAX ? fmaxf(v, w) : v + w;
-  }
-  const int warp = threadIdx.x >> 5;
-  __syncthreads();  // scratch free from the previous reduction
-  if ((threadIdx.x & 31) == 0) scratch[warp] = v;
-  __syncthreads();
-  float r = scratch[0];
-  for (int w = 1; w < kCombineThreads / 32; ++w) r = MAX ? fmaxf(r, scratch[w]) : r + scratch[w];
-  return r;
-}
-
-__global__ void __launch_bounds__(kCombineThreads) block_mass_combine_kernel(const __grid_constant__ BlockMassLaunch a) {
-  __shared__ float scratch[kCombineThreads / 32];
+__global__ void __launch_bounds__(kCombineThreads)
+    block_mass_combine_kernel(const __grid_constant__ BlockMassLaunch a) {
+  // one warp per q-head of the group (two for G > 8): its maximum and sum over the blocks by
+  // lane-strided loops and a fixed butterfly, no block-wide barrier per head
   __shared__ float s_max[16], s_inv[16];
   const int bk = blockIdx.x, b = bk / a.Hkv, kv = bk % a.Hkv;
   const int L = a.L[b], nb = (L + kMassBlock - 1) / kMassBlock;
-  const int G = a.G;
-  for (int h = 0; h < G; ++h) {
+  const int G = a.G, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int h = warp; h < G; h += kCombineThreads / 32) {
     const int64_t row = (int64_t(b) * a.Hq + kv * G + h) * a.nb_max;
     float m = -INFINITY;
-    for (int i = threadIdx.x; i < nb; i += kCombineThreads) m = fmaxf(m, a.ws_m[row + i]);
-    const float M = block_reduce<true>(m, scratch);
+    for (int i = lane; i < nb; i += 32) m = fmaxf(m, a.ws_m[row + i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
     float z = 0.f;
-    for (int i = threadIdx.x; i < nb; i += kCombineThreads) z += a.ws_s[row + i] * exp2f(a.ws_m[row + i] - M);
-    const float Z = block_reduce<false>(z, scratch);
-    if (threadIdx.x == 0) s_max[h] = M, s_inv[h] = 1.f / Z;
+    for (int i = lane; i < nb; i += 32) z += a.ws_s[row + i] * exp2f(a.ws_m[row + i] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(kFull, z, o);
+    if (lane == 0) s_max[h] = m, s_inv[h] = 1.f / z;
   }
   __syncthreads();
   float* out = a.mass + int64_t(bk) * a.mass_stride;
@@ -225,7 +212,8 @@ extern "C" sp_status segpaged_block_mass(const sp_problem* problem, const void* 
   sp_status st = mass_shape(problem, G, nb_max);
   if (st != SP_OK) return st;
   auto al = [](const void* ptr, uintptr_t n) { return (reinterpret_cast<uintptr_t>(ptr) % n) == 0; };
-  if (!k_dense || !q || !mass || !workspace) return fail(SP_ERR_INVALID_ARG, "k_dense, q, mass and workspace must be non-NULL");
+  if (!k_dense || !q || !mass || !workspace)
+    return fail(SP_ERR_INVALID_ARG, "k_dense, q, mass and workspace must be non-NULL");
   if (!al(k_dense, 16) || !al(q, 16) || !al(mass, 4) || !al(workspace, 256))
     return fail(SP_ERR_INVALID_ARG, "k_dense and q must be 16-byte aligned, mass 4-byte, workspace 256-byte");
   if (stride_seq < 0 || stride_head < 0 || stride_tok < 0 || stride_seq % 8 || stride_head % 8 || stride_tok % 8)
@@ -252,5 +240,6 @@ extern "C" sp_status segpaged_block_mass(const sp_problem* problem, const void* 
   a.mass = mass, a.mass_stride = mass_stride;
   for (int b = 0; b < a.B; ++b) a.L[b] = problem->ctx_len[b];
   const cudaError_t e = launch_block_mass(a, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SP_OK : fail(SP_ERR_CUDA, std::string("segpaged_block_mass launch: ") + cudaGetErrorString(e));
+  return e == cudaSuccess ? SP_OK
+                          : fail(SP_ERR_CUDA, std::string("segpaged_block_mass launch: ") + cudaGetErrorString(e));
 }
