@@ -395,3 +395,19 @@ def test_block_mass_argument_checks():
         args = list(good)
         args[i] = bad
         assert S.segpaged_block_mass_status(p, *args) == code, (i, bad, S.last_error())
+
+
+def test_runtime_block_mass_rejects_bad_tensors():
+    """runtime.block_mass checks dtypes, shapes and lengths before it reaches the library."""
+    import torch
+
+    from head_aware_paged_build_b200.runtime import block_mass
+
+    k = torch.zeros(2, 2, 128, 64, dtype=torch.bfloat16)
+    q = torch.zeros(2, 8, 64, dtype=torch.bfloat16)
+    for kk, qq, lens in ((k.float(), q, [128, 100]), (k, q.float(), [128, 100]),   # dtypes
+                         (k, q[:, :7], [128, 100]),                                 # Hq not a multiple of Hkv
+                         (k, q[:, :, :32], [128, 100]),                             # head_dim mismatch
+                         (k, q, [129, 100]), (k, q, [0, 100]), (k, q, [128])):      # lengths
+        with pytest.raises(ValueError):
+            block_mass(kk, qq, lens)
