@@ -69,3 +69,60 @@ def test_block_mass_reads_any_key_layout():
     m = block_mass(tok_major, q, lens)
     assert torch.equal(m, block_mass(k, q, lens))
     _check(m, k, q, lens, 2)
+
+
+def test_gpu_scores_choose_the_oracles_blocks():
+    """Scoring on the GPU, top-p selection by the planner, attention on the GPU, against the oracle's
+    own scoring and selection from the same keys and queries.
+
+    For each sequence's retrieval head, top_p sits halfway between two steps of the oracle's
+    cumulative block mass where the blocks on either side differ by more than 1 %, so the GPU's
+    masses (within 2e-4 of the oracle's) pick the same blocks: the plan's stored positions must
+    equal the oracle's, and the decode output must match the oracle's attention over them.
+    """
+    import numpy as np
+
+    from head_aware_paged_build_b200.runtime import layer_for
+    from test_retrieval_plan import _held
+
+    lens, B, hq, hkv, d, g = (3000, 4500), 2, 8, 2, 128, 4
+    pol = [("retrieval", 4, 256, 1.0), ("local", 4, 256)] * B
+    wl0 = W.custom("score_select", 13, B, hq, hkv, d, "bf16", 64, lens, pol)
+    k, v = W.dense_kv(wl0.decode_problem(), device="cuda", gen_device="cuda")
+    q = W.queries(wl0.decode_problem(), device="cuda", gen_device="cuda")
+    kh, vh, qh = k.cpu().double().numpy(), v.cpu().double().numpy(), q.cpu().double().numpy()
+    sels = {}
+    for b, L in enumerate(lens):
+        om = oracle.block_mass(qh[b, :g], kh[b, 0, :L], 64)  # kv-head 0 is the retrieval head
+        srt = np.sort(om)[::-1]
+        cum = np.cumsum(srt) / srt.sum()
+        gap = (srt[:-1] - srt[1:]) / srt[:-1]  # gap[i]: the (i+1)-th largest mass vs the (i+2)-th
+        # keep c blocks: top_p halfway between the shares of the top c - 1 and the top c blocks,
+        # with the c-th and (c+1)-th largest masses more than 1 % apart
+        c = next(c for c in range(5, len(srt) - 1) if gap[c - 1] > 0.01 and cum[c - 1] < 0.9)
+        top_p = float(np.float32((cum[c - 2] + cum[c - 1]) / 2))
+        pol[b * hkv] = ("retrieval", 4, 256, top_p)
+        sels[b] = oracle.retrieval_select(L, 64, 4, top_p, om.astype(np.float32))
+        assert sels[b].sum() == c
+    wl = W.custom("score_select", 13, B, hq, hkv, d, "bf16", 64, lens, pol)  # same draws, chosen top_p
+    prob = wl.decode_problem()
+    m = block_mass(k, q, lens)
+    masses = [m[b, kv, :-(-L // 64)].tolist() if kv == 0 else None for b, L in enumerate(lens) for kv in range(hkv)]
+    layer = layer_for(prob, block_mass=masses)
+    layer.build(k, v)
+    out, _ = layer.attention(q)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    out = out.float().cpu().double().numpy()
+    for b, L in enumerate(lens):
+        held = _held(layer.plan, b, 0, L)
+        assert np.array_equal(held, oracle.stored_mask("retrieval", 4, 256, L, L - 1, sel=sels[b], block=64)), b
+        for h in range(hq):
+            kv = h // g
+            kind, s, w = pol[b * hkv + kv][:3]
+            extra = dict(sel=sels[b], block=64) if kind == "retrieval" else {}
+            ref, _ = oracle.attention_rows(qh[b, h][None], np.array([L - 1]), kh[b, kv, :L], vh[b, kv, :L], kind, s, w,
+                                           **extra)
+            o = out[b, h][None]
+            cos = float((o * ref).sum() / (np.linalg.norm(o) * np.linalg.norm(ref)))
+            assert cos >= 0.99998 and float(np.abs(o - ref).max()) <= 2e-2, (b, h, cos)
