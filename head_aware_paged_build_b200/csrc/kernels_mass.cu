@@ -190,6 +190,8 @@ sp_status mass_shape(const sp_problem* p, int32_t& G, int32_t& nb_max) {
   if (p->page_size != kMassBlock) return fail(SP_ERR_UNSUPPORTED, "segpaged_block_mass: page_size must be 64");
   if (p->num_q_heads % p->num_kv_heads != 0 || p->num_q_heads / p->num_kv_heads > 16)
     return fail(SP_ERR_UNSUPPORTED, "num_q_heads must be a multiple of num_kv_heads, at most 16 times it");
+  if (int64_t(p->batch) * p->num_kv_heads > 65535)  // the pass's grid.y
+    return fail(SP_ERR_UNSUPPORTED, "segpaged_block_mass: batch * num_kv_heads above 65535");
   if (!p->ctx_len) return fail(SP_ERR_INVALID_ARG, "ctx_len is NULL");
   int64_t lmax = 0;
   for (int b = 0; b < p->batch; ++b) {

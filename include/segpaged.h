@@ -462,7 +462,8 @@ SP_API sp_status segpaged_clear_device_status(void* workspace, void* stream);
  *   problem   host; only batch, num_q_heads, num_kv_heads, head_dim,
  *             page_size, dtype and ctx_len are read.  bf16 only, page_size 64,
  *             head_dim 64 or 128, g = num_q_heads / num_kv_heads <= 16,
- *             batch <= 2048 (else SP_ERR_UNSUPPORTED); ctx_len[b] >= 1.
+ *             batch <= 2048, batch * num_kv_heads <= 65535 (else
+ *             SP_ERR_UNSUPPORTED); ctx_len[b] >= 1.
  *   k_dense   device bf16 keys, element strides stride_seq, stride_head,
  *             stride_tok (multiples of 8, head_dim contiguous), 16-byte aligned
  *             (the layout build_segpaged_cache reads)

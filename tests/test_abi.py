@@ -379,6 +379,10 @@ def test_block_mass_argument_checks():
                      (dict(head_dim=96), S.SP_ERR_UNSUPPORTED),
                      (dict(num_q_heads=34, num_kv_heads=2, policy=[("global", 0, 0)] * 4), S.SP_ERR_UNSUPPORTED),
                      (dict(num_q_heads=7), S.SP_ERR_UNSUPPORTED),
+                     (dict(batch=1100, num_q_heads=64, num_kv_heads=64, ctx_len=[64] * 1100, q_start=[63] * 1100,
+                           policy=[("global", 0, 0)] * (1100 * 64)), S.SP_ERR_UNSUPPORTED),  # grid limit
+                     (dict(batch=2049, ctx_len=[64] * 2049, q_start=[63] * 2049,
+                           policy=[("global", 0, 0)] * (2049 * 2)), S.SP_ERR_UNSUPPORTED),  # batch limit
                      (dict(ctx_len=[700, 0]), S.SP_ERR_INVALID_ARG)):
         assert S.load().segpaged_block_mass_workspace(ctypes.byref(prob(**kw)), ctypes.byref(n)) == code, kw
     p = prob()
