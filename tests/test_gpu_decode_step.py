@@ -95,17 +95,22 @@ def test_decode_step_ring_without_room_reports_like_the_append():
     assert torch.equal(a.table, b.table) and torch.equal(a.k_pool, b.k_pool)
 
 
-def test_decode_step_graph_fused_equals_unfused():
+@pytest.mark.parametrize("kv_dtype", [None, "e4m3"])
+def test_decode_step_graph_fused_equals_unfused(kv_dtype):
     """The serving step captured in a CUDA graph, fused and unfused, on the 32K layer at the bench's
-    batch of 8: outputs every step, and pools and tables at the end, bit for bit."""
+    batch of 8 (bf16 and E4M3 pages): outputs every step, and pools and tables at the end, bit for bit."""
     wl = W.llama()
     n = 6
     dec = wl.decode_problem()
     start = W.Problem(wl, tuple(L - n for L in dec.ctx_lens), tuple(L - n - 1 for L in dec.ctx_lens))
     k, v = W.dense_kv(dec, device="cuda", gen_device="cuda")
+    kw = {}
+    if kv_dtype:
+        kw = dict(kv_dtype=kv_dtype, k_scale=float(k.float().abs().max()) / 448,
+                  v_scale=float(v.float().abs().max()) / 448)
     steps, layers = [], []
     for fused in (True, False):
-        layer = layer_for(start, flags=S.SP_FLAG_RING, append_capacity=n)
+        layer = layer_for(start, flags=S.SP_FLAG_RING, append_capacity=n, **kw)
         layer.build(k, v)
         g = DecodeStepGraph(layer, fused=fused)
         outs = []
