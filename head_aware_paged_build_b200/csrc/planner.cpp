@@ -29,7 +29,7 @@ sp_status fail(sp_status st, const std::string& msg) {
 namespace {
 
 constexpr int kDefaultDecodeCtas = 2 * 148;
-constexpr int64_t kItemCostPages100 = 200;  // a head start costs as much as two pages (measured)
+constexpr int64_t kItemCostPages100 = 350;  // a head start costs about 3.5 pages (measured)
 constexpr int32_t kMergeOneLevel = 16;      // split heads with more items merge in two levels
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -412,7 +412,7 @@ sp_status plan_build(sp_plan& pl) {
   if (decode) {
     const int64_t G = std::min<int64_t>(p.target_ctas ? p.target_ctas : kDefaultDecodeCtas, n_pages);
     // A CTA pays for every head it starts (Q load, warp merge, partial publish) on
-    // top of its pages: cut the page list at equal shares of (pages + two pages
+    // top of its pages: cut the page list at equal shares of (pages + 3.5 pages
     // per head start), so CTAs that cross a head boundary take fewer pages.
     // Costs are in hundredths of a page.
     std::vector<int64_t> cost(n_pages + 1, 0);  // cost of pages [0, i)

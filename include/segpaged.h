@@ -124,8 +124,8 @@ typedef struct {
  *               reported by segpaged_plan_sizes of a plan made with NULL
  *   target_ctas decode work is split into this many CTAs (at most one per
  *               page): contiguous ranges of the heads' concatenated page
- *               lists, balanced on pages plus a two-page cost for each head
- *               a range starts; 0 picks 2 x 148 (two CTAs on each B200 SM).
+ *               lists, balanced on pages plus a cost of 3.5 pages for each
+ *               head a range starts; 0 picks 2 x 148 (two CTAs on each B200 SM).
  *               A CTA whose share is below one head start's cost can be left
  *               without work; it exits at once
  *   append_capacity  SP_FLAG_RING plans: extra tokens per sequence that
