@@ -7,13 +7,16 @@ flushed (256 MB written, then 512 MB read so no dirty line is written back
 inside a timed kernel) before every timed kernel; each kernel is timed with
 CUDA events on the stream it is launched on.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama|mistral|mha|ragged]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama|mistral|mha|ragged|llama_b1]
     python bench.py --impl reference ...   # the CPU oracle, timed on the host cores
 
 Under torchrun each rank runs its own batch (a different seed) on its own GPU:
 weak scaling with no collective on the data path; the timing is the max over
 ranks.  `value` is the decode visible-KV throughput; prefill TFLOP/s, the
-packing rate and the dense-plus-mask variant are reported beside it.
+packing rate and the dense-plus-mask variant are reported beside it, with the
+serving decode step through the public API with pinned host buffers (`e2e`),
+E4M3 pages, and, on the Llama-shaped layers, a layer with retrieval heads
+(decode, prefill and the scoring pass that gives them their importance).
 """
 from __future__ import annotations
 
