@@ -477,8 +477,9 @@ SP_API sp_status segpaged_clear_device_status(void* workspace, void* stream);
  *             segpaged_block_mass_workspace gives (SP_ERR_WORKSPACE if smaller);
  *             fully overwritten, no zeroing needed
  * Two launches on `stream` (a pass over the keys, one warp per block, then a
- * per (sequence, kv-head) normalisation); fixed summation orders, so the
- * result is bitwise reproducible.  Argument errors are reported before any
+ * per (sequence, kv-head) normalisation, launched as a programmatic dependent
+ * of the pass: it is placed while the pass ends and waits for it on the
+ * device); fixed summation orders, so the result is bitwise reproducible.  Argument errors are reported before any
  * launch.  Calls from several host threads are serialised on the host. */
 SP_API sp_status segpaged_block_mass_workspace(const sp_problem* problem, size_t* bytes);
 SP_API sp_status segpaged_block_mass(const sp_problem* problem, const void* k_dense, int64_t stride_seq,
