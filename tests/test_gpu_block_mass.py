@@ -5,7 +5,8 @@ the same keys and queries: every entry within 2e-4 relative + 1e-7 absolute
 (fp32 scores of bf16 products, fp32 sums), rows summing to 1, zeros after a
 row's blocks.  Shapes: the Llama-70B-shaped 32K layer at batch 8, head_dim 64
 with 16 q-heads per kv-head, one q-head per kv-head, ragged lengths (1, one
-block, one position past a block, a partial last block), keys read through
+block, one position past a block, a partial last block), contexts past 512
+blocks (the normalisation then takes a row in several passes), keys read through
 a [B, L, Hkv, d] layout; repeated calls are bitwise equal.
 """
 from __future__ import annotations
@@ -51,6 +52,7 @@ def _check(m, k, q, lens, hkv):
     ("mass_d64_g16", 2, 32, 2, 64, (4000, 1500)),
     ("mass_mha", 2, 4, 4, 128, (3000, 700)),
     ("mass_ragged", 5, 16, 4, 128, (1, 64, 65, 130, 1999)),
+    ("mass_long", 2, 8, 2, 128, (40000, 70001)),  # rows of more than 512 blocks
 ])
 def test_block_mass_matches_oracle(name, B, hq, hkv, d, lens):
     wl, k, q = _inputs(name, 11, B, hq, hkv, d, lens)
