@@ -45,6 +45,8 @@ MUTANTS = {
                                  "mass[(j > 0 ? j - 1 : 0) / block] += a[j] / z / (double)g;"),
     "block_mass_scale_dropped": ("a[j] = scale * acc;", "a[j] = acc;"),
     "block_mass_rotated_dims": ("acc += qh[t] * k[j * d + t];", "acc += qh[t] * k[j * d + (t + 1) % d];"),
+    "block_mass_base_two": ("a[j] = exp(a[j] - m);", "a[j] = exp2(a[j] - m);"),
+    "block_mass_first_query_only": ("const double* qh = q + h * d;", "const double* qh = q;"),
     # FP8 E4M3 encoder / decoder
     "e4m3_bias_8": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
     "e4m3_subnormal_step": ("ldexp((double)m, -9)", "ldexp((double)m, -10)"),
